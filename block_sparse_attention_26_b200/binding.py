@@ -1,0 +1,205 @@
+"""ctypes binding of libbsa.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls and takes
+torch tensors (device memory) in place of raw pointers.  No step of the
+method runs in Python; if the shared library cannot be loaded, importing this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbsa.so")
+
+BSA_OK = 0
+BSA_ERR_INVALID_ARG = 1
+BSA_ERR_UNSUPPORTED = 2
+BSA_ERR_CAPACITY = 3
+BSA_ERR_WORKSPACE = 4
+BSA_ERR_CUDA = 5
+BSA_ERR_DEVICE = 6
+
+BSA_DT_BF16, BSA_DT_F32 = 0, 1
+BSA_SOL, BSA_SLA = 0, 1
+
+
+class bsa_params(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("stride_b", ctypes.c_int64), ("stride_n", ctypes.c_int64), ("stride_h", ctypes.c_int64),
+        ("dtype", ctypes.c_int32), ("method", ctypes.c_int32),
+        ("q_block", ctypes.c_int32), ("k_block", ctypes.c_int32),
+        ("tau", ctypes.c_double), ("keep_percent", ctypes.c_double),
+        ("sink_blocks", ctypes.c_int32), ("keep_diag", ctypes.c_int32),
+        ("prefix_len", ctypes.c_int32),
+        ("dense_row_begin", ctypes.c_int32), ("dense_row_end", ctypes.c_int32),
+        ("extra_tokens", ctypes.c_int32), ("centroid", ctypes.c_int32),
+    ]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: status {status} ({msg})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libbsa.so not built at {LIB_PATH}; run block_sparse_attention_26_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    PP = ctypes.POINTER(bsa_params)
+    lib.bsa_default_params.argtypes = [PP, I32]
+    lib.bsa_default_params.restype = None
+    lib.bsa_workspace_size.argtypes = [PP, ctypes.POINTER(SZ), ctypes.POINTER(I64)]
+    lib.bsa_pool.argtypes = [PP, P, P, P, P, P, P, P, P]
+    lib.bsa_select.argtypes = [PP, P, P, P, P, P, I64, P, P, P, P, SZ, P]
+    lib.bsa_attention.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    lib.bsa_dense_ref_rows.argtypes = [PP, P, P, P, I32, I32, P, P, P, SZ, P]
+    lib.bsa_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
+    lib.bsa_status_string.argtypes = [I32]
+    lib.bsa_status_string.restype = ctypes.c_char_p
+    lib.bsa_last_error.argtypes = []
+    lib.bsa_last_error.restype = ctypes.c_char_p
+    for f in ("bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_attention", "bsa_dense_ref_rows",
+              "bsa_device_status"):
+        getattr(lib, f).restype = I32
+    return lib
+
+
+lib = _load()
+
+EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_attention",
+            "bsa_dense_ref_rows", "bsa_device_status", "bsa_status_string", "bsa_last_error")
+
+
+def _check(status: int, where: str):
+    if status != BSA_OK:
+        msg = lib.bsa_last_error().decode() or lib.bsa_status_string(status).decode()
+        raise BsaError(status, where, msg)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ------------------------------------------------------------------ params
+
+def make_params(q: torch.Tensor, method: str = "sol", *, q_block: Optional[int] = None,
+                tau: float = 1.3, keep_percent: float = 10.0, sink_blocks: int = 1,
+                keep_diag: int = 1, prefix_len: int = 0, dense_rows=(0, 0), extra_tokens: int = 0,
+                centroid: Optional[int] = None) -> bsa_params:
+    """Parameters for a [B, N, H, d] query tensor `q` (strides taken from q)."""
+    m = {"sol": BSA_SOL, "sla": BSA_SLA}[method]
+    p = bsa_params()
+    lib.bsa_default_params(ctypes.byref(p), m)
+    B, N, H, d = q.shape
+    p.B, p.H, p.N, p.d = B, H, N, d
+    p.stride_b, p.stride_n, p.stride_h = q.stride(0), q.stride(1), q.stride(2)
+    p.dtype = {torch.bfloat16: BSA_DT_BF16, torch.float32: BSA_DT_F32}[q.dtype]
+    if q_block is not None:
+        p.q_block = q_block
+    p.tau = float(tau)
+    p.keep_percent = float(keep_percent)
+    p.sink_blocks, p.keep_diag, p.prefix_len = sink_blocks, keep_diag, prefix_len
+    p.dense_row_begin, p.dense_row_end = dense_rows
+    p.extra_tokens = extra_tokens
+    if centroid is not None:
+        p.centroid = centroid
+    return p
+
+
+def dims(p: bsa_params):
+    nQB = -(-p.N // p.q_block)
+    nKB = -(-p.N // p.k_block)
+    return nQB, nKB, p.B * p.H * nQB
+
+
+# ------------------------------------------------------------------ entry points
+
+def bsa_workspace_size(p: bsa_params):
+    nbytes, nnz = ctypes.c_size_t(), ctypes.c_int64()
+    _check(lib.bsa_workspace_size(ctypes.byref(p), ctypes.byref(nbytes), ctypes.byref(nnz)),
+           "bsa_workspace_size")
+    return nbytes.value, nnz.value
+
+
+def bsa_pool(p, q, k, v, qbar, kbar, vbar, blk_count, stream=None):
+    _check(lib.bsa_pool(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(qbar), _ptr(kbar), _ptr(vbar),
+                        _ptr(blk_count), _stream(stream)), "bsa_pool")
+
+
+def bsa_select(p, qbar, kbar, k, row_ptr, col_idx, kept_count, extra_idx, extra_count, ws,
+               stream=None):
+    cap = 0 if col_idx is None else col_idx.numel()
+    _check(lib.bsa_select(ctypes.byref(p), _ptr(qbar), _ptr(kbar), _ptr(k), _ptr(row_ptr), _ptr(col_idx),
+                          cap, _ptr(kept_count), _ptr(extra_idx), _ptr(extra_count), _ptr(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)), "bsa_select")
+
+
+def bsa_attention(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra_idx, extra_count, out,
+                  lse, ws, stream=None):
+    _check(lib.bsa_attention(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vbar),
+                             _ptr(blk_count), _ptr(row_ptr), _ptr(col_idx), _ptr(extra_idx),
+                             _ptr(extra_count), _ptr(out), _ptr(lse), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream(stream)), "bsa_attention")
+
+
+def bsa_dense_ref_rows(p, q, k, v, row_begin, row_end, out, lse, ws, stream=None):
+    _check(lib.bsa_dense_ref_rows(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), int(row_begin),
+                                  int(row_end), _ptr(out), _ptr(lse), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)),
+           "bsa_dense_ref_rows")
+
+
+def bsa_device_status(ws, stream=None) -> int:
+    code = ctypes.c_int32()
+    _check(lib.bsa_device_status(_ptr(ws), _stream(stream), ctypes.byref(code)), "bsa_device_status")
+    return code.value
+
+
+# ------------------------------------------------------------------ buffers
+
+class Buffers:
+    """Device buffers for one layer of a given parameter set (allocated by torch)."""
+
+    def __init__(self, p: bsa_params, device, capacity: Optional[int] = None):
+        nQB, nKB, rows = dims(p)
+        BH, d = p.B * p.H, p.d
+        f32, i32 = torch.float32, torch.int32
+        self.qbar = torch.empty((p.B, p.H, nQB, d), dtype=f32, device=device)
+        self.kbar = torch.empty((p.B, p.H, nKB, d), dtype=f32, device=device)
+        self.vbar = torch.empty((p.B, p.H, nKB, d), dtype=f32, device=device)
+        self.blk_count = torch.empty((nKB,), dtype=i32, device=device)
+        self.row_ptr = torch.empty((rows + 1,), dtype=torch.int64, device=device)
+        ws_bytes, max_nnz = bsa_workspace_size(p)
+        if capacity is None:
+            capacity = max_nnz
+        self.col_idx = torch.empty((max(capacity, 1),), dtype=i32, device=device)
+        self.kept_count = torch.empty((rows,), dtype=i32, device=device)
+        E = p.extra_tokens
+        self.extra_idx = torch.empty((rows, E), dtype=i32, device=device) if E > 0 else None
+        self.extra_count = torch.empty((rows,), dtype=i32, device=device) if E > 0 else None
+        self.ws = torch.zeros((ws_bytes + 255) // 256 * 256, dtype=torch.uint8, device=device)
+        self.lse = torch.empty((p.B, p.H, p.N), dtype=f32, device=device)
+        del BH
+
+
+def run_layer(p: bsa_params, q, k, v, out, buf: Buffers, stream=None, lse: bool = True):
+    """The whole hot path for one layer: pool -> select -> attention (+ dense rows)."""
+    bsa_pool(p, q, k, v, buf.qbar, buf.kbar, buf.vbar, buf.blk_count, stream)
+    bsa_select(p, buf.qbar, buf.kbar, k, buf.row_ptr, buf.col_idx, buf.kept_count, buf.extra_idx,
+               buf.extra_count, buf.ws, stream)
+    bsa_attention(p, q, k, v, buf.kbar, buf.vbar, buf.blk_count, buf.row_ptr, buf.col_idx,
+                  buf.extra_idx, buf.extra_count, out, buf.lse if lse else None, buf.ws, stream)

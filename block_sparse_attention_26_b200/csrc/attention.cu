@@ -1,0 +1,656 @@
+// attention.cu -- step 3: the fine pass (exact kept blocks + centroids, one
+// FP32 online softmax) and the dense rows.
+//
+// "minimax-h3-chunk-star7" README, section "Sol": selected K/V blocks are
+// computed exactly; unselected blocks are not dropped but contribute through
+// their K/V centroids, merged into the same FP32 online softmax.  Section
+// "SLA": only the routed K/V blocks take part; softmax state and the final
+// accumulation stay FP32.  "BlockSparseAttention - ComfyUI Built-in Node
+// Documentation", general inputs, sink_conditioning: exact_kv (the packed
+// prefix blocks arrive here as kept blocks) and exact_kv_and_rows (designated
+// query rows run dense and replace the sparse result).
+//
+// One CTA computes a tile of 128 query rows of one (batch, head): two 64-row
+// query blocks (Sol, Q64) or one 128-row block (SLA, Q128), so that every
+// tensor-core instruction is a full M = 128 UMMA.  The tile walks the sorted
+// union of its query blocks' kept key blocks, then the centroid chunks; a
+// per-tile row mask tells each row whether a tile is its own.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S from
+//              TMEM, masks, online softmax in the log2 domain with a lazily
+//              updated reference max, writes P (bf16) to shared memory, rescales
+//              the TMEM accumulator only when the max grows by > 2^8, and runs
+//              the epilogue O / l -> global.
+//   warp 4     producer: builds the tile list and issues TMA tile loads of K/V
+//              (or of bf16 centroid tiles) into a 3-stage ring.
+//   warp 5     MMA issuer: S = Q K^T (M=128, N=64) into one of two TMEM
+//              S buffers; O += P V (M=128, N=d) into the TMEM accumulator.
+// TMEM: columns [0,64) and [64,128) hold the two S buffers, [128, 128+d) hold O.
+#include <math.h>
+
+#include <algorithm>
+
+#include "bsa_device.cuh"
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+constexpr int kM = 128;        // query rows per tile (UMMA M)
+constexpr int kBK = 64;        // keys per tile (one key block)
+constexpr int kStages = 3;     // K/V ring depth
+constexpr int kThreads = 192;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kTmemCols = 256;
+
+enum : int32_t { TILE_EXACT = 0, TILE_CENT = 1, TILE_END = 2 };
+
+struct TileInfo {
+    int32_t kind;
+    int32_t blk;          // key block (exact) or centroid chunk of 64 blocks (centroid)
+    uint32_t who;         // exact: bit q set = query block q of the tile keeps the block
+    int32_t ncols;        // exact: valid key columns; centroid: column of a partial block or -1
+    float last_bias;      // centroid: log2 of the partial block's size
+    int32_t pad[3];
+    uint64_t cmask[2];    // centroid: active centroid columns for query block 0 / 1
+};
+
+struct AttnArgs {
+    int B, H, N, nQB, nKB, nW, Bq;
+    int64_t sb, sn, sh;          // output element strides
+    const int64_t *row_ptr;
+    const int32_t *col_idx;
+    void *out;
+    float *lse;
+    int out_f32;
+    int centroid;
+    int dense;                   // 1: rows [row_begin, row_end) over all key blocks
+    int row_begin, row_end;      // dense: rows computed; sparse: rows left to the dense pass
+    float scale_log2;            // log2(e) / sqrt(d)
+    int32_t *status;
+};
+
+template <int D>
+struct Lay {
+    static constexpr int kQBytes = kM * D * 2;
+    static constexpr int kKVBytes = kBK * D * 2;
+    static constexpr int kPBytes = kM * kBK * 2;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kStages * kKVBytes;
+    static constexpr int kOffP = kOffV + kStages * kKVBytes;
+    static constexpr int kOffInfo = kOffP + 2 * kPBytes;
+    static constexpr int kOffBar = kOffInfo + kStages * (int)sizeof(TileInfo);
+    // q, done, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], p_free[2]
+    static constexpr int kNumBar = 2 + 2 * kStages + 8;
+    static constexpr int kOffMisc = kOffBar + kNumBar * 8;
+    static constexpr int kOffMask = kOffMisc + 16;
+    static size_t bytes(int nW) { return (size_t)kOffMask + 2 * (size_t)nW * 4 + 1024; }
+};
+
+// 2^x on the MUFU unit (ex2.approx, relative error ~2^-22; 2^-inf = +0).
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
+                const __grid_constant__ CUtensorMap tm_vc, const AttnArgs a)
+{
+    using L = Lay<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~(uintptr_t)1023);
+    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    int row0, row_end;
+    if (a.dense) {
+        row0 = a.row_begin + tile * kM;
+        row_end = a.row_end;
+    } else {
+        row0 = tile * kM;
+        row_end = a.N;
+        if (row0 >= a.row_begin && min(row0 + kM, a.N) <= a.row_end) return;   // all rows dense
+    }
+    const int nvalid = min(kM, row_end - row0);
+    if (nvalid <= 0) return;
+    const int qb0 = row0 / a.Bq;
+    const int nq = a.dense ? 1 : ((a.Bq == 64 && qb0 + 1 < a.nQB) ? 2 : 1);
+    const int64_t rbase = ((int64_t)b * a.H + h) * a.nQB + qb0;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kOffBar);
+    uint64_t *bar_q = bars, *bar_done = bars + 1;
+    uint64_t *kv_full = bars + 2, *kv_empty = bars + 2 + kStages;
+    uint64_t *s_full = bars + 2 + 2 * kStages, *s_free = s_full + 2, *p_full = s_full + 4,
+             *p_free = s_full + 6;
+    volatile TileInfo *info = reinterpret_cast<volatile TileInfo *>(sm + L::kOffInfo);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kOffMisc);
+    volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(sm + L::kOffMisc + 4);
+    uint32_t *kept = reinterpret_cast<uint32_t *>(sm + L::kOffMask);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        mbar_init(bar_done, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 4);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&p_free[i], 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 4 && !a.dense) {
+        // kept-block bitmasks of the tile's query blocks, from the CSR lists
+        for (int w = lane; w < 2 * a.nW; w += 32) kept[w] = 0u;
+        __syncwarp();
+        for (int q = 0; q < nq; ++q) {
+            const int64_t p0 = a.row_ptr[rbase + q], p1 = a.row_ptr[rbase + q + 1];
+            for (int64_t p = p0 + lane; p < p1; p += 32) {
+                const int c = a.col_idx[p];
+                if (c >= 0 && c < a.nKB)
+                    atomicOr(&kept[q * a.nW + (c >> 5)], 1u << (c & 31));
+                else
+                    report(a.status, BSA_DEV_INTERNAL, 1);
+            }
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_kc);
+            prefetch_tmap(&tm_vc);
+            mbar_expect_tx(bar_q, L::kQBytes);
+            for (int dc = 0; dc < D / 64; ++dc)
+                tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
+            int j = 0;
+            int issued[kStages] = {};
+            bool ok = true;
+            auto push = [&](int kind, int blk, uint32_t who, int ncols, float last_bias, uint64_t m0,
+                            uint64_t m1) -> bool {
+                const int s = j % kStages;
+                if (j >= kStages &&
+                    !mbar_wait(&kv_empty[s], ((j / kStages) - 1) & 1, abort_flag, a.status, 10))
+                    return false;
+                info[s].kind = kind;
+                info[s].blk = blk;
+                info[s].who = who;
+                info[s].ncols = ncols;
+                info[s].last_bias = last_bias;
+                info[s].cmask[0] = m0;
+                info[s].cmask[1] = m1;
+                uint8_t *kd = sm + L::kOffK + s * L::kKVBytes;
+                uint8_t *vd = sm + L::kOffV + s * L::kKVBytes;
+                if (kind == TILE_EXACT) {
+                    mbar_expect_tx(&kv_full[s], 2 * L::kKVBytes);
+                    for (int dc = 0; dc < D / 64; ++dc) {
+                        tma_load_4d(kd + dc * (kBK * 128), &tm_k, &kv_full[s], dc * 64, h, blk * kBK, b);
+                        tma_load_4d(vd + dc * (kBK * 128), &tm_v, &kv_full[s], dc * 64, h, blk * kBK, b);
+                    }
+                } else if (kind == TILE_CENT) {
+                    mbar_expect_tx(&kv_full[s], 2 * L::kKVBytes);
+                    const int bh = b * a.H + h;
+                    for (int dc = 0; dc < D / 64; ++dc) {
+                        tma_load_3d(kd + dc * (kBK * 128), &tm_kc, &kv_full[s], dc * 64, blk * kBK, bh);
+                        tma_load_3d(vd + dc * (kBK * 128), &tm_vc, &kv_full[s], dc * 64, blk * kBK, bh);
+                    }
+                } else {
+                    mbar_arrive(&kv_full[s]);
+                }
+                issued[s]++;
+                ++j;
+                return true;
+            };
+            const int last_n = a.N - (a.nKB - 1) * kBK;
+            if (a.dense) {
+                for (int blk = 0; blk < a.nKB && ok; ++blk)
+                    ok = push(TILE_EXACT, blk, 3u, min(kBK, a.N - blk * kBK), 0.f, 0, 0);
+            } else {
+                const uint32_t *k0 = kept, *k1 = kept + a.nW;
+                for (int w = 0; w < a.nW && ok; ++w) {
+                    uint32_t u = k0[w] | k1[w];
+                    while (u && ok) {
+                        const int bit = __ffs(u) - 1;
+                        u &= u - 1;
+                        const int blk = w * 32 + bit;
+                        const uint32_t who = ((k0[w] >> bit) & 1u) | (((k1[w] >> bit) & 1u) << 1);
+                        ok = push(TILE_EXACT, blk, who, min(kBK, a.N - blk * kBK), 0.f, 0, 0);
+                    }
+                }
+                if (a.centroid) {
+                    const int nchunk = (a.nKB + kBK - 1) / kBK;
+                    for (int cc = 0; cc < nchunk && ok; ++cc) {
+                        const int nb = min(kBK, a.nKB - cc * kBK);
+                        const uint64_t valid = nb == 64 ? ~0ull : ((1ull << nb) - 1ull);
+                        auto words = [&](const uint32_t *k) -> uint64_t {
+                            const int w0 = 2 * cc;
+                            const uint64_t lo = w0 < a.nW ? k[w0] : 0u;
+                            const uint64_t hi = w0 + 1 < a.nW ? k[w0 + 1] : 0u;
+                            return lo | (hi << 32);
+                        };
+                        const uint64_t m0 = valid & ~words(k0);
+                        const uint64_t m1 = nq > 1 ? (valid & ~words(k1)) : 0ull;
+                        if ((m0 | m1) == 0ull) continue;
+                        const int lastcol = (a.nKB - 1) - cc * kBK;
+                        const bool partial = last_n < kBK && lastcol < kBK;
+                        ok = push(TILE_CENT, cc, 0u, partial ? lastcol : -1,
+                                  partial ? log2f((float)last_n) : 0.f, m0, m1);
+                    }
+                }
+            }
+            if (ok) ok = push(TILE_END, 0, 0u, 0, 0.f, 0, 0);
+            // make sure no TMA write is still in flight before the CTA can exit
+            for (int s = 0; s < kStages; ++s)
+                if (issued[s] > 0) {
+                    volatile int32_t no_abort = 0;
+                    mbar_wait(&kv_full[s], (issued[s] - 1) & 1, &no_abort, a.status, 11);
+                }
+            volatile int32_t no_abort = 0;
+            mbar_wait(bar_q, 0, &no_abort, a.status, 12);
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(kM, kBK, 0, 0);
+            const uint32_t idesc_o = idesc_bf16_f32(kM, D, 0, 1);
+            const uint32_t q_addr = smem_u32(sm + L::kOffQ);
+            const uint32_t k_addr = smem_u32(sm + L::kOffK);
+            const uint32_t v_addr = smem_u32(sm + L::kOffV);
+            const uint32_t p_addr = smem_u32(sm + L::kOffP);
+            auto issue_pv = [&](int t) -> bool {
+                const int pb = t & 1, s = t % kStages;
+                if (!mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag, a.status, 20)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kBK / 16; ++ks) {
+                    const uint64_t ad = sdesc_sw128(p_addr + pb * L::kPBytes + ks * 32, 16, 1024);
+                    const uint64_t bd =
+                        sdesc_sw128(v_addr + s * L::kKVBytes + ks * 2048, kBK * 128, 1024);
+                    umma_bf16(tmem + 128, ad, bd, idesc_o, (t > 0 || ks > 0) ? 1u : 0u);
+                }
+                umma_commit(&kv_empty[s]);
+                umma_commit(&p_free[pb]);
+                return true;
+            };
+            bool ok = mbar_wait(bar_q, 0, abort_flag, a.status, 21);
+            tc_fence_after();
+            int j = 0;
+            while (ok) {
+                const int s = j % kStages;
+                if (!(ok = mbar_wait(&kv_full[s], (j / kStages) & 1, abort_flag, a.status, 22))) break;
+                tc_fence_after();
+                if (info[s].kind == TILE_END) break;
+                const int sb = j & 1;
+                if (j >= 2 && !(ok = mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, abort_flag, a.status, 23)))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t ad =
+                        sdesc_sw128(q_addr + (ks >> 2) * (kM * 128) + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(
+                        k_addr + s * L::kKVBytes + (ks >> 2) * (kBK * 128) + (ks & 3) * 32, 16, 1024);
+                    umma_bf16(tmem + sb * kBK, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[sb]);
+                if (j >= 1 && !(ok = issue_pv(j - 1))) break;
+                ++j;
+            }
+            if (ok && j >= 1) ok = issue_pv(j - 1);
+            if (ok) umma_commit(&s_full[j & 1]);      // end-of-list marker for the softmax warps
+            // wait for every MMA this thread issued before TMEM can be released
+            umma_commit(bar_done);
+            volatile int32_t no_abort = 0;
+            mbar_wait(bar_done, 0, &no_abort, a.status, 24);
+        }
+    } else {
+        // ---------------------------------------------------------- softmax
+        const int r = threadIdx.x;                               // tile row == TMEM lane
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int qsel = (a.Bq == 64 && !a.dense) ? (r >> 6) : 0;
+        const float scale = a.scale_log2;
+        const uint32_t p_row = smem_u32(sm + L::kOffP) + (r >> 3) * 1024 + (r & 7) * 128;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        int j = 0;
+        for (;; ++j) {
+            const int sb = j & 1, s = j % kStages;
+            ok = mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag, a.status, 30) &&
+                 mbar_wait(&kv_full[s], (j / kStages) & 1, abort_flag, a.status, 31);
+            if (!(ok = __all_sync(0xffffffffu, ok))) break;
+            tc_fence_after();
+            const int kind = info[s].kind;
+            if (kind == TILE_END) break;
+            uint32_t sr[64];
+            tmem_ld32(tmem + lane_base + sb * kBK, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+            tmem_ld32(tmem + lane_base + sb * kBK + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[sb]);
+
+            float x[64];
+            if (kind == TILE_EXACT) {
+                const bool act = (info[s].who >> qsel) & 1u;
+                const int nc = act ? info[s].ncols : 0;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) x[c] = c < nc ? __uint_as_float(sr[c]) * scale : -INFINITY;
+            } else {
+                const uint64_t msk = info[s].cmask[qsel];
+                const int pc = info[s].ncols;
+                const float pbias = info[s].last_bias;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const float bias = c == pc ? pbias : 6.0f;       // log2(64) for full blocks
+                    x[c] = ((msk >> c) & 1ull) ? fmaf(__uint_as_float(sr[c]), scale, bias) : -INFINITY;
+                }
+            }
+            float mt = x[0];
+#pragma unroll
+            for (int c = 1; c < 64; ++c) mt = fmaxf(mt, x[c]);
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mt > m_ref) {
+                if (m_ref == -INFINITY) {
+                    m_ref = mt;
+                } else if (mt > m_ref + kRescaleLog2) {
+                    alpha = ex2(m_ref - mt);
+                    l *= alpha;
+                    m_ref = mt;
+                    rescale = true;
+                }
+            }
+            const float mref = m_ref == -INFINITY ? 0.f : m_ref;
+            uint32_t pk[32];
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const float p0 = ex2(x[2 * c] - mref);
+                const float p1 = ex2(x[2 * c + 1] - mref);
+                rs += p0 + p1;
+                pk[c] = pack_bf16x2(p0, p1);
+            }
+            l += rs;
+            if (j >= 2) {
+                ok = mbar_wait(&p_free[sb], ((j >> 1) - 1) & 1, abort_flag, a.status, 32);
+                if (!(ok = __all_sync(0xffffffffu, ok))) break;
+            }
+            const uint32_t pbase = p_row + sb * L::kPBytes;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(pbase + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                             pk[4 * c + 3]);
+            if (__any_sync(0xffffffffu, rescale)) {
+                // the accumulator must hold every earlier P V product before it is scaled
+                ok = mbar_wait(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status, 33);
+                if (!(ok = __all_sync(0xffffffffu, ok))) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_base + 128 + cc * 32, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tmem + lane_base + 128 + cc * 32, o);
+                }
+                tmem_st_wait();
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[sb]);
+        }
+        const int T = j;
+        if (ok && T >= 1)
+            ok = mbar_wait(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, a.status, 34);
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        if (ok) {
+            const bool row_ok = r < nvalid;
+            const int n = row0 + r;
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const bool have_o = T >= 1 && l > 0.f;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                __syncwarp();
+                tmem_ld32(tmem + lane_base + 128 + cc * 32, o);
+                tmem_ld_wait();
+                if (!row_ok) continue;
+                float v[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = have_o ? __uint_as_float(o[e]) * inv_l : 0.f;
+                const int64_t off = (int64_t)b * a.sb + (int64_t)n * a.sn + (int64_t)h * a.sh + cc * 32;
+                if (a.out_f32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + off);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + off);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]), pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
+                                            pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
+                                            pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+                }
+            }
+            if (row_ok && a.lse != nullptr)
+                a.lse[((int64_t)b * a.H + h) * a.N + n] =
+                    l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// bf16 copies of f32 centroids (or of f32 inputs): elementwise, grid-stride.
+__global__ void to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst, int64_t n)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+// f32 [B, N, H, d] strided -> bf16 contiguous [B, N, H, d].
+__global__ void inputs_to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst,
+                                      int B, int N, int H, int d, int64_t sb, int64_t sn, int64_t sh)
+{
+    const int64_t total = (int64_t)B * N * H * d;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int c = (int)(i % d);
+        const int64_t t = i / d;
+        const int hh = (int)(t % H);
+        const int64_t t2 = t / H;
+        const int n = (int)(t2 % N);
+        const int bb = (int)(t2 / N);
+        dst[i] = __float2bfloat16_rn(src[(int64_t)bb * sb + (int64_t)n * sn + (int64_t)hh * sh + c]);
+    }
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// bf16 [B, N, H, d] with element strides; box = 64 channels x 1 head x rows tokens x 1.
+bool make_map_bnhd(CUtensorMap *m, const void *base, int B, int N, int H, int d, int64_t sb, int64_t sn,
+                   int64_t sh, int rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)sh * 2, (cuuint64_t)sn * 2, (cuuint64_t)sb * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [BH, nKB, d] centroids; box = 64 channels x 64 centroids x 1.
+bool make_map_cent(CUtensorMap *m, const void *base, int BH, int nKB, int d)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)nKB, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)nKB * d * 2};
+    cuuint32_t box[3] = {64, 64, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_attn_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                               const CUtensorMap &tkc, const CUtensorMap &tvc, const AttnArgs &a, int tiles,
+                               cudaStream_t st)
+{
+    const size_t smem = Lay<D>::bytes(a.nW);
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)tiles, (unsigned)a.H, (unsigned)a.B);
+    attn_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attention_smem_bytes(int d, int nW)
+{
+    return d == 64 ? Lay<64>::bytes(nW) : Lay<128>::bytes(nW);
+}
+
+cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, const void *k,
+                             const void *v, const float *kbar, const float *vbar,
+                             const int64_t *row_ptr, const int32_t *col_idx, const int32_t *extra_idx,
+                             const int32_t *extra_count, void *out, float *lse, int dense_only,
+                             int row_begin, int row_end, char *ws, const WsLayout &L, cudaStream_t st)
+{
+    (void)extra_idx;
+    (void)extra_count;
+    const int BH = D.B * D.H;
+    int64_t sb = p.stride_b, sn = p.stride_n, sh = p.stride_h;
+    const void *q16 = q, *k16 = k, *v16 = v;
+    if (p.dtype == BSA_DT_F32) {
+        // the tensor cores take bf16 operands: round the f32 inputs once
+        const int64_t n = (int64_t)D.B * D.N * D.H * D.d;
+        const unsigned g = (unsigned)std::min<int64_t>(ceil_div(n, 256), 148 * 16);
+        __nv_bfloat16 *dq = reinterpret_cast<__nv_bfloat16 *>(ws + L.q16);
+        __nv_bfloat16 *dk = reinterpret_cast<__nv_bfloat16 *>(ws + L.k16);
+        __nv_bfloat16 *dv = reinterpret_cast<__nv_bfloat16 *>(ws + L.v16);
+        inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(q), dq, D.B, D.N, D.H, D.d, sb, sn, sh);
+        inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(k), dk, D.B, D.N, D.H, D.d, sb, sn, sh);
+        inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(v), dv, D.B, D.N, D.H, D.d, sb, sn, sh);
+        q16 = dq;
+        k16 = dk;
+        v16 = dv;
+        sh = D.d;
+        sn = (int64_t)D.H * D.d;
+        sb = (int64_t)D.N * D.H * D.d;
+    }
+    __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(ws + L.kc16);
+    __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(ws + L.vc16);
+    const bool use_cent = !dense_only && p.centroid;
+    if (use_cent) {
+        const int64_t n = (int64_t)BH * D.nKB * D.d;
+        const unsigned g = (unsigned)std::min<int64_t>(ceil_div(n, 256), 148 * 8);
+        to_bf16_kernel<<<g, 256, 0, st>>>(kbar, kc, n);
+        to_bf16_kernel<<<g, 256, 0, st>>>(vbar, vc, n);
+    }
+    CUtensorMap tq, tk, tv, tkc, tvc;
+    if (!make_map_bnhd(&tq, q16, D.B, D.N, D.H, D.d, sb, sn, sh, kM) ||
+        !make_map_bnhd(&tk, k16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) ||
+        !make_map_bnhd(&tv, v16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) ||
+        !make_map_cent(&tkc, kc, BH, D.nKB, D.d) || !make_map_cent(&tvc, vc, BH, D.nKB, D.d)) {
+        set_error("cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)");
+        return cudaErrorInvalidValue;
+    }
+    AttnArgs a;
+    a.B = D.B;
+    a.H = D.H;
+    a.N = D.N;
+    a.nQB = D.nQB;
+    a.nKB = D.nKB;
+    a.nW = D.nW;
+    a.Bq = D.Bq;
+    a.sb = p.stride_b;
+    a.sn = p.stride_n;
+    a.sh = p.stride_h;
+    a.row_ptr = row_ptr;
+    a.col_idx = col_idx;
+    a.out = out;
+    a.lse = lse;
+    a.out_f32 = p.dtype == BSA_DT_F32;
+    a.centroid = p.centroid;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D.d));
+    a.status = reinterpret_cast<int32_t *>(ws + L.status);
+    cudaError_t e = cudaSuccess;
+    if (!dense_only) {
+        a.dense = 0;
+        a.row_begin = p.dense_row_begin;
+        a.row_end = p.dense_row_end;
+        const int tiles = (int)ceil_div(D.N, kM);
+        e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, a, tiles, st)
+                      : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, a, tiles, st);
+        if (e != cudaSuccess) return e;
+    }
+    if (row_end > row_begin) {
+        a.dense = 1;
+        a.row_begin = row_begin;
+        a.row_end = row_end;
+        const int tiles = (int)ceil_div(row_end - row_begin, kM);
+        e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, a, tiles, st)
+                      : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, a, tiles, st);
+    }
+    return e;
+}
+
+}  // namespace bsa

@@ -1,0 +1,298 @@
+// bsa_api.cu -- the extern "C" entry points declared in bsa.h: host-side
+// validation, workspace layout and kernel launches.  No device memory is
+// allocated here; every launch goes to the caller's stream.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "bsa_internal.h"
+
+namespace bsa {
+
+static thread_local char g_err[512] = "";
+
+void set_error(const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+}
+
+Dims dims_of(const bsa_params &p)
+{
+    Dims D;
+    D.B = p.B;
+    D.H = p.H;
+    D.N = p.N;
+    D.d = p.d;
+    D.Bq = p.q_block;
+    D.Bk = p.k_block;
+    D.nQB = (int)ceil_div(p.N, p.q_block);
+    D.nKB = (int)ceil_div(p.N, p.k_block);
+    D.nW = (int)ceil_div(D.nKB, 32);
+    D.rows = (int64_t)p.B * p.H * D.nQB;
+    D.E = p.extra_tokens;
+    return D;
+}
+
+WsLayout ws_layout(const bsa_params &p)
+{
+    const Dims D = dims_of(p);
+    WsLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + bytes, 256);
+        return at;
+    };
+    const int64_t BH = (int64_t)D.B * D.H;
+    L.status = take(sizeof(int32_t) * 2);
+    L.scores = take((size_t)D.rows * D.nKB * sizeof(float));
+    L.bitmask = take((size_t)D.rows * D.nW * sizeof(uint32_t));
+    L.counts = take((size_t)D.rows * sizeof(int32_t));
+    L.kc16 = take((size_t)BH * D.nKB * D.d * 2);
+    L.vc16 = take((size_t)BH * D.nKB * D.d * 2);
+    L.cbias = take(0);
+    L.xk16 = take(0);
+    L.xv16 = take(0);
+    const size_t in16 = p.dtype == BSA_DT_F32 ? (size_t)D.B * D.N * D.H * D.d * 2 : 0;
+    L.q16 = take(in16);
+    L.k16 = take(in16);
+    L.v16 = take(in16);
+    L.total = off;
+    return L;
+}
+
+}  // namespace bsa
+
+using namespace bsa;
+
+namespace {
+
+#define FAIL(code, ...)            \
+    do {                           \
+        set_error(__VA_ARGS__);    \
+        return (code);             \
+    } while (0)
+
+bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+bsa_status check_params(const bsa_params *p)
+{
+    if (p == nullptr) FAIL(BSA_ERR_INVALID_ARG, "params is NULL");
+    if (p->B < 1 || p->H < 1 || p->N < 1) FAIL(BSA_ERR_INVALID_ARG, "B, H, N must be >= 1");
+    if (p->d != 64 && p->d != 128) FAIL(BSA_ERR_UNSUPPORTED, "d = %d; supported head dims are 64 and 128", p->d);
+    if (p->dtype != BSA_DT_BF16 && p->dtype != BSA_DT_F32) FAIL(BSA_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
+    if (p->method != BSA_SOL && p->method != BSA_SLA) FAIL(BSA_ERR_UNSUPPORTED, "unknown method %d", p->method);
+    if (p->k_block != 64) FAIL(BSA_ERR_UNSUPPORTED, "k_block must be 64");
+    if (p->q_block != 64 && p->q_block != 128) FAIL(BSA_ERR_UNSUPPORTED, "q_block must be 64 or 128");
+    const int64_t align_elems = p->dtype == BSA_DT_BF16 ? 8 : 4;
+    if (p->stride_b <= 0 || p->stride_n <= 0 || p->stride_h <= 0)
+        FAIL(BSA_ERR_INVALID_ARG, "strides must be positive");
+    if (p->stride_b % align_elems || p->stride_n % align_elems || p->stride_h % align_elems)
+        FAIL(BSA_ERR_INVALID_ARG, "strides must be multiples of %lld elements (16 bytes)", (long long)align_elems);
+    if (p->stride_h < p->d) FAIL(BSA_ERR_INVALID_ARG, "stride_h smaller than d would overlap heads");
+    if (isnan(p->tau)) FAIL(BSA_ERR_INVALID_ARG, "tau is NaN");
+    if (p->method == BSA_SLA && !(p->keep_percent > 0.0 && p->keep_percent <= 100.0))
+        FAIL(BSA_ERR_INVALID_ARG, "keep_percent must be in (0, 100]");
+    if (p->sink_blocks < 0) FAIL(BSA_ERR_INVALID_ARG, "sink_blocks < 0");
+    if (p->keep_diag != 0 && p->keep_diag != 1) FAIL(BSA_ERR_INVALID_ARG, "keep_diag must be 0 or 1");
+    if (p->prefix_len < 0 || p->prefix_len > p->N) FAIL(BSA_ERR_INVALID_ARG, "prefix_len outside [0, N]");
+    if (p->dense_row_begin < 0 || p->dense_row_end < p->dense_row_begin || p->dense_row_end > p->N)
+        FAIL(BSA_ERR_INVALID_ARG, "dense rows must satisfy 0 <= begin <= end <= N");
+    if (p->extra_tokens < 0 || p->extra_tokens > 256) FAIL(BSA_ERR_INVALID_ARG, "extra_tokens outside [0, 256]");
+    if (p->centroid != 0 && p->centroid != 1) FAIL(BSA_ERR_INVALID_ARG, "centroid must be 0 or 1");
+    const int64_t nKB = ceil_div(p->N, p->k_block);
+    if (nKB > 65536) FAIL(BSA_ERR_UNSUPPORTED, "N too large: at most 65536 key blocks");
+    const int64_t span = (int64_t)(p->B - 1) * p->stride_b + (int64_t)(p->N - 1) * p->stride_n +
+                         (int64_t)(p->H - 1) * p->stride_h + p->d;
+    if (span >= (int64_t)1 << 40) FAIL(BSA_ERR_UNSUPPORTED, "tensor span too large");
+    return BSA_OK;
+}
+
+bsa_status check_ws(const bsa_params *p, void *ws, size_t ws_bytes)
+{
+    if (ws == nullptr) FAIL(BSA_ERR_WORKSPACE, "workspace is NULL");
+    if (!aligned16(ws)) FAIL(BSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    const WsLayout L = ws_layout(*p);
+    if (ws_bytes < L.total)
+        FAIL(BSA_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+    return BSA_OK;
+}
+
+bsa_status check_tensor(const void *t, const char *name)
+{
+    if (t == nullptr) FAIL(BSA_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(t)) FAIL(BSA_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+    return BSA_OK;
+}
+
+bsa_status from_cuda(cudaError_t e, const char *what)
+{
+    if (e == cudaSuccess) return BSA_OK;
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return BSA_ERR_CUDA;
+}
+
+#define TRY(x)                              \
+    do {                                    \
+        const bsa_status _s = (x);          \
+        if (_s != BSA_OK) return _s;        \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+void bsa_default_params(bsa_params *p, int32_t method)
+{
+    if (p == nullptr) return;
+    memset(p, 0, sizeof *p);
+    p->method = method;
+    p->dtype = BSA_DT_BF16;
+    p->k_block = 64;
+    p->q_block = method == BSA_SLA ? 128 : 64;
+    p->tau = 1.3;
+    p->keep_percent = 10.0;
+    p->sink_blocks = 1;
+    p->keep_diag = 1;
+    p->centroid = method == BSA_SLA ? 0 : 1;
+}
+
+bsa_status bsa_workspace_size(const bsa_params *p, size_t *bytes, int64_t *max_nnz)
+{
+    g_err[0] = 0;
+    TRY(check_params(p));
+    if (bytes == nullptr) FAIL(BSA_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = ws_layout(*p).total;
+    if (max_nnz != nullptr) {
+        const Dims D = dims_of(*p);
+        *max_nnz = D.rows * D.nKB;
+    }
+    return BSA_OK;
+}
+
+bsa_status bsa_pool(const bsa_params *p, const void *q, const void *k, const void *v, float *qbar,
+                    float *kbar, float *vbar, int32_t *blk_count, void *stream)
+{
+    g_err[0] = 0;
+    TRY(check_params(p));
+    TRY(check_tensor(q, "q"));
+    TRY(check_tensor(k, "k"));
+    TRY(check_tensor(v, "v"));
+    TRY(check_tensor(qbar, "qbar"));
+    TRY(check_tensor(kbar, "kbar"));
+    TRY(check_tensor(vbar, "vbar"));
+    const Dims D = dims_of(*p);
+    return from_cuda(launch_pool(*p, D, q, k, v, qbar, kbar, vbar, blk_count, (cudaStream_t)stream), "bsa_pool");
+}
+
+bsa_status bsa_select(const bsa_params *p, const float *qbar, const float *kbar, const void *k,
+                      int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity, int32_t *kept_count,
+                      int32_t *extra_idx, int32_t *extra_count, void *ws, size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    TRY(check_params(p));
+    TRY(check_tensor(qbar, "qbar"));
+    TRY(check_tensor(kbar, "kbar"));
+    if (row_ptr == nullptr || kept_count == nullptr) FAIL(BSA_ERR_INVALID_ARG, "row_ptr / kept_count is NULL");
+    if (col_capacity < 0) FAIL(BSA_ERR_INVALID_ARG, "col_capacity < 0");
+    if (col_capacity > 0 && col_idx == nullptr) FAIL(BSA_ERR_INVALID_ARG, "col_idx is NULL");
+    if (p->extra_tokens > 0) {
+        (void)k;
+        (void)extra_idx;
+        (void)extra_count;
+        FAIL(BSA_ERR_UNSUPPORTED, "extra_tokens > 0 is not available in this build yet");
+    }
+    TRY(check_ws(p, ws, ws_bytes));
+    const Dims D = dims_of(*p);
+    const WsLayout L = ws_layout(*p);
+    return from_cuda(launch_select(*p, D, qbar, kbar, row_ptr, col_idx, col_capacity, kept_count,
+                                   static_cast<char *>(ws), L, (cudaStream_t)stream),
+                     "bsa_select");
+}
+
+bsa_status bsa_attention(const bsa_params *p, const void *q, const void *k, const void *v, const float *kbar,
+                         const float *vbar, const int32_t *blk_count, const int64_t *row_ptr,
+                         const int32_t *col_idx, const int32_t *extra_idx, const int32_t *extra_count,
+                         void *out, float *lse, void *ws, size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    TRY(check_params(p));
+    TRY(check_tensor(q, "q"));
+    TRY(check_tensor(k, "k"));
+    TRY(check_tensor(v, "v"));
+    TRY(check_tensor(out, "out"));
+    if (p->centroid) {
+        TRY(check_tensor(kbar, "kbar"));
+        TRY(check_tensor(vbar, "vbar"));
+    }
+    (void)blk_count;
+    if (row_ptr == nullptr || col_idx == nullptr) FAIL(BSA_ERR_INVALID_ARG, "row_ptr / col_idx is NULL");
+    if (p->extra_tokens > 0)
+        FAIL(BSA_ERR_UNSUPPORTED, "extra_tokens > 0 is not available in this build yet");
+    TRY(check_ws(p, ws, ws_bytes));
+    const Dims D = dims_of(*p);
+    const WsLayout L = ws_layout(*p);
+    return from_cuda(launch_attention(*p, D, q, k, v, kbar, vbar, row_ptr, col_idx, extra_idx, extra_count,
+                                      out, lse, 0, p->dense_row_begin, p->dense_row_end,
+                                      static_cast<char *>(ws), L, (cudaStream_t)stream),
+                     "bsa_attention");
+}
+
+bsa_status bsa_dense_ref_rows(const bsa_params *p, const void *q, const void *k, const void *v,
+                              int32_t row_begin, int32_t row_end, void *out, float *lse, void *ws,
+                              size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    TRY(check_params(p));
+    TRY(check_tensor(q, "q"));
+    TRY(check_tensor(k, "k"));
+    TRY(check_tensor(v, "v"));
+    TRY(check_tensor(out, "out"));
+    if (row_begin < 0 || row_end < row_begin || row_end > p->N)
+        FAIL(BSA_ERR_INVALID_ARG, "rows must satisfy 0 <= begin <= end <= N");
+    TRY(check_ws(p, ws, ws_bytes));
+    if (row_end == row_begin) return BSA_OK;
+    const Dims D = dims_of(*p);
+    const WsLayout L = ws_layout(*p);
+    return from_cuda(launch_attention(*p, D, q, k, v, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, out,
+                                      lse, 1, row_begin, row_end, static_cast<char *>(ws), L,
+                                      (cudaStream_t)stream),
+                     "bsa_dense_ref_rows");
+}
+
+bsa_status bsa_device_status(void *ws, void *stream, int32_t *device_status)
+{
+    g_err[0] = 0;
+    if (ws == nullptr || device_status == nullptr) FAIL(BSA_ERR_INVALID_ARG, "ws / device_status is NULL");
+    cudaStream_t st = (cudaStream_t)stream;
+    TRY(from_cuda(cudaStreamSynchronize(st), "cudaStreamSynchronize"));
+    int32_t h[2] = {0, 0};
+    TRY(from_cuda(cudaMemcpyAsync(h, ws, sizeof h, cudaMemcpyDeviceToHost, st), "status copy"));
+    TRY(from_cuda(cudaMemsetAsync(ws, 0, sizeof h, st), "status reset"));
+    TRY(from_cuda(cudaStreamSynchronize(st), "cudaStreamSynchronize"));
+    *device_status = h[0];
+    if (h[0] != 0) set_error("device status %d (detail %d)", h[0], h[1]);
+    return BSA_OK;
+}
+
+const char *bsa_status_string(bsa_status s)
+{
+    switch (s) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported";
+    case BSA_ERR_CAPACITY: return "capacity exceeded";
+    case BSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case BSA_ERR_CUDA: return "CUDA error";
+    case BSA_ERR_DEVICE: return "device-side error";
+    }
+    return "unknown status";
+}
+
+const char *bsa_last_error(void) { return g_err; }
+
+}  // extern "C"

@@ -1,0 +1,59 @@
+// bsa_internal.h -- declarations shared by the host API and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "bsa.h"
+
+namespace bsa {
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Derived sizes of one problem.
+struct Dims {
+    int B, H, N, d;
+    int Bq, Bk;
+    int nQB, nKB, nW;      // nW = 32-bit words of a per-row key-block bitmask
+    int64_t rows;          // B * H * nQB
+    int E;
+};
+
+Dims dims_of(const bsa_params &p);
+
+// Byte offsets of the workspace regions (each 256-byte aligned).
+struct WsLayout {
+    size_t status;         // DevStatus
+    size_t scores;         // [rows, nKB] f32 block scores (select)
+    size_t bitmask;        // [rows, nW] u32 kept-block bitmask (select)
+    size_t counts;         // [rows] i32 kept counts (select)
+    size_t kc16, vc16;     // [B*H, nKB, d] bf16 centroids (attention)
+    size_t cbias;          // [rows, nKB_pad] f32 per-row centroid bias overrides (extra tokens)
+    size_t xk16, xv16;     // [rows, E, d] bf16 modified centroids (extra tokens)
+    size_t q16, k16, v16;  // [B, N, H, d] bf16 copies of f32 inputs (attention, f32 only)
+    size_t total;
+};
+
+WsLayout ws_layout(const bsa_params &p);
+
+cudaError_t launch_pool(const bsa_params &p, const Dims &D, const void *q, const void *k,
+                        const void *v, float *qbar, float *kbar, float *vbar, int32_t *blk_count,
+                        cudaStream_t st);
+
+cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar, const float *kbar,
+                          int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                          int32_t *kept_count, char *ws, const WsLayout &L, cudaStream_t st);
+
+cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, const void *k,
+                             const void *v, const float *kbar, const float *vbar,
+                             const int64_t *row_ptr, const int32_t *col_idx, const int32_t *extra_idx,
+                             const int32_t *extra_count, void *out, float *lse, int dense_only,
+                             int row_begin, int row_end, char *ws, const WsLayout &L,
+                             cudaStream_t st);
+
+// Thread-local host error text.
+void set_error(const char *fmt, ...);
+
+}  // namespace bsa

@@ -1,0 +1,337 @@
+// select.cu -- step 2: routing of key blocks per (batch, head, query block).
+//
+// "BlockSparseAttention - ComfyUI Built-in Node Documentation":
+//   "sol-attn inputs", tau: a threshold counted in standard deviations of the
+//   row's score distribution (higher = sparser);
+//   "sla inputs", keep_percent: the percentage of key blocks kept exactly per
+//   query block, sink and diagonal blocks kept in addition;
+//   general inputs, sink_conditioning = exact_kv: every query attends exactly
+//   to the packed conditioning rows.
+//
+// Kernels:
+//   scores_kernel  S[r, j] = fl32((qbar_r . kbar_j) / sqrt d) with fp64 FMAs in
+//                  channel order (the same value the definition gives).  A CTA
+//                  computes a 32-row x 128-key tile per pass over kbar, staging
+//                  channel slices of kbar in shared memory as fp64.
+//   rows_kernel    one warp per row: two-pass fp64 mean / population std,
+//                  thr = fl32(mean + tau * std), keep S > thr (Sol) or an exact
+//                  radix select of the top k (SLA); forced blocks OR'ed in;
+//                  result as a bitmask word per 32 key blocks (ballot) + count.
+//   scan_kernel    exclusive scan of the counts -> CSR row_ptr (int64).
+//   expand_kernel  bitmask -> ascending CSR column lists (popc prefix per warp).
+#include <math.h>
+
+#include "bsa_device.cuh"
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+constexpr int kRows = 32;     // query-block rows per CTA
+constexpr int kKeys = 128;    // key blocks per pass
+constexpr int kChan = 32;     // channels staged per step
+
+__global__ void __launch_bounds__(256) scores_kernel(const float *__restrict__ qbar,
+                                                     const float *__restrict__ kbar, int nQB,
+                                                     int nKB, int d, float *__restrict__ S)
+{
+    extern __shared__ double sel_smem[];
+    double(*qs)[128] = reinterpret_cast<double(*)[128]>(sel_smem);
+    double(*ks)[kKeys + 1] = reinterpret_cast<double(*)[kKeys + 1]>(sel_smem + kRows * 128);
+    const int bh = blockIdx.y;
+    const int r0 = blockIdx.x * kRows;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const double rs = sqrt((double)d);
+
+    for (int idx = threadIdx.x; idx < kRows * d; idx += blockDim.x) {
+        const int r = idx / d, c = idx % d;
+        qs[r][c] = (r0 + r < nQB) ? (double)qbar[((int64_t)bh * nQB + r0 + r) * d + c] : 0.0;
+    }
+    const float *kb = kbar + (int64_t)bh * nKB * d;
+    for (int j0 = 0; j0 < nKB; j0 += kKeys) {
+        double acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+        for (int c0 = 0; c0 < d; c0 += kChan) {
+            __syncthreads();
+            for (int idx = threadIdx.x; idx < kKeys * kChan; idx += blockDim.x) {
+                const int j = idx / kChan, c = idx % kChan;
+                ks[c][j] = (j0 + j < nKB) ? (double)kb[(int64_t)(j0 + j) * d + c0 + c] : 0.0;
+            }
+            __syncthreads();
+#pragma unroll 2
+            for (int c = 0; c < kChan; ++c) {
+                double qv[4], kv[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) qv[a] = qs[4 * warp + a][c0 + c];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) kv[b] = ks[c][lane + 32 * b];
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(qv[a], kv[b], acc[a][b]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int r = r0 + 4 * warp + a;
+            if (r >= nQB) continue;
+            float *row = S + ((int64_t)bh * nQB + r) * nKB;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int j = j0 + lane + 32 * b;
+                if (j < nKB) row[j] = (float)(acc[a][b] / rs);
+            }
+        }
+    }
+}
+
+struct RowArgs {
+    const float *S;
+    int64_t rows;
+    int nQB, nKB, nW, N, Bq, Bk;
+    int method;
+    double tau;
+    int topk;
+    int sink_blocks, prefix_blocks, keep_diag;
+    uint32_t *bitmask;
+    int32_t *count;
+};
+
+__device__ __forceinline__ double warp_sum(double v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Order-preserving map of a float to uint32 (larger float -> larger key);
+// -0 and +0 map to the same key so that they tie, as in a float comparison.
+__device__ __forceinline__ uint32_t ord_key(float f)
+{
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) == 0) u = 0;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(256) rows_kernel(RowArgs a)
+{
+    __shared__ uint32_t hist_all[8][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * 8 + warp;
+    if (r >= a.rows) return;
+    const float *s = a.S + r * a.nKB;
+    const int i = (int)(r % a.nQB);
+    const int nKB = a.nKB;
+
+    // forced: [0, fb) sink/prefix, and the diagonal range [d0, d1]
+    const int fb = max(min(a.sink_blocks, nKB), min(a.prefix_blocks, nKB));
+    int d0 = 1, d1 = 0;
+    if (a.keep_diag) {
+        const int q0 = i * a.Bq, q1 = min(a.N, q0 + a.Bq) - 1;
+        d0 = q0 / a.Bk;
+        d1 = min(q1 / a.Bk, nKB - 1);
+    }
+
+    int mode = 0;            // 0: threshold, 1: keep all, 2: none, 3: top-k
+    float thr = 0.f;
+    uint32_t vk = 0;
+    int need = 0;
+    if (a.method == BSA_SOL) {
+        if (isinf(a.tau) && a.tau < 0) {
+            mode = 1;
+        } else {
+            double sum = 0.0;
+            for (int j = lane; j < nKB; j += 32) sum += (double)s[j];
+            const double mu = warp_sum(sum) / (double)nKB;
+            double sq = 0.0;
+            for (int j = lane; j < nKB; j += 32) {
+                const double e = __dadd_rn((double)s[j], -mu);
+                sq = __dadd_rn(sq, __dmul_rn(e, e));
+            }
+            const double sigma = sqrt(warp_sum(sq) / (double)nKB);
+            if (isinf(a.tau) || !(sigma > 0.0)) {
+                mode = 2;
+            } else {
+                thr = (float)__dadd_rn(mu, __dmul_rn(a.tau, sigma));
+            }
+        }
+    } else {
+        // exact k-th largest key by 8-bit radix passes, then ties to the lower index
+        uint32_t *hist = hist_all[warp];
+        uint32_t prefix = 0, pmask = 0;
+        int remaining = a.topk;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int t = lane; t < 256; t += 32) hist[t] = 0;
+            __syncwarp();
+            for (int j = lane; j < nKB; j += 32) {
+                const uint32_t u = ord_key(s[j]);
+                if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+            }
+            __syncwarp();
+            int digit = 0, above = 0;
+            if (lane == 0) {
+                int acc = 0;
+                for (int bin = 255; bin >= 0; --bin) {
+                    const int c = (int)hist[bin];
+                    if (acc + c >= remaining) {
+                        digit = bin;
+                        above = acc;
+                        break;
+                    }
+                    acc += c;
+                }
+            }
+            digit = __shfl_sync(0xffffffffu, digit, 0);
+            above = __shfl_sync(0xffffffffu, above, 0);
+            remaining -= above;
+            prefix |= (uint32_t)digit << shift;
+            pmask |= 0xFFu << shift;
+            __syncwarp();
+        }
+        vk = prefix;
+        need = remaining;    // elements equal to vk still to take, lowest index first
+        mode = 3;
+    }
+
+    int total = 0, eq_taken = 0;
+    uint32_t *bm = a.bitmask + r * a.nW;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int w = 0; w < a.nW; ++w) {
+        const int j = w * 32 + lane;
+        const bool valid = j < nKB;
+        const float sj = valid ? s[j] : 0.f;
+        bool keep = false;
+        if (mode == 0) {
+            keep = valid && sj > thr;
+        } else if (mode == 1) {
+            keep = valid;
+        } else if (mode == 3) {
+            const uint32_t u = ord_key(sj);
+            const bool eq = valid && u == vk;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const int rank = eq_taken + __popc(eqm & lt_mask);
+            keep = valid && (u > vk || (eq && rank < need));
+            eq_taken += __popc(eqm);
+        }
+        keep = keep || (valid && (j < fb || (j >= d0 && j <= d1)));
+        const uint32_t word = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) bm[w] = word;
+        total += __popc(word);
+    }
+    if (lane == 0) a.count[r] = total;
+}
+
+// Exclusive scan of counts into int64 row_ptr (single CTA of 1024 threads).
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ count, int64_t rows,
+                                                    int64_t *__restrict__ row_ptr)
+{
+    __shared__ int64_t part[1024];
+    const int t = threadIdx.x;
+    const int64_t per = (rows + 1023) / 1024;
+    const int64_t lo = min(rows, t * per), hi = min(rows, lo + per);
+    int64_t s = 0;
+    for (int64_t i = lo; i < hi; ++i) s += count[i];
+    part[t] = s;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {
+        const int64_t v = t >= off ? part[t - off] : 0;
+        __syncthreads();
+        part[t] += v;
+        __syncthreads();
+    }
+    int64_t run = part[t] - s;
+    for (int64_t i = lo; i < hi; ++i) {
+        row_ptr[i] = run;
+        run += count[i];
+    }
+    if (t == 1023) row_ptr[rows] = part[1023];
+}
+
+__global__ void __launch_bounds__(256) expand_kernel(const uint32_t *__restrict__ bitmask,
+                                                     const int32_t *__restrict__ count,
+                                                     const int64_t *__restrict__ row_ptr,
+                                                     int64_t rows, int nW, int64_t capacity,
+                                                     int32_t *__restrict__ col,
+                                                     int32_t *__restrict__ kept_count,
+                                                     int32_t *status)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * 8 + warp;
+    if (r >= rows) return;
+    const int64_t start = row_ptr[r];
+    if (lane == 0) {
+        kept_count[r] = count[r];
+        if (start + count[r] > capacity) report(status, BSA_DEV_CAPACITY, (int32_t)(r & 0x7fffffff));
+    }
+    const uint32_t *bm = bitmask + r * nW;
+    int64_t base = start;
+    for (int w0 = 0; w0 < nW; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t word = w < nW ? bm[w] : 0u;
+        const int pc = __popc(word);
+        int incl = pc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int64_t pos = base + (incl - pc);
+        while (word) {
+            const int bit = __ffs(word) - 1;
+            word &= word - 1;
+            if (pos < capacity) col[pos] = w * 32 + bit;
+            ++pos;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar, const float *kbar,
+                          int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                          int32_t *kept_count, char *ws, const WsLayout &L, cudaStream_t st)
+{
+    float *S = reinterpret_cast<float *>(ws + L.scores);
+    uint32_t *bm = reinterpret_cast<uint32_t *>(ws + L.bitmask);
+    int32_t *cnt = reinterpret_cast<int32_t *>(ws + L.counts);
+    int32_t *status = reinterpret_cast<int32_t *>(ws + L.status);
+
+    dim3 g1((unsigned)ceil_div(D.nQB, kRows), (unsigned)(D.B * D.H));
+    const int smem = (kRows * 128 + kChan * (kKeys + 1)) * (int)sizeof(double);
+    cudaError_t e = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    scores_kernel<<<g1, 256, smem, st>>>(qbar, kbar, D.nQB, D.nKB, D.d, S);
+
+    RowArgs a;
+    a.S = S;
+    a.rows = D.rows;
+    a.nQB = D.nQB;
+    a.nKB = D.nKB;
+    a.nW = D.nW;
+    a.N = D.N;
+    a.Bq = D.Bq;
+    a.Bk = D.Bk;
+    a.method = p.method;
+    a.tau = p.tau;
+    long kk = lround(p.keep_percent * (double)D.nKB / 100.0);
+    if (kk < 1) kk = 1;
+    if (kk > D.nKB) kk = D.nKB;
+    a.topk = (int)kk;
+    a.sink_blocks = p.sink_blocks;
+    a.prefix_blocks = p.prefix_len > 0 ? (int)ceil_div(p.prefix_len, D.Bk) : 0;
+    a.keep_diag = p.keep_diag;
+    a.bitmask = bm;
+    a.count = cnt;
+    const unsigned g2 = (unsigned)ceil_div(D.rows, 8);
+    rows_kernel<<<g2, 256, 0, st>>>(a);
+    scan_kernel<<<1, 1024, 0, st>>>(cnt, D.rows, row_ptr);
+    expand_kernel<<<g2, 256, 0, st>>>(bm, cnt, row_ptr, D.rows, D.nW, col_capacity, col_idx,
+                                      kept_count, status);
+    return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -1,0 +1,177 @@
+/*
+ * bsa.h -- C ABI of libbsa: training-free block-sparse "sol-attn" attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation (sources are web pages, cited by title and section):
+ *   [DOC]  "BlockSparseAttention - ComfyUI Built-in Node Documentation":
+ *          general-inputs table (extra_tokens, sink_conditioning),
+ *          "sol-attn inputs" (tau), "sla inputs" (keep_percent).
+ *   [STAR] "minimax-h3-chunk-star7" README, sections "SLA" and "Sol".
+ *
+ *   1. bsa_pool       -- Q and K (and V, for the centroids) are mean-pooled per
+ *                        block of consecutive tokens (Q64/K64 for Sol, Q128/K64
+ *                        for SLA: [STAR] "SLA", "Sol").
+ *   2. bsa_select     -- per (batch, head, query block) row of pooled scores
+ *                        S = qbar . kbar / sqrt(d): Sol keeps the blocks above
+ *                        mean + tau * std of the row ([DOC] tau: a threshold in
+ *                        standard deviations of the score distribution); SLA
+ *                        keeps the top keep_percent % ([DOC] keep_percent).  Sink,
+ *                        prefix and diagonal blocks are kept in addition.
+ *                        Optionally picks extra_tokens top-scoring tokens per
+ *                        query block outside its kept blocks ([DOC] extra_tokens).
+ *   3. bsa_attention  -- exact attention over the kept key blocks (and extra
+ *                        tokens); every unselected block contributes through its
+ *                        K/V centroid with logit q.kbar/sqrt(d) + ln(n_b); both
+ *                        merge into one FP32 online softmax ([STAR] "Sol").
+ *                        Rows in [dense_row_begin, dense_row_end) are computed
+ *                        densely and replace the sparse result ([DOC]
+ *                        sink_conditioning = exact_kv_and_rows).
+ *   4. bsa_dense_ref_rows -- dense softmax attention for a range of query rows.
+ *
+ * Conventions shared by every call:
+ *   - Tensors Q, K, V and O are [B, N, H, d] with element strides stride_b,
+ *     stride_n, stride_h and a contiguous channel dimension; all four share the
+ *     same strides.  Base pointers must be 16-byte aligned and stride_b,
+ *     stride_n, stride_h multiples of 8 elements (bf16) or 4 elements (f32).
+ *   - Every pointer argument is a device pointer unless stated otherwise; the
+ *     caller owns all memory.  The library allocates no device memory.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = legacy default stream).  Argument errors are detected on the host
+ *     and returned before anything is launched; launch failures return
+ *     BSA_ERR_CUDA.  Errors found by the kernels (e.g. a CSR capacity overflow)
+ *     are written to a status word inside the workspace and read back with
+ *     bsa_device_status().  No kernel traps.
+ *   - Calls are thread-safe; the library keeps no global state apart from a
+ *     thread-local message describing the last host-side error.
+ *   - Rows are ordered [B, H, nQB]: row r = (b * H + h) * nQB + i, where
+ *     nQB = ceil(N / q_block) and nKB = ceil(N / k_block).
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BSA_OK = 0,
+    BSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, stride, alignment or parameter */
+    BSA_ERR_UNSUPPORTED = 2,   /* valid request outside this build (d not in {64,128}, ...) */
+    BSA_ERR_CAPACITY = 3,      /* an output array is too small (host- or device-detected) */
+    BSA_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than bsa_workspace_size() */
+    BSA_ERR_CUDA = 5,          /* a CUDA runtime call or a kernel launch failed */
+    BSA_ERR_DEVICE = 6         /* a kernel reported an internal error (status word) */
+} bsa_status;
+
+typedef enum { BSA_DT_BF16 = 0, BSA_DT_F32 = 1 } bsa_dtype;
+typedef enum { BSA_SOL = 0, BSA_SLA = 1 } bsa_method;   /* vsa: not provided (needs trained weights) */
+
+typedef struct {
+    int32_t B, H, N, d;            /* batch, heads, tokens, head dim (64 or 128) */
+    int64_t stride_b, stride_n, stride_h;   /* element strides of Q, K, V, O */
+    int32_t dtype;                 /* bsa_dtype of Q, K, V and O */
+    int32_t method;                /* bsa_method */
+    int32_t q_block, k_block;      /* Sol 64/64, SLA 128/64 ([STAR] "SLA", "Sol"); k_block must be 64 */
+    double  tau;                   /* Sol threshold in standard deviations; -inf keeps all, +inf none */
+    double  keep_percent;          /* SLA: percent of key blocks kept per query block, (0, 100] */
+    int32_t sink_blocks;           /* leading key blocks always kept (default 1) */
+    int32_t keep_diag;             /* 1: key blocks meeting the query block's tokens always kept */
+    int32_t prefix_len;            /* P: packed conditioning rows [0, P) every query attends to exactly
+                                      (exact_kv); 0 disables */
+    int32_t dense_row_begin;       /* query rows [begin, end) run dense and replace the sparse result */
+    int32_t dense_row_end;         /*   (exact_kv_and_rows); begin == end disables */
+    int32_t extra_tokens;          /* E: extra top-scoring tokens per query block, 0..256; 0 disables */
+    int32_t centroid;              /* 1: unselected blocks contribute through centroids (Sol);
+                                      0: they are dropped (SLA without its trained linear branch) */
+} bsa_params;
+
+/* Fill *p with the defaults of the node documentation for `method`
+ * (Sol: tau 1.3, Q64/K64, centroid on; SLA: keep_percent 10, Q128/K64,
+ * centroid off; both: sink 1, diagonal kept, no prefix, no dense rows, E 0).
+ * Shapes and strides are left zero. */
+BSA_API void bsa_default_params(bsa_params *p, int32_t method);
+
+/* Bytes of device workspace the select and attention calls need for these
+ * parameters (*bytes), and the largest possible number of kept entries,
+ * B*H*nQB*nKB (*max_nnz), an always-sufficient CSR capacity. */
+BSA_API bsa_status bsa_workspace_size(const bsa_params *p, size_t *bytes, int64_t *max_nnz);
+
+/* Step 1, pooling ([STAR] "SLA", "Sol": Q/K blocks; K/V centroids).
+ *   q, k, v   : [B, N, H, d] inputs (dtype, strides from p).
+ *   qbar      : out [B, H, nQB, d] f32, mean of Q over each query block.
+ *   kbar, vbar: out [B, H, nKB, d] f32, means of K and V over each key block.
+ *   blk_count : out [nKB] int32, tokens in each key block (the last may be partial).
+ * Sums run in fp64 in token order; each mean is rounded once to f32. */
+BSA_API bsa_status bsa_pool(const bsa_params *p, const void *q, const void *k, const void *v,
+                    float *qbar, float *kbar, float *vbar, int32_t *blk_count, void *stream);
+
+/* Step 2, selection ([DOC] "sol-attn inputs" tau, "sla inputs" keep_percent,
+ * general inputs extra_tokens).
+ *   qbar, kbar  : pooled means from bsa_pool.
+ *   k           : [B, N, H, d] keys (read only when p->extra_tokens > 0).
+ *   row_ptr     : out [rows + 1] int64 CSR offsets.
+ *   col_idx     : out [col_capacity] int32 kept key-block indices, ascending per row.
+ *   kept_count  : out [rows] int32 kept blocks per row.
+ *   extra_idx   : out [rows, E] int32 extra tokens, ascending, -1 padded (NULL if E == 0).
+ *   extra_count : out [rows] int32 (NULL if E == 0).
+ *   ws, ws_bytes: workspace of at least bsa_workspace_size() bytes.
+ * Scores are computed in fp64 and rounded to f32 (S = fl32(qbar.kbar / sqrt d));
+ * row mean and population std are taken in fp64 over all nKB scores;
+ * thr = fl32(mean + tau * std); block b is kept iff S_b > thr.  If the total
+ * kept count exceeds col_capacity, the status word reports BSA_ERR_CAPACITY and
+ * col_idx holds only the entries that fit. */
+BSA_API bsa_status bsa_select(const bsa_params *p, const float *qbar, const float *kbar, const void *k,
+                      int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                      int32_t *kept_count, int32_t *extra_idx, int32_t *extra_count,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/* Step 3, fine pass ([STAR] "Sol": exact kept blocks + centroids of the
+ * others in one FP32 online softmax; [DOC] sink_conditioning).
+ *   q, k, v        : [B, N, H, d] inputs.
+ *   kbar, vbar     : [B, H, nKB, d] f32 centroids from bsa_pool.
+ *   blk_count      : [nKB] int32 block sizes from bsa_pool.
+ *   row_ptr, col_idx: CSR of kept blocks (ascending within each row), e.g. from bsa_select.
+ *   extra_idx, extra_count: extra tokens ([rows, E], [rows]); NULL when E == 0.
+ *   out            : out [B, N, H, d] attention output, dtype of q.
+ *   lse            : out [B, H, N] f32 natural-log softmax normaliser; may be NULL.
+ * A block that gave extra tokens keeps a centroid over its remaining tokens
+ * (bias ln of their count); a block left empty contributes nothing.  Rows in
+ * [dense_row_begin, dense_row_end) are computed densely by this call. */
+BSA_API bsa_status bsa_attention(const bsa_params *p, const void *q, const void *k, const void *v,
+                         const float *kbar, const float *vbar, const int32_t *blk_count,
+                         const int64_t *row_ptr, const int32_t *col_idx,
+                         const int32_t *extra_idx, const int32_t *extra_count,
+                         void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* Step 4, dense rows ([DOC] sink_conditioning = exact_kv_and_rows: designated
+ * query rows attend densely): rows [row_begin, row_end) of every (b, h) attend
+ * to all N keys; writes those rows of out (and lse, if not NULL). */
+BSA_API bsa_status bsa_dense_ref_rows(const bsa_params *p, const void *q, const void *k, const void *v,
+                              int32_t row_begin, int32_t row_end, void *out, float *lse,
+                              void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, return the status the kernels wrote into `ws` since the
+ * last call (BSA_OK if none) in *device_status, and clear it.  The return value
+ * is BSA_ERR_CUDA if the synchronisation itself failed. */
+BSA_API bsa_status bsa_device_status(void *ws, void *stream, int32_t *device_status);
+
+/* Static description of a status code. */
+BSA_API const char *bsa_status_string(bsa_status s);
+
+/* Thread-local text of the most recent host-side error of this thread ("" if none). */
+BSA_API const char *bsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */

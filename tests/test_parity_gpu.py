@@ -1,0 +1,161 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle,
+element by element, on seeded inputs that span several tiles and ragged tails.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_26_b200 as bsa
+import oracle
+from tests.gpu_helpers import (compare_masks, compare_outputs, csr_to_mask, gpu_layer, params_for,
+                               to_cpu_raw)
+from workloads import TINY_SOL, Workload, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny_sol": TINY_SOL,
+    "sol_grid": Workload("sol_grid", B=1, H=3, N=3000, d=128, dtype="bf16", method="sol", q_block=64,
+                         k_block=64, tau=1.3, grid=(3, 20, 50), seed=11),
+    "sla_grid": Workload("sla_grid", B=1, H=2, N=2880, d=128, dtype="bf16", method="sla", q_block=128,
+                         k_block=64, keep_percent=15.0, centroid=0, grid=(4, 24, 30), seed=12),
+    "sol_sinks": Workload("sol_sinks", B=1, H=2, N=2120, d=128, dtype="bf16", method="sol", q_block=64,
+                          k_block=64, tau=1.3, prefix_len=200, dense_rows=(72, 200), grid=(3, 16, 40),
+                          seed=13),
+    "sol_b2_d64": Workload("sol_b2_d64", B=2, H=2, N=1500, d=64, dtype="bf16", method="sol", q_block=64,
+                           k_block=64, tau=0.8, grid=(3, 10, 50), seed=14),
+    "sol_dense_tau": Workload("sol_dense_tau", B=1, H=2, N=1100, d=128, dtype="bf16", method="sol",
+                              q_block=64, k_block=64, tau=-math.inf, grid=(2, 10, 55), seed=15),
+    "sla_keep_all": Workload("sla_keep_all", B=1, H=2, N=1000, d=128, dtype="bf16", method="sla",
+                             q_block=128, k_block=64, keep_percent=100.0, centroid=0, grid=(2, 10, 50),
+                             seed=16),
+    "single_block": Workload("single_block", B=1, H=2, N=40, d=128, dtype="bf16", method="sol", q_block=64,
+                             k_block=64, tau=1.0, grid=(1, 5, 8), seed=17),
+    "no_diag_no_sink": Workload("no_diag_no_sink", B=1, H=2, N=1300, d=128, dtype="bf16", method="sol",
+                                q_block=64, k_block=64, tau=1.0, sink_blocks=0, keep_diag=0,
+                                grid=(2, 13, 50), seed=18),
+}
+
+
+def _inputs(w, layout="bnhd"):
+    q, k, v = make_qkv(w, "cpu", layout)
+    return q, k, v, q.cuda(), k.cuda(), v.cuda()
+
+
+def _to_cuda_like(t):
+    """Copy a (possibly strided) CPU tensor to the GPU keeping its strides."""
+    out = torch.empty_strided(t.shape, t.stride(), dtype=t.dtype, device="cuda")
+    out.copy_(t)
+    return out
+
+
+@pytest.fixture(scope="module")
+def runs():
+    cache = {}
+
+    def get(name, layout="bnhd"):
+        key = (name, layout)
+        if key not in cache:
+            w = SMALL[name]
+            qc, kc, vc = make_qkv(w, "cpu", layout)
+            q, k, v = (_to_cuda_like(t) for t in (qc, kc, vc))
+            p, buf, out, status = gpu_layer(w, q, k, v)
+            res = oracle.routing(w, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc))
+            cache[key] = (w, (qc, kc, vc), (q, k, v), p, buf, out, status, res)
+        return cache[key]
+
+    return get
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_pool_bit_exact(runs, name):
+    w, _, _, p, buf, _, status, res = runs(name)
+    assert status == 0
+    assert np.array_equal(buf.qbar.cpu().numpy(), res.qbar)
+    assert np.array_equal(buf.kbar.cpu().numpy(), res.kbar)
+    assert np.array_equal(buf.vbar.cpu().numpy(), res.vbar)
+    assert np.array_equal(buf.blk_count.cpu().numpy(), res.count)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_select_masks_match(runs, name):
+    w, _, _, p, buf, _, status, res = runs(name)
+    assert status == 0
+    mask = csr_to_mask(buf.row_ptr, buf.col_idx, w.rows, w.nKB)
+    exempt = compare_masks(mask, res, w)
+    assert exempt <= max(1, w.rows // 1000), exempt
+    kc = buf.kept_count.cpu().numpy()
+    assert np.array_equal(kc, mask.sum(axis=1))
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_attention_matches_oracle(runs, name):
+    w, (qc, kc, vc), _, p, buf, out, status, res = runs(name)
+    assert status == 0
+    tokens = oracle.all_tokens(w)
+    ref, ref_lse = oracle.layer_rows(w, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc), res, tokens)
+    got = out.float().cpu().permute(0, 2, 1, 3).reshape(-1, w.d).numpy()   # (b, h, n) order
+    compare_outputs(got, ref, f"{name} out")
+    lse = buf.lse.cpu().numpy().reshape(-1)
+    err = np.abs(lse - ref_lse)
+    assert err.max() < 2e-2, err.max()
+
+
+def test_strided_layout_matches_contiguous(runs):
+    """[B, H, N, d] storage (head-major) gives the same result as [B, N, H, d]."""
+    a = runs("sol_grid", "bnhd")
+    b = runs("sol_grid", "bhnd")
+    assert np.array_equal(a[4].qbar.cpu().numpy(), b[4].qbar.cpu().numpy())
+    assert torch.equal(a[4].row_ptr.cpu(), b[4].row_ptr.cpu())
+    assert torch.equal(a[5].cpu(), b[5].cpu())
+
+
+def test_dense_ref_rows_matches_dense_attention():
+    w = SMALL["sol_grid"]
+    qc, kc, vc = make_qkv(w, "cpu")
+    q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
+    p = params_for(w, q)
+    buf = bsa.Buffers(p, q.device)
+    out = torch.zeros_like(q)
+    lse = torch.zeros((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+    r0, r1 = 100, 333
+    bsa.bsa_dense_ref_rows(p, q, k, v, r0, r1, out, lse, buf.ws)
+    assert bsa.bsa_device_status(buf.ws) == 0
+    tokens = np.array([(0, h, n) for h in range(w.H) for n in range(r0, r1)], np.int64)
+    wd = w.replace(dense_rows=(r0, r1))
+    res = oracle.routing(wd, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc))
+    ref, ref_lse = oracle.layer_rows(wd, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc), res, tokens)
+    got = out[0, r0:r1].float().cpu().permute(1, 0, 2).reshape(-1, w.d).numpy()
+    compare_outputs(got, ref, "dense rows")
+    assert torch.count_nonzero(out[0, :r0]) == 0 and torch.count_nonzero(out[0, r1:]) == 0
+    got_lse = lse[0, :, r0:r1].cpu().numpy().reshape(-1)
+    assert np.abs(got_lse - ref_lse).max() < 2e-2
+
+
+def test_capacity_overflow_reported_on_device():
+    w = SMALL["sol_grid"]
+    qc, kc, vc = make_qkv(w, "cpu")
+    q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
+    p = params_for(w, q)
+    buf = bsa.Buffers(p, q.device, capacity=10)
+    bsa.bsa_pool(p, q, k, v, buf.qbar, buf.kbar, buf.vbar, buf.blk_count)
+    bsa.bsa_select(p, buf.qbar, buf.kbar, k, buf.row_ptr, buf.col_idx, buf.kept_count, None, None, buf.ws)
+    assert bsa.bsa_device_status(buf.ws) == 3          # BSA_ERR_CAPACITY
+    assert bsa.bsa_device_status(buf.ws) == 0          # cleared by the read
+    assert int(buf.row_ptr[-1]) > 10                   # counts and offsets are still complete
+
+
+def test_sigma_zero_rows_keep_only_forced():
+    """Block-constant Q and K make every pooled score of a row equal (sigma = 0)."""
+    w = Workload("flat", B=1, H=2, N=640, d=128, dtype="bf16", method="sol", q_block=64, k_block=64,
+                 tau=1.0, grid=None, seed=19)
+    q = torch.ones((1, w.N, w.H, w.d), dtype=torch.bfloat16, device="cuda")
+    k = torch.ones_like(q)
+    v = torch.randn(q.shape, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).cuda()
+    p, buf, out, status = gpu_layer(w, q, k, v)
+    assert status == 0
+    kc = buf.kept_count.cpu().numpy()
+    # sink block 0 plus the diagonal block (the same block for query block 0)
+    assert kc[0] == 1 and (kc[1:w.nQB] == 2).all()
