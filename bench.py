@@ -1,0 +1,412 @@
+"""Benchmark: one layer of block-sparse "sol-attn" attention per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+A step is the whole hot path on one batch of synthetic inputs already resident
+in HBM: bsa_pool -> bsa_select -> bsa_attention (sparse + centroid + dense
+rows).  Rank 0 prints one JSON line.  Metric: sparse-attention ms per layer
+and dense-equivalent TFLOP/s (4*B*H*N^2*d / layer time); the roofline block
+reports the fine pass (bsa_attention) against the measured bf16 tensor peak on
+the FLOPs it really has to do (kept FLOPs, counted from the CSR of the run).
+
+Multi-GPU (torchrun): attention is independent per (batch, head), so every
+rank runs its own layer on its own inputs (weak scaling, no collective on the
+data path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, make_qkv  # noqa: E402
+
+DEFAULT_CONFIG = "long"
+METRIC = "sparse-attn ms/layer & dense-equiv TFLOP/s at N tokens; % roofline (kept FLOPs)"
+UNIT = "TFLOP/s (dense-equivalent)"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def dense_equiv_flops(w) -> float:
+    return 4.0 * w.B * w.H * float(w.N) * w.N * w.d
+
+
+def kept_flops(w, row_ptr: torch.Tensor, col: torch.Tensor) -> float:
+    """FLOPs of the fine pass actually required: 4*d per (query row, key) pair over
+    the exact keys and centroids of every sparse row, plus 4*d*N per dense row."""
+    rp = row_ptr.to(torch.int64)
+    cnt = (rp[1:] - rp[:-1]).view(w.B, w.H, w.nQB)
+    nnz = int(rp[-1])
+    c = col[:nnz].to(torch.int64)
+    last_n = w.N - (w.nKB - 1) * w.k_block
+    # exact keys per row: kept blocks x 64, minus the short last block where kept
+    row_of = torch.repeat_interleave(torch.arange(cnt.numel(), device=c.device), cnt.reshape(-1))
+    short = torch.zeros(cnt.numel(), dtype=torch.int64, device=c.device)
+    short.index_add_(0, row_of, (c == w.nKB - 1).to(torch.int64))
+    exact_keys = cnt.reshape(-1) * w.k_block - short * (w.k_block - last_n)
+    cent = (w.nKB - cnt.reshape(-1)) if w.centroid else torch.zeros_like(exact_keys)
+    per_row_keys = (exact_keys + cent).view(w.B, w.H, w.nQB).double()
+    # query rows per query block (the last one may be short)
+    qrows = torch.full((w.nQB,), float(w.q_block), dtype=torch.float64, device=c.device)
+    qrows[-1] = w.N - (w.nQB - 1) * w.q_block
+    r0, r1 = w.dense_rows
+    if r1 > r0:
+        # rows in the dense range are computed by the dense pass instead
+        for i in range(w.nQB):
+            lo, hi = i * w.q_block, min(w.N, (i + 1) * w.q_block)
+            ov = max(0, min(hi, r1) - max(lo, r0))
+            qrows[i] -= ov
+    sparse = float((per_row_keys * qrows.view(1, 1, -1)).sum())
+    dense = float(w.B * w.H * (r1 - r0) * w.N) if r1 > r0 else 0.0
+    return 4.0 * w.d * (sparse + dense)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+
+        def mhz(s):
+            try:
+                return float(s.split()[0])
+            except (ValueError, IndexError):
+                return None
+        sm = [mhz(r[1]) for r in rows if mhz(r[1]) is not None]
+        smax = max((mhz(r[2]) for r in rows if mhz(r[2]) is not None), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [x for x in sm if smax and x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(w, q, k, v, budget_s: float = 20.0):
+    """The CPU oracle, as it stands, on a bounded sample of the workload.
+
+    Sample: one head (b=0, h=0): pooling of Q, K and V, block scores and
+    selection for all of that head's query blocks, then exact/centroid attention
+    for a seeded sample of that head's query rows.  The layer time is
+    extrapolated: H*B x (pool + select of one head) + (B*H*N / rows) x attention.
+    """
+    import numpy as np
+
+    import oracle
+
+    w1 = w.replace(B=1, H=1)
+    qc, kc, vc = (t[:1, :, :1].cpu() for t in (q, k, v))
+    qr, kr, vr = oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc)
+    t0 = time.perf_counter()
+    res = oracle.routing(w1, qr, kr, vr, extra_rows=[], with_extra=False)
+    t_route = time.perf_counter() - t0
+    t_extra = 0.0
+    n_extra = 0
+    if w.extra_tokens > 0:
+        rows = list(range(0, w1.nQB, max(1, w1.nQB // 8)))[:8]
+        t0 = time.perf_counter()
+        ex, ec, rr = oracle.extra_tokens(res.qbar, kr, res.keep, w.q_block, w.k_block, w.extra_tokens, rows)
+        t_extra = time.perf_counter() - t0
+        n_extra = len(rows)
+        res.extra = np.full((w1.rows, w.extra_tokens), -1, np.int32)
+        res.ecnt = np.zeros((w1.rows,), np.int32)
+        res.extra[rr] = ex
+        res.ecnt[rr] = ec
+    # attention rows: grow the sample until about a quarter of the budget is used
+    g = np.random.default_rng(0)
+    m = 64
+    t_attn, done = 0.0, 0
+    while True:
+        toks = np.stack([np.zeros(m, np.int64), np.zeros(m, np.int64),
+                         g.integers(0, w.N, m).astype(np.int64)], axis=1)
+        if w.extra_tokens > 0:
+            # keep to query blocks whose extra tokens were computed
+            allowed = np.array(sorted(set(int(r) for r in range(0, w1.nQB, max(1, w1.nQB // 8)))))[:8]
+            toks[:, 2] = (allowed[g.integers(0, len(allowed), m)] * w.q_block +
+                          g.integers(0, w.q_block, m)).clip(max=w.N - 1)
+        t0 = time.perf_counter()
+        oracle.layer_rows(w1, qr, kr, vr, res, toks)
+        t_attn += time.perf_counter() - t0
+        done += m
+        if t_attn > budget_s / 4 or done >= 65536:
+            break
+        m *= 2
+    per_row = t_attn / done
+    layer_s = w.B * w.H * (t_route + (t_extra / max(n_extra, 1)) * w1.nQB) + w.B * w.H * w.N * per_row
+    sample = (f"1 head of {w.B * w.H}: pool + select of all {w1.nQB} query blocks "
+              f"({t_route:.2f} s), attention for {done} sampled query rows ({t_attn:.2f} s)"
+              + (f", extra tokens for {n_extra} query blocks ({t_extra:.2f} s)" if n_extra else "")
+              + "; layer time extrapolated linearly")
+    return {"value": dense_equiv_flops(w) / layer_s / 1e12, "unit": UNIT, "cores": oracle.threads(),
+            "kind": "oracle", "sample": sample, "layer_s_extrapolated": layer_s}
+
+
+def run_reference(args, w, rank, world):
+    """--impl reference: the CPU oracle timed as it stands (rank 0 only)."""
+    if rank != 0:
+        return
+    dev = "cpu"
+    q, k, v = make_qkv(w.replace(B=1, H=1), dev)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(w, q, k, v, budget_s=max(4.0, 60.0 / (args.warmup + args.steps)))
+        if i >= args.warmup:
+            per_step.append(cb["layer_s_extrapolated"])
+    layer_s = statistics.median(per_step)
+    val = dense_equiv_flops(w) / layer_s / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config_json(w, world),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+                             "sample": cb["sample"]},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config_json(w, world):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "dtype": w.dtype,
+            "method": w.method, "q_block": w.q_block, "k_block": w.k_block,
+            "tau": w.tau if w.method == "sol" else None,
+            "keep_percent": w.keep_percent if w.method == "sla" else None,
+            "prefix_len": w.prefix_len, "dense_rows": list(w.dense_rows), "extra_tokens": w.extra_tokens,
+            "centroid": w.centroid, "grid": list(w.grid) if w.grid else None,
+            "parallelism": f"replicas x{world} (heads independent, no collective)",
+            "l2": "inputs larger than L2 (126 MB); no flush" if 3 * w.B * w.N * w.H * w.d * 2 > 126e6
+            else "L2 flushed between steps"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = CONFIGS[args.config]
+    if world > 1:
+        w = w.replace(seed=w.seed + 17 * rank)
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+
+    import block_sparse_attention_26_b200 as bsa
+    from block_sparse_attention_26_b200 import params_for
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    q, k, v = make_qkv(w, dev)
+    p = params_for(w, q)
+    buf = bsa.Buffers(p, dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    l2_flush = None
+    if 3 * q.numel() * q.element_size() <= 126e6:
+        l2_flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if l2_flush is not None:
+            l2_flush.zero_()
+        if ev:
+            ev[0].record(stream)
+        bsa.bsa_pool(p, q, k, v, buf.qbar, buf.kbar, buf.vbar, buf.blk_count, stream)
+        if ev:
+            ev[1].record(stream)
+        bsa.bsa_select(p, buf.qbar, buf.kbar, k, buf.row_ptr, buf.col_idx, buf.kept_count, buf.extra_idx,
+                       buf.extra_count, buf.ws, stream)
+        if ev:
+            ev[2].record(stream)
+        bsa.bsa_attention(p, q, k, v, buf.kbar, buf.vbar, buf.blk_count, buf.row_ptr, buf.col_idx,
+                          buf.extra_idx, buf.extra_count, out, buf.lse, buf.ws, stream)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = bsa.bsa_device_status(buf.ws, stream)
+    if status != 0:
+        raise SystemExit(f"device status {status} after warm-up")
+    flops_kept = kept_flops(w, buf.row_ptr, buf.col_idx)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    total_ms = start.elapsed_time(stop)
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t)
+    status = bsa.bsa_device_status(buf.ws, stream)
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed steps")
+    ph = {"pool": [], "select": [], "attention": []}
+    for e in evs:
+        ph["pool"].append(e[0].elapsed_time(e[1]))
+        ph["select"].append(e[1].elapsed_time(e[2]))
+        ph["attention"].append(e[2].elapsed_time(e[3]))
+    ms_step = total_ms / args.steps
+    attn_ms = statistics.mean(ph["attention"])
+
+    # end to end through the public API with host buffers: H2D of Q/K/V, the
+    # layer, D2H of the output, every step
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for i in range(args.e2e_steps + 1):
+            if i == 1:
+                torch.cuda.synchronize(dev)
+                s0.record(stream)
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            bsa.run_layer(p, dq, dk, dv, out, buf, stream)
+            hout.copy_(out, non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = s0.elapsed_time(s1) / args.e2e_steps
+        if pg:
+            t = torch.tensor([e2e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t)
+        nbytes = q.numel() * q.element_size()
+        e2e = {"value": world * dense_equiv_flops(w) / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms}
+        del hq, hk, hv, hout, dq, dk, dv
+
+    peaks, peak_src = _peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    achieved = flops_kept / (attn_ms * 1e-3) / 1e12
+    per_launch = 2 if w.dense_rows[1] > w.dense_rows[0] else 1
+    launches_per_step = 1 + 4 + per_launch + (2 if w.centroid else 0) + (3 if w.dtype == "f32" else 0)
+    line = {
+        "metric": METRIC,
+        "value": world * dense_equiv_flops(w) / (ms_step * 1e-3) / 1e12,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (smooth Gaussian-filtered fields + noise, seeded)",
+        "config": _config_json(w, world),
+        "ms_per_layer": ms_step,
+        "phases_ms": {k2: statistics.mean(v2) for k2, v2 in ph.items()},
+        "kept_tflop": flops_kept / 1e12,
+        "dense_equiv_tflop": dense_equiv_flops(w) / 1e12,
+        "kept_fraction_of_dense": flops_kept / dense_equiv_flops(w),
+        "roofline": {"bound": "tensor", "kernel": "bsa_attention (fine pass: sparse + centroid + dense rows)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "traffic": None},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k2: v2 for k2, v2 in cpu_baseline(w, q, k, v).items()
+                                if k2 != "layer_s_extrapolated"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -120,6 +120,15 @@ def make_params(q: torch.Tensor, method: str = "sol", *, q_block: Optional[int] 
     return p
 
 
+def params_for(w, q: torch.Tensor) -> bsa_params:
+    """Parameters from any object carrying the method's fields (method, q_block,
+    tau, keep_percent, sink_blocks, keep_diag, prefix_len, dense_rows,
+    extra_tokens, centroid) for query tensor `q`."""
+    return make_params(q, w.method, q_block=w.q_block, tau=w.tau, keep_percent=w.keep_percent,
+                       sink_blocks=w.sink_blocks, keep_diag=w.keep_diag, prefix_len=w.prefix_len,
+                       dense_rows=tuple(w.dense_rows), extra_tokens=w.extra_tokens, centroid=w.centroid)
+
+
 def dims(p: bsa_params):
     nQB = -(-p.N // p.q_block)
     nKB = -(-p.N // p.k_block)

@@ -15,10 +15,7 @@ MEAN_ABS = 2e-3
 EXEMPT_REL = 1e-5
 
 
-def params_for(w, q):
-    return bsa.make_params(q, w.method, q_block=w.q_block, tau=w.tau, keep_percent=w.keep_percent,
-                           sink_blocks=w.sink_blocks, keep_diag=w.keep_diag, prefix_len=w.prefix_len,
-                           dense_rows=w.dense_rows, extra_tokens=w.extra_tokens, centroid=w.centroid)
+params_for = bsa.params_for
 
 
 def gpu_layer(w, q, k, v, capacity=None):

@@ -139,7 +139,7 @@ def make_qkv(w: Workload, device="cpu", layout: str = "bnhd"):
             qv[b].copy_(torch.randn((N, H, d), generator=gq, device=dev))
             kv[b].copy_(torch.randn((N, H, d), generator=gk, device=dev))
             vv[b].copy_(torch.randn((N, H, d), generator=gv, device=dev))
-        return q, k, v
+        return qv, kv, vv
 
     T, Hs, Ws = w.grid
     G = T * Hs * Ws
@@ -158,7 +158,7 @@ def make_qkv(w: Workload, device="cpu", layout: str = "bnhd"):
             qv[b, P:, h].copy_(field + w.noise * eq)
             kv[b, P:, h].copy_(field + w.noise * ek)
             vv[b, P:, h].copy_(ev)
-    return q, k, v
+    return qv, kv, vv
 
 
 def sample_query_blocks(w: Workload, count: int = 64, seed: int = 7):
