@@ -248,12 +248,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--heads", type=int, default=0, help="override H (profiling a smaller case)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = CONFIGS[args.config]
+    if args.heads > 0:
+        w = w.replace(H=args.heads)
     if world > 1:
         w = w.replace(seed=w.seed + 17 * rank)
 

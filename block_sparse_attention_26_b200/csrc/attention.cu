@@ -10,23 +10,32 @@
 // prefix blocks arrive here as kept blocks) and exact_kv_and_rows (designated
 // query rows run dense and replace the sparse result).
 //
-// One CTA computes a tile of 128 query rows of one (batch, head): two 64-row
-// query blocks (Sol, Q64) or one 128-row block (SLA, Q128), so that every
-// tensor-core instruction is a full M = 128 UMMA.  The tile walks the sorted
-// union of its query blocks' kept key blocks, then the centroid chunks; a
-// per-tile row mask tells each row whether a tile is its own.
+// Work items (one CTA each, two CTAs resident per SM):
+//   dense item   128 rows of the dense range x one chunk of the key blocks;
+//                writes an unnormalised partial (O, m, l) that
+//                combine_kernel merges (split over keys so the few dense rows
+//                spread over the whole GPU);
+//   sparse item  128 query rows of one (batch, head): two 64-row query blocks
+//                (Sol, Q64) or one 128-row block (SLA, Q128), so that every
+//                tensor-core instruction is a full M = 128 UMMA.  It walks the
+//                sorted union of its query blocks' kept key blocks, then the
+//                centroid chunks; a per-tile row mask tells each row whether
+//                a tile is its own.
+// Dense items come first in the grid so that they start early.
 //
 // Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S from
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Reads S from
 //              TMEM, masks, online softmax in the log2 domain with a lazily
-//              updated reference max, writes P (bf16) to shared memory, rescales
-//              the TMEM accumulator only when the max grows by > 2^8, and runs
-//              the epilogue O / l -> global.
-//   warp 4     producer: builds the tile list and issues TMA tile loads of K/V
-//              (or of bf16 centroid tiles) into a 3-stage ring.
-//   warp 5     MMA issuer: S = Q K^T (M=128, N=64) into one of two TMEM
-//              S buffers; O += P V (M=128, N=d) into the TMEM accumulator.
-// TMEM: columns [0,64) and [64,128) hold the two S buffers, [128, 128+d) hold O.
+//              updated reference max (the accumulator is rescaled only when the
+//              row max grows by more than 2^8), writes P (bf16) into TMEM and
+//              runs the epilogue.
+//   warp 4     producer: builds the tile list; TMA loads of K and V tiles (or of
+//              bf16 centroid tiles) into separate 2-deep rings; a K slot is
+//              released as soon as its S = Q K^T product is done.
+//   warp 5     MMA issuer: S = Q K^T (M=128, N=64, A and B from shared memory)
+//              and O += P V (M=128, N=d, A = P from TMEM, B = V from shared memory).
+// TMEM (256 columns): S [0,64), P double buffer [64,96) and [96,128) (bf16
+// pairs), O [128, 128+d).
 #include <math.h>
 
 #include <algorithm>
@@ -39,10 +48,12 @@ namespace {
 
 constexpr int kM = 128;        // query rows per tile (UMMA M)
 constexpr int kBK = 64;        // keys per tile (one key block)
-constexpr int kStages = 3;     // K/V ring depth
+constexpr int kKS = 2;         // K ring depth
+constexpr int kVS = 2;         // V ring depth
 constexpr int kThreads = 192;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0, kColP = 64, kColO = 128;
 
 enum : int32_t { TILE_EXACT = 0, TILE_CENT = 1, TILE_END = 2 };
 
@@ -65,8 +76,14 @@ struct AttnArgs {
     float *lse;
     int out_f32;
     int centroid;
-    int dense;                   // 1: rows [row_begin, row_end) over all key blocks
-    int row_begin, row_end;      // dense: rows computed; sparse: rows left to the dense pass
+    int n_sparse;                // sparse items per (b, h)
+    int skip_begin, skip_end;    // sparse tiles fully inside are left to the dense items
+    int dense_begin, dense_end;  // dense rows
+    int n_dense;                 // dense row tiles per (b, h)
+    int dense_split;             // key chunks per dense row tile
+    int split_blocks;            // key blocks per chunk
+    float *part_o;               // [tiles, split, 128, d] unnormalised partial outputs
+    float *part_ml;              // [tiles, split, 128, 2] (m, l) in the log2 domain
     float scale_log2;            // log2(e) / sqrt(d)
     int32_t *status;
 };
@@ -75,15 +92,14 @@ template <int D>
 struct Lay {
     static constexpr int kQBytes = kM * D * 2;
     static constexpr int kKVBytes = kBK * D * 2;
-    static constexpr int kPBytes = kM * kBK * 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
-    static constexpr int kOffV = kOffK + kStages * kKVBytes;
-    static constexpr int kOffP = kOffV + kStages * kKVBytes;
-    static constexpr int kOffInfo = kOffP + 2 * kPBytes;
-    static constexpr int kOffBar = kOffInfo + kStages * (int)sizeof(TileInfo);
-    // q, done, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full[2], p_free[2]
-    static constexpr int kNumBar = 2 + 2 * kStages + 8;
+    static constexpr int kOffV = kOffK + kKS * kKVBytes;
+    static constexpr int kOffKind = kOffV + kVS * kKVBytes;
+    static constexpr int kOffInfo = kOffKind + 16;
+    static constexpr int kOffBar = kOffInfo + kVS * (int)sizeof(TileInfo);
+    // q, done, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full, s_free, p_full[2], p_free[2]
+    static constexpr int kNumBar = 2 + 2 * kKS + 2 * kVS + 2 + 4;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
     static constexpr int kOffMask = kOffMisc + 16;
     static size_t bytes(int nW) { return (size_t)kOffMask + 2 * (size_t)nW * 4 + 1024; }
@@ -97,8 +113,31 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// O[tmem] (+)= A[tmem] * B[smem]: A (M x K, bf16 pairs per 32-bit column) from TMEM.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ float max64(const float (&x)[64])
+{
+    float m[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m[i] = fmaxf(fmaxf(x[4 * i], x[4 * i + 1]), fmaxf(x[4 * i + 2], x[4 * i + 3]));
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+    return m[0];
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
                 const __grid_constant__ CUtensorMap tm_vc, const AttnArgs a)
@@ -107,29 +146,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~(uintptr_t)1023);
-    const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    int row0, row_end;
-    if (a.dense) {
-        row0 = a.row_begin + tile * kM;
-        row_end = a.row_end;
+    // ------------------------------------------------------------ work item
+    int64_t item = blockIdx.x;
+    const int64_t nd_items = (int64_t)a.B * a.H * a.n_dense * a.dense_split;
+    const bool dense = item < nd_items;
+    int bh, row0, nvalid, kb0 = 0, kb1 = 0;
+    int64_t pidx = 0;
+    if (dense) {
+        const int split = (int)(item % a.dense_split);
+        const int64_t tt = item / a.dense_split;          // (bh, tile)
+        const int t = (int)(tt % a.n_dense);
+        bh = (int)(tt / a.n_dense);
+        row0 = a.dense_begin + t * kM;
+        nvalid = min(kM, a.dense_end - row0);
+        kb0 = split * a.split_blocks;
+        kb1 = min(a.nKB, kb0 + a.split_blocks);
+        pidx = tt * a.dense_split + split;
     } else {
+        item -= nd_items;
+        const int tile = (int)(item % a.n_sparse);
+        bh = (int)(item / a.n_sparse);
         row0 = tile * kM;
-        row_end = a.N;
-        if (row0 >= a.row_begin && min(row0 + kM, a.N) <= a.row_end) return;   // all rows dense
+        if (row0 >= a.skip_begin && min(row0 + kM, a.N) <= a.skip_end) return;   // all rows dense
+        nvalid = min(kM, a.N - row0);
     }
-    const int nvalid = min(kM, row_end - row0);
-    if (nvalid <= 0) return;
+    const int b = bh / a.H, h = bh % a.H;
     const int qb0 = row0 / a.Bq;
-    const int nq = a.dense ? 1 : ((a.Bq == 64 && qb0 + 1 < a.nQB) ? 2 : 1);
-    const int64_t rbase = ((int64_t)b * a.H + h) * a.nQB + qb0;
+    const int nq = dense ? 1 : ((a.Bq == 64 && qb0 + 1 < a.nQB) ? 2 : 1);
+    const int64_t rbase = (int64_t)bh * a.nQB + qb0;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kOffBar);
     uint64_t *bar_q = bars, *bar_done = bars + 1;
-    uint64_t *kv_full = bars + 2, *kv_empty = bars + 2 + kStages;
-    uint64_t *s_full = bars + 2 + 2 * kStages, *s_free = s_full + 2, *p_full = s_full + 4,
-             *p_free = s_full + 6;
+    uint64_t *k_full = bars + 2, *k_empty = k_full + kKS;
+    uint64_t *v_full = k_empty + kKS, *v_empty = v_full + kVS;
+    uint64_t *s_full = v_empty + kVS, *s_free = s_full + 1, *p_full = s_full + 2, *p_free = s_full + 4;
+    volatile int32_t *kkind = reinterpret_cast<volatile int32_t *>(sm + L::kOffKind);
     volatile TileInfo *info = reinterpret_cast<volatile TileInfo *>(sm + L::kOffInfo);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kOffMisc);
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(sm + L::kOffMisc + 4);
@@ -138,13 +191,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
         mbar_init(bar_done, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+        for (int s = 0; s < kKS; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
         }
+        for (int s = 0; s < kVS; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 4);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);
             mbar_init(&p_full[i], 4);
             mbar_init(&p_free[i], 1);
         }
@@ -155,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && !a.dense) {
+    if (warp == 4 && !dense) {
         // kept-block bitmasks of the tile's query blocks, from the CSR lists
         for (int w = lane; w < 2 * a.nW; w += 32) kept[w] = 0u;
         __syncwarp();
@@ -182,52 +239,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            prefetch_tmap(&tm_kc);
-            prefetch_tmap(&tm_vc);
+            if (!dense && a.centroid) {
+                prefetch_tmap(&tm_kc);
+                prefetch_tmap(&tm_vc);
+            }
             mbar_expect_tx(bar_q, L::kQBytes);
             for (int dc = 0; dc < D / 64; ++dc)
                 tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
             int j = 0;
-            int issued[kStages] = {};
-            bool ok = true;
+            int kiss[kKS] = {}, viss[kVS] = {};
             auto push = [&](int kind, int blk, uint32_t who, int ncols, float last_bias, uint64_t m0,
                             uint64_t m1) -> bool {
-                const int s = j % kStages;
-                if (j >= kStages &&
-                    !mbar_wait(&kv_empty[s], ((j / kStages) - 1) & 1, abort_flag, a.status, 10))
+                const int ks = j % kKS, vs = j % kVS;
+                if (j >= kKS && !mbar_wait(&k_empty[ks], ((j / kKS) - 1) & 1, abort_flag, a.status, 10))
                     return false;
-                info[s].kind = kind;
-                info[s].blk = blk;
-                info[s].who = who;
-                info[s].ncols = ncols;
-                info[s].last_bias = last_bias;
-                info[s].cmask[0] = m0;
-                info[s].cmask[1] = m1;
-                uint8_t *kd = sm + L::kOffK + s * L::kKVBytes;
-                uint8_t *vd = sm + L::kOffV + s * L::kKVBytes;
+                kkind[ks] = kind;
+                uint8_t *kd = sm + L::kOffK + ks * L::kKVBytes;
                 if (kind == TILE_EXACT) {
-                    mbar_expect_tx(&kv_full[s], 2 * L::kKVBytes);
-                    for (int dc = 0; dc < D / 64; ++dc) {
-                        tma_load_4d(kd + dc * (kBK * 128), &tm_k, &kv_full[s], dc * 64, h, blk * kBK, b);
-                        tma_load_4d(vd + dc * (kBK * 128), &tm_v, &kv_full[s], dc * 64, h, blk * kBK, b);
-                    }
+                    mbar_expect_tx(&k_full[ks], L::kKVBytes);
+                    for (int dc = 0; dc < D / 64; ++dc)
+                        tma_load_4d(kd + dc * (kBK * 128), &tm_k, &k_full[ks], dc * 64, h, blk * kBK, b);
                 } else if (kind == TILE_CENT) {
-                    mbar_expect_tx(&kv_full[s], 2 * L::kKVBytes);
-                    const int bh = b * a.H + h;
-                    for (int dc = 0; dc < D / 64; ++dc) {
-                        tma_load_3d(kd + dc * (kBK * 128), &tm_kc, &kv_full[s], dc * 64, blk * kBK, bh);
-                        tma_load_3d(vd + dc * (kBK * 128), &tm_vc, &kv_full[s], dc * 64, blk * kBK, bh);
-                    }
+                    mbar_expect_tx(&k_full[ks], L::kKVBytes);
+                    for (int dc = 0; dc < D / 64; ++dc)
+                        tma_load_3d(kd + dc * (kBK * 128), &tm_kc, &k_full[ks], dc * 64, blk * kBK, bh);
                 } else {
-                    mbar_arrive(&kv_full[s]);
+                    mbar_arrive(&k_full[ks]);
                 }
-                issued[s]++;
+                kiss[ks]++;
+                if (j >= kVS && !mbar_wait(&v_empty[vs], ((j / kVS) - 1) & 1, abort_flag, a.status, 11))
+                    return false;
+                info[vs].kind = kind;
+                info[vs].blk = blk;
+                info[vs].who = who;
+                info[vs].ncols = ncols;
+                info[vs].last_bias = last_bias;
+                info[vs].cmask[0] = m0;
+                info[vs].cmask[1] = m1;
+                uint8_t *vd = sm + L::kOffV + vs * L::kKVBytes;
+                if (kind == TILE_EXACT) {
+                    mbar_expect_tx(&v_full[vs], L::kKVBytes);
+                    for (int dc = 0; dc < D / 64; ++dc)
+                        tma_load_4d(vd + dc * (kBK * 128), &tm_v, &v_full[vs], dc * 64, h, blk * kBK, b);
+                } else if (kind == TILE_CENT) {
+                    mbar_expect_tx(&v_full[vs], L::kKVBytes);
+                    for (int dc = 0; dc < D / 64; ++dc)
+                        tma_load_3d(vd + dc * (kBK * 128), &tm_vc, &v_full[vs], dc * 64, blk * kBK, bh);
+                } else {
+                    mbar_arrive(&v_full[vs]);
+                }
+                viss[vs]++;
                 ++j;
                 return true;
             };
+            bool ok = true;
             const int last_n = a.N - (a.nKB - 1) * kBK;
-            if (a.dense) {
-                for (int blk = 0; blk < a.nKB && ok; ++blk)
+            if (dense) {
+                for (int blk = kb0; blk < kb1 && ok; ++blk)
                     ok = push(TILE_EXACT, blk, 3u, min(kBK, a.N - blk * kBK), 0.f, 0, 0);
             } else {
                 const uint32_t *k0 = kept, *k1 = kept + a.nW;
@@ -263,14 +331,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (ok) ok = push(TILE_END, 0, 0u, 0, 0.f, 0, 0);
-            // make sure no TMA write is still in flight before the CTA can exit
-            for (int s = 0; s < kStages; ++s)
-                if (issued[s] > 0) {
-                    volatile int32_t no_abort = 0;
-                    mbar_wait(&kv_full[s], (issued[s] - 1) & 1, &no_abort, a.status, 11);
-                }
+            // no TMA write may still be in flight when the CTA exits
             volatile int32_t no_abort = 0;
-            mbar_wait(bar_q, 0, &no_abort, a.status, 12);
+            for (int s = 0; s < kKS; ++s)
+                if (kiss[s] > 0) mbar_wait(&k_full[s], (kiss[s] - 1) & 1, &no_abort, a.status, 12);
+            for (int s = 0; s < kVS; ++s)
+                if (viss[s] > 0) mbar_wait(&v_full[s], (viss[s] - 1) & 1, &no_abort, a.status, 13);
+            mbar_wait(bar_q, 0, &no_abort, a.status, 14);
         }
     } else if (warp == 5) {
         // ---------------------------------------------------------- MMA issuer
@@ -280,98 +347,95 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t q_addr = smem_u32(sm + L::kOffQ);
             const uint32_t k_addr = smem_u32(sm + L::kOffK);
             const uint32_t v_addr = smem_u32(sm + L::kOffV);
-            const uint32_t p_addr = smem_u32(sm + L::kOffP);
             auto issue_pv = [&](int t) -> bool {
-                const int pb = t & 1, s = t % kStages;
-                if (!mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag, a.status, 20)) return false;
+                const int pb = t & 1, vs = t % kVS;
+                if (!mbar_wait(&v_full[vs], (t / kVS) & 1, abort_flag, a.status, 20)) return false;
+                if (!mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag, a.status, 21)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < kBK / 16; ++ks) {
-                    const uint64_t ad = sdesc_sw128(p_addr + pb * L::kPBytes + ks * 32, 16, 1024);
-                    const uint64_t bd =
-                        sdesc_sw128(v_addr + s * L::kKVBytes + ks * 2048, kBK * 128, 1024);
-                    umma_bf16(tmem + 128, ad, bd, idesc_o, (t > 0 || ks > 0) ? 1u : 0u);
+                    const uint64_t bd = sdesc_sw128(v_addr + vs * L::kKVBytes + ks * 2048, kBK * 128, 1024);
+                    umma_bf16_ts(tmem + kColO, tmem + kColP + 32 * pb + 8 * ks, bd, idesc_o,
+                                 (t > 0 || ks > 0) ? 1u : 0u);
                 }
-                umma_commit(&kv_empty[s]);
+                umma_commit(&v_empty[vs]);
                 umma_commit(&p_free[pb]);
                 return true;
             };
-            bool ok = mbar_wait(bar_q, 0, abort_flag, a.status, 21);
+            bool ok = mbar_wait(bar_q, 0, abort_flag, a.status, 22);
             tc_fence_after();
             int j = 0;
             while (ok) {
-                const int s = j % kStages;
-                if (!(ok = mbar_wait(&kv_full[s], (j / kStages) & 1, abort_flag, a.status, 22))) break;
+                const int ks = j % kKS;
+                if (!(ok = mbar_wait(&k_full[ks], (j / kKS) & 1, abort_flag, a.status, 23))) break;
                 tc_fence_after();
-                if (info[s].kind == TILE_END) break;
-                const int sb = j & 1;
-                if (j >= 2 && !(ok = mbar_wait(&s_free[sb], ((j >> 1) - 1) & 1, abort_flag, a.status, 23)))
-                    break;
+                if (kkind[ks] == TILE_END) break;
+                if (j >= 1 && !(ok = mbar_wait(s_free, (j - 1) & 1, abort_flag, a.status, 24))) break;
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ad =
-                        sdesc_sw128(q_addr + (ks >> 2) * (kM * 128) + (ks & 3) * 32, 16, 1024);
+                        sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd = sdesc_sw128(
-                        k_addr + s * L::kKVBytes + (ks >> 2) * (kBK * 128) + (ks & 3) * 32, 16, 1024);
-                    umma_bf16(tmem + sb * kBK, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+                        k_addr + ks * L::kKVBytes + (kk >> 2) * (kBK * 128) + (kk & 3) * 32, 16, 1024);
+                    umma_bf16(tmem + kColS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_full[sb]);
+                umma_commit(s_full);
+                umma_commit(&k_empty[ks]);
                 if (j >= 1 && !(ok = issue_pv(j - 1))) break;
                 ++j;
             }
             if (ok && j >= 1) ok = issue_pv(j - 1);
-            if (ok) umma_commit(&s_full[j & 1]);      // end-of-list marker for the softmax warps
-            // wait for every MMA this thread issued before TMEM can be released
+            if (ok) umma_commit(s_full);      // end-of-list marker for the softmax warps
             umma_commit(bar_done);
             volatile int32_t no_abort = 0;
-            mbar_wait(bar_done, 0, &no_abort, a.status, 24);
+            mbar_wait(bar_done, 0, &no_abort, a.status, 25);
         }
     } else {
         // ---------------------------------------------------------- softmax
         const int r = threadIdx.x;                               // tile row == TMEM lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const int qsel = (a.Bq == 64 && !a.dense) ? (r >> 6) : 0;
+        const int qsel = (a.Bq == 64 && !dense) ? (r >> 6) : 0;
         const float scale = a.scale_log2;
-        const uint32_t p_row = smem_u32(sm + L::kOffP) + (r >> 3) * 1024 + (r & 7) * 128;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         int j = 0;
         for (;; ++j) {
-            const int sb = j & 1, s = j % kStages;
-            ok = mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag, a.status, 30) &&
-                 mbar_wait(&kv_full[s], (j / kStages) & 1, abort_flag, a.status, 31);
+            const int vs = j % kVS;
+            ok = mbar_wait(s_full, j & 1, abort_flag, a.status, 30) &&
+                 mbar_wait(&v_full[vs], (j / kVS) & 1, abort_flag, a.status, 31);
             if (!(ok = __all_sync(0xffffffffu, ok))) break;
             tc_fence_after();
-            const int kind = info[s].kind;
+            const int kind = info[vs].kind;
             if (kind == TILE_END) break;
-            uint32_t sr[64];
-            tmem_ld32(tmem + lane_base + sb * kBK, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(tmem + lane_base + sb * kBK + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+            float s[64];
+            tmem_ld32(tmem + lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+            tmem_ld32(tmem + lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[sb]);
+            if (lane == 0) mbar_arrive(s_free);
 
-            float x[64];
+            bool fast = false;
             if (kind == TILE_EXACT) {
-                const bool act = (info[s].who >> qsel) & 1u;
-                const int nc = act ? info[s].ncols : 0;
+                const bool act = (info[vs].who >> qsel) & 1u;
+                const int nc = act ? info[vs].ncols : 0;
+                fast = nc == kBK;
+                if (!fast) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) x[c] = c < nc ? __uint_as_float(sr[c]) * scale : -INFINITY;
+                    for (int c = 0; c < 64; ++c) s[c] = c < nc ? s[c] * scale : -INFINITY;
+                }
             } else {
-                const uint64_t msk = info[s].cmask[qsel];
-                const int pc = info[s].ncols;
-                const float pbias = info[s].last_bias;
+                const uint64_t msk = info[vs].cmask[qsel];
+                const int pc = info[vs].ncols;
+                const float pbias = info[vs].last_bias;
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const float bias = c == pc ? pbias : 6.0f;       // log2(64) for full blocks
-                    x[c] = ((msk >> c) & 1ull) ? fmaf(__uint_as_float(sr[c]), scale, bias) : -INFINITY;
+                    s[c] = ((msk >> c) & 1ull) ? fmaf(s[c], scale, bias) : -INFINITY;
                 }
             }
-            float mt = x[0];
-#pragma unroll
-            for (int c = 1; c < 64; ++c) mt = fmaxf(mt, x[c]);
+            const float mt = fast ? max64(s) * scale : max64(s);
             float alpha = 1.f;
             bool rescale = false;
             if (mt > m_ref) {
@@ -386,24 +450,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float mref = m_ref == -INFINITY ? 0.f : m_ref;
             uint32_t pk[32];
-            float rs = 0.f;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (fast) {
+                const float nm = -mref;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float p0 = ex2(x[2 * c] - mref);
-                const float p1 = ex2(x[2 * c + 1] - mref);
-                rs += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2(fmaf(s[2 * c], scale, nm));
+                    const float p1 = ex2(fmaf(s[2 * c + 1], scale, nm));
+                    acc[c & 3] += p0 + p1;
+                    pk[c] = pack_bf16x2(p0, p1);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2(s[2 * c] - mref);
+                    const float p1 = ex2(s[2 * c + 1] - mref);
+                    acc[c & 3] += p0 + p1;
+                    pk[c] = pack_bf16x2(p0, p1);
+                }
             }
-            l += rs;
+            l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
             if (j >= 2) {
-                ok = mbar_wait(&p_free[sb], ((j >> 1) - 1) & 1, abort_flag, a.status, 32);
+                ok = mbar_wait(&p_free[j & 1], ((j >> 1) - 1) & 1, abort_flag, a.status, 32);
                 if (!(ok = __all_sync(0xffffffffu, ok))) break;
             }
-            const uint32_t pbase = p_row + sb * L::kPBytes;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(pbase + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-                             pk[4 * c + 3]);
+            tmem_st32(tmem + lane_base + kColP + 32 * (j & 1), pk);
             if (__any_sync(0xffffffffu, rescale)) {
                 // the accumulator must hold every earlier P V product before it is scaled
                 ok = mbar_wait(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status, 33);
@@ -412,18 +483,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t o[32];
-                    tmem_ld32(tmem + lane_base + 128 + cc * 32, o);
+                    tmem_ld32(tmem + lane_base + kColO + cc * 32, o);
                     tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(tmem + lane_base + 128 + cc * 32, o);
+                    tmem_st32(tmem + lane_base + kColO + cc * 32, o);
                 }
-                tmem_st_wait();
             }
-            fence_async_smem();
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[sb]);
+            if (lane == 0) mbar_arrive(&p_full[j & 1]);
         }
         const int T = j;
         if (ok && T >= 1)
@@ -433,36 +503,60 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             const bool row_ok = r < nvalid;
             const int n = row0 + r;
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
             const bool have_o = T >= 1 && l > 0.f;
+            if (dense && a.dense_split > 1) {
+                // unnormalised partial in the frame of m_ref, merged by combine_kernel
+                float *po = a.part_o + (pidx * kM + r) * D;
 #pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[32];
-                __syncwarp();
-                tmem_ld32(tmem + lane_base + 128 + cc * 32, o);
-                tmem_ld_wait();
-                if (!row_ok) continue;
-                float v[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = have_o ? __uint_as_float(o[e]) * inv_l : 0.f;
-                const int64_t off = (int64_t)b * a.sb + (int64_t)n * a.sn + (int64_t)h * a.sh + cc * 32;
-                if (a.out_f32) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + off);
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    __syncwarp();
+                    tmem_ld32(tmem + lane_base + kColO + cc * 32, o);
+                    tmem_ld_wait();
+                    float4 *dst = reinterpret_cast<float4 *>(po + cc * 32);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-                } else {
-                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + off);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]), pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
-                                            pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
-                                            pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+                        dst[e] = have_o ? make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                                      __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
+                float *ml = a.part_ml + (pidx * kM + r) * 2;
+                ml[0] = have_o ? m_ref : -INFINITY;
+                ml[1] = have_o ? l : 0.f;
+            } else {
+                // a sparse item leaves rows of the dense range to the dense items
+                const bool mine = row_ok && (dense || n < a.dense_begin || n >= a.dense_end);
+                const float inv_l = have_o ? 1.f / l : 0.f;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    __syncwarp();
+                    tmem_ld32(tmem + lane_base + kColO + cc * 32, o);
+                    tmem_ld_wait();
+                    if (!mine) continue;
+                    float v[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = have_o ? __uint_as_float(o[e]) * inv_l : 0.f;
+                    const int64_t off = (int64_t)b * a.sb + (int64_t)n * a.sn + (int64_t)h * a.sh + cc * 32;
+                    if (a.out_f32) {
+                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + off);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+                    } else {
+                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + off);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]),
+                                                pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
+                                                pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
+                                                pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+                    }
+                }
+                if (mine && a.lse != nullptr)
+                    a.lse[(int64_t)bh * a.N + n] =
+                        have_o ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
             }
-            if (row_ok && a.lse != nullptr)
-                a.lse[((int64_t)b * a.H + h) * a.N + n] =
-                    l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
         }
     }
 
@@ -474,7 +568,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// bf16 copies of f32 centroids (or of f32 inputs): elementwise, grid-stride.
+// Merge the key-chunk partials of the dense rows: one thread per row.
+__global__ void __launch_bounds__(128) combine_kernel(AttnArgs a, int d)
+{
+    const int64_t tt = blockIdx.x;                 // (bh, tile)
+    const int r = threadIdx.x;
+    const int t = (int)(tt % a.n_dense);
+    const int bh = (int)(tt / a.n_dense);
+    const int b = bh / a.H, h = bh % a.H;
+    const int n = a.dense_begin + t * kM + r;
+    if (n >= a.dense_end) return;
+    const int S = a.dense_split;
+    float m = -INFINITY;
+    for (int s = 0; s < S; ++s) m = fmaxf(m, a.part_ml[((tt * S + s) * kM + r) * 2]);
+    float l = 0.f;
+    for (int s = 0; s < S; ++s) {
+        const float *ml = a.part_ml + ((tt * S + s) * kM + r) * 2;
+        if (ml[0] > -INFINITY) l += ml[1] * exp2f(ml[0] - m);
+    }
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    const int64_t off = (int64_t)b * a.sb + (int64_t)n * a.sn + (int64_t)h * a.sh;
+    for (int c0 = 0; c0 < d; c0 += 4) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < S; ++s) {
+            const float ms = a.part_ml[((tt * S + s) * kM + r) * 2];
+            if (!(ms > -INFINITY)) continue;
+            const float w = exp2f(ms - m) * inv_l;
+            const float4 o = *reinterpret_cast<const float4 *>(a.part_o + ((tt * S + s) * kM + r) * d + c0);
+            acc.x += w * o.x;
+            acc.y += w * o.y;
+            acc.z += w * o.z;
+            acc.w += w * o.w;
+        }
+        if (a.out_f32) {
+            *reinterpret_cast<float4 *>(static_cast<float *>(a.out) + off + c0) = acc;
+        } else {
+            uint2 pk = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.out) + off + c0) = pk;
+        }
+    }
+    if (a.lse != nullptr)
+        a.lse[(int64_t)bh * a.N + n] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+}
+
+// bf16 copies of f32 centroids: elementwise, grid-stride.
 __global__ void to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst, int64_t n)
 {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -550,22 +687,35 @@ bool make_map_cent(CUtensorMap *m, const void *base, int BH, int nKB, int d)
 
 template <int D>
 cudaError_t launch_attn_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                               const CUtensorMap &tkc, const CUtensorMap &tvc, const AttnArgs &a, int tiles,
+                               const CUtensorMap &tkc, const CUtensorMap &tvc, const AttnArgs &a, int64_t items,
                                cudaStream_t st)
 {
     const size_t smem = Lay<D>::bytes(a.nW);
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)tiles, (unsigned)a.H, (unsigned)a.B);
-    attn_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, a);
+    attn_kernel<D><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t attention_smem_bytes(int d, int nW)
+// Key-chunk split of the dense rows: enough items to cover the GPU, chunks of
+// at least 256 key blocks, bounded by `max_partials` partial tiles.
+int dense_split_for(const Dims &D, int nrows, int64_t max_partials)
 {
-    return d == 64 ? Lay<64>::bytes(nW) : Lay<128>::bytes(nW);
+    if (nrows <= 0) return 1;
+    const int64_t tiles = (int64_t)D.B * D.H * ceil_div(nrows, kM);
+    if (tiles >= 2 * 148) return 1;
+    int split = (int)std::min<int64_t>(ceil_div(D.nKB, 256), ceil_div(2 * 148, tiles));
+    split = std::max(1, split);
+    while (split > 1 && tiles * split > max_partials) --split;
+    return split;
+}
+
+int64_t dense_partial_tiles(const Dims &D, int nrows)
+{
+    const int split = dense_split_for(D, nrows, INT64_MAX);
+    return split > 1 ? (int64_t)D.B * D.H * ceil_div(nrows, kM) * split : 0;
 }
 
 cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, const void *k,
@@ -632,23 +782,25 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     a.centroid = p.centroid;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D.d));
     a.status = reinterpret_cast<int32_t *>(ws + L.status);
-    cudaError_t e = cudaSuccess;
-    if (!dense_only) {
-        a.dense = 0;
-        a.row_begin = p.dense_row_begin;
-        a.row_end = p.dense_row_end;
-        const int tiles = (int)ceil_div(D.N, kM);
-        e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, a, tiles, st)
-                      : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, a, tiles, st);
-        if (e != cudaSuccess) return e;
-    }
-    if (row_end > row_begin) {
-        a.dense = 1;
-        a.row_begin = row_begin;
-        a.row_end = row_end;
-        const int tiles = (int)ceil_div(row_end - row_begin, kM);
-        e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, a, tiles, st)
-                      : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, a, tiles, st);
+    a.n_sparse = dense_only ? 0 : (int)ceil_div(D.N, kM);
+    a.skip_begin = row_begin;
+    a.skip_end = row_end;
+    const int nrows = std::max(0, row_end - row_begin);
+    a.dense_begin = row_begin;
+    a.dense_end = row_end;
+    a.n_dense = (int)ceil_div(nrows, kM);
+    a.dense_split = dense_split_for(D, nrows, L.part_tiles);
+    a.split_blocks = (int)ceil_div(D.nKB, a.dense_split);
+    a.part_o = reinterpret_cast<float *>(ws + L.part_o);
+    a.part_ml = reinterpret_cast<float *>(ws + L.part_ml);
+    const int64_t items = (int64_t)BH * (a.n_dense * (int64_t)a.dense_split + a.n_sparse);
+    if (items == 0) return cudaSuccess;
+    cudaError_t e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, a, items, st)
+                              : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, a, items, st);
+    if (e != cudaSuccess) return e;
+    if (a.n_dense > 0 && a.dense_split > 1) {
+        combine_kernel<<<(unsigned)(BH * (int64_t)a.n_dense), kM, 0, st>>>(a, D.d);
+        e = cudaGetLastError();
     }
     return e;
 }

@@ -61,6 +61,9 @@ WsLayout ws_layout(const bsa_params &p)
     L.q16 = take(in16);
     L.k16 = take(in16);
     L.v16 = take(in16);
+    L.part_tiles = dense_partial_tiles(D, p.dense_row_end - p.dense_row_begin);
+    L.part_o = take((size_t)L.part_tiles * 128 * D.d * sizeof(float));
+    L.part_ml = take((size_t)L.part_tiles * 128 * 2 * sizeof(float));
     L.total = off;
     return L;
 }

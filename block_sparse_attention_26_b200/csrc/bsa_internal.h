@@ -33,10 +33,18 @@ struct WsLayout {
     size_t cbias;          // [rows, nKB_pad] f32 per-row centroid bias overrides (extra tokens)
     size_t xk16, xv16;     // [rows, E, d] bf16 modified centroids (extra tokens)
     size_t q16, k16, v16;  // [B, N, H, d] bf16 copies of f32 inputs (attention, f32 only)
+    size_t part_o;         // [part_tiles, 128, d] f32 dense-row partial outputs
+    size_t part_ml;        // [part_tiles, 128, 2] f32 dense-row partial (max, sum)
+    int64_t part_tiles;    // capacity of the partial buffers, in 128-row tiles
     size_t total;
 };
 
 WsLayout ws_layout(const bsa_params &p);
+
+// Key-chunk split of `nrows` dense rows (1 = no split), limited to max_partials tiles.
+int dense_split_for(const Dims &D, int nrows, int64_t max_partials);
+// Partial tiles the dense rows of a parameter set need (0 if they are not split).
+int64_t dense_partial_tiles(const Dims &D, int nrows);
 
 cudaError_t launch_pool(const bsa_params &p, const Dims &D, const void *q, const void *k,
                         const void *v, float *qbar, float *kbar, float *vbar, int32_t *blk_count,

@@ -33,6 +33,9 @@ SMALL = {
                              seed=16),
     "single_block": Workload("single_block", B=1, H=2, N=40, d=128, dtype="bf16", method="sol", q_block=64,
                              k_block=64, tau=1.0, grid=(1, 5, 8), seed=17),
+    "dense_split": Workload("dense_split", B=1, H=1, N=20032, d=128, dtype="bf16", method="sol", q_block=64,
+                            k_block=64, tau=1.5, prefix_len=256, dense_rows=(100, 300), grid=(4, 24, 206),
+                            seed=20),
     "no_diag_no_sink": Workload("no_diag_no_sink", B=1, H=2, N=1300, d=128, dtype="bf16", method="sol",
                                 q_block=64, k_block=64, tau=1.0, sink_blocks=0, keep_diag=0,
                                 grid=(2, 13, 50), seed=18),
