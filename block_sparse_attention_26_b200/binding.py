@@ -14,7 +14,8 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libbsa.so")
+# BSA_LIBRARY may name another build of the same library (e.g. a debug build).
+LIB_PATH = os.environ.get("BSA_LIBRARY") or os.path.join(_PKG, "libbsa.so")
 
 BSA_OK = 0
 BSA_ERR_INVALID_ARG = 1

@@ -10,32 +10,37 @@
 // prefix blocks arrive here as kept blocks) and exact_kv_and_rows (designated
 // query rows run dense and replace the sparse result).
 //
-// Work items (one CTA each, two CTAs resident per SM):
+// Work items (one CTA each, one CTA per SM):
 //   dense item   128 rows of the dense range x one chunk of the key blocks;
-//                writes an unnormalised partial (O, m, l) that
-//                combine_kernel merges (split over keys so the few dense rows
-//                spread over the whole GPU);
+//                with more than one chunk it writes an unnormalised partial
+//                (O, m, l) that combine_kernel merges, so that the few dense
+//                rows spread over the whole GPU;
 //   sparse item  128 query rows of one (batch, head): two 64-row query blocks
 //                (Sol, Q64) or one 128-row block (SLA, Q128), so that every
-//                tensor-core instruction is a full M = 128 UMMA.  It walks the
-//                sorted union of its query blocks' kept key blocks, then the
-//                centroid chunks; a per-tile row mask tells each row whether
-//                a tile is its own.
+//                tensor-core instruction has M = 128.  It walks the sorted union
+//                of its query blocks' kept key blocks, then the centroid chunks.
 // Dense items come first in the grid so that they start early.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r).  Reads S from
-//              TMEM, masks, online softmax in the log2 domain with a lazily
-//              updated reference max (the accumulator is rescaled only when the
-//              row max grows by more than 2^8), writes P (bf16) into TMEM and
-//              runs the epilogue.
-//   warp 4     producer: builds the tile list; TMA loads of K and V tiles (or of
-//              bf16 centroid tiles) into separate 2-deep rings; a K slot is
-//              released as soon as its S = Q K^T product is done.
-//   warp 5     MMA issuer: S = Q K^T (M=128, N=64, A and B from shared memory)
-//              and O += P V (M=128, N=d, A = P from TMEM, B = V from shared memory).
-// TMEM (256 columns): S [0,64), P double buffer [64,96) and [96,128) (bf16
-// pairs), O [128, 128+d).
+// A tile is 128 keys: two key blocks (or two chunks of 64 centroids) loaded
+// into the two halves of the K and V tiles, so that S = Q K^T is an N = 128
+// UMMA (N = 64 UMMAs run at two thirds of the rate).  Softmax warpgroup h owns
+// the tile's half h -- one key block -- with its own online softmax state and
+// its own accumulator O_h; the halves are merged in the epilogue.
+//
+// Warp roles (320 threads):
+//   warps 0-3, 4-7  softmax warpgroups h = 0, 1: thread r owns query row r
+//              (TMEM lane r).  Read S from TMEM, mask, online softmax in the log2
+//              domain with a lazily updated reference max (the accumulator is
+//              rescaled only when the row max grows by more than 2^8), write P
+//              (bf16) into TMEM, and run the epilogue.
+//   warp 8     producer: builds the tile list; TMA loads of K and V tiles (or of
+//              bf16 centroid tiles) into separate rings; a K slot is released as
+//              soon as its S product is done.
+//   warp 9     MMA issuer (one thread, event loop): S = Q K^T (A and B from
+//              shared memory) runs ahead of the softmax; O_h += P_h V_h (A = P_h
+//              from TMEM) is issued as soon as half h of a tile's P is in.
+// TMEM (512 columns): S [0,128); P of half h, buffer b at 128 + 64 h + 32 b;
+// O_h at 256 + 128 h.
 #include <math.h>
 
 #include <algorithm>
@@ -47,24 +52,43 @@ namespace bsa {
 namespace {
 
 constexpr int kM = 128;        // query rows per tile (UMMA M)
-constexpr int kBK = 64;        // keys per tile (one key block)
-constexpr int kKS = 2;         // K ring depth
-constexpr int kVS = 2;         // V ring depth
-constexpr int kThreads = 192;
+constexpr int kBK = 64;        // keys per key block
+constexpr int kTK = 128;       // keys per tile (two blocks)
+constexpr int kKS = 2;         // K ring depth (tiles)
+constexpr int kVS = 3;         // V ring depth (tiles)
+constexpr int kThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
 constexpr float kRescaleLog2 = 8.0f;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColP = 64, kColO = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;          // S, 128 columns
+constexpr uint32_t kColP = 128;        // P of half h, buffer b at kColP + 64 h + 32 b
+constexpr uint32_t kColO = 256;        // O of half h at kColO + 128 h
 
 enum : int32_t { TILE_EXACT = 0, TILE_CENT = 1, TILE_END = 2 };
 
+#ifdef BSA_TRACE
+// Per-tile clock64() stamps of a few CTAs (development builds only), kept in
+// shared memory while the CTA runs and copied out at its end.
+constexpr int kTraceCtas = 8, kTraceTiles = 64, kTraceEvents = 16;
+constexpr int kTraceBytes = kTraceTiles * kTraceEvents * 8;
+#define TRACE(ev, j)                                                                       \
+    do {                                                                                   \
+        if ((j) < kTraceTiles) trace_sm[(ev) * kTraceTiles + (j)] = clock64();              \
+    } while (0)
+#else
+constexpr int kTraceBytes = 0;
+#define TRACE(ev, j) ((void)0)
+#endif
+
+// What one 128-key tile holds; half h is one key block (or 64 centroids).
 struct TileInfo {
     int32_t kind;
-    int32_t blk;          // key block (exact) or centroid chunk of 64 blocks (centroid)
-    uint32_t who;         // exact: bit q set = query block q of the tile keeps the block
-    int32_t ncols;        // exact: valid key columns; centroid: column of a partial block or -1
+    int32_t blk[2];       // key block of each half (exact) or centroid chunk (centroid)
+    uint32_t who[2];      // exact: bit q set = query block q of the tile keeps the half's block
+    int32_t ncols[2];     // exact: valid key columns of each half (0 = empty half)
+    int32_t pcol[2];      // centroid: column of a partial block in each half, or -1
     float last_bias;      // centroid: log2 of the partial block's size
-    int32_t pad[3];
-    uint64_t cmask[2];    // centroid: active centroid columns for query block 0 / 1
+    int32_t pad;
+    uint64_t cmask[2][2]; // centroid: [query block][half] active centroid columns
 };
 
 struct AttnArgs {
@@ -86,23 +110,34 @@ struct AttnArgs {
     float *part_ml;              // [tiles, split, 128, 2] (m, l) in the log2 domain
     float scale_log2;            // log2(e) / sqrt(d)
     int32_t *status;
+    long long *trace;            // development builds: per-tile timestamps
+    int trace_base;
 };
 
 template <int D>
 struct Lay {
     static constexpr int kQBytes = kM * D * 2;
-    static constexpr int kKVBytes = kBK * D * 2;
+    static constexpr int kTileBytes = kTK * D * 2;              // one K or V tile (128 keys)
+    static constexpr int kHalfBytes = kBK * 128;                // one 64-key box of one channel chunk
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
-    static constexpr int kOffV = kOffK + kKS * kKVBytes;
-    static constexpr int kOffKind = kOffV + kVS * kKVBytes;
+    static constexpr int kOffV = kOffK + kKS * kTileBytes;
+    static constexpr int kOffKind = kOffV + kVS * kTileBytes;
     static constexpr int kOffInfo = kOffKind + 16;
     static constexpr int kOffBar = kOffInfo + kVS * (int)sizeof(TileInfo);
-    // q, done, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full, s_free, p_full[2], p_free[2]
-    static constexpr int kNumBar = 2 + 2 * kKS + 2 * kVS + 2 + 4;
+    // q, done, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full, s_free,
+    // p_full[2 halves][2], p_free[2 halves][2]
+    static constexpr int kNumBar = 2 + 2 * kKS + 2 * kVS + 2 + 8;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
-    static constexpr int kOffMask = kOffMisc + 16;
-    static size_t bytes(int nW) { return (size_t)kOffMask + 2 * (size_t)nW * 4 + 1024; }
+    static constexpr int kOffML = kOffMisc + 16;                 // [2][128] (m, l) per half
+    static constexpr int kOffTrace = kOffML + 2 * kM * 8;
+    static constexpr int kOffMask = kOffTrace + kTraceBytes;
+    // at least 116 KB so that a single CTA owns an SM (it allocates all 512 TMEM columns)
+    static size_t bytes(int nW)
+    {
+        const size_t b = (size_t)kOffMask + 2 * (size_t)nW * 4 + 1024;
+        return b < 116 * 1024 ? 116 * 1024 : b;
+    }
 };
 
 // 2^x on the MUFU unit (ex2.approx, relative error ~2^-22; 2^-inf = +0).
@@ -136,8 +171,13 @@ __device__ __forceinline__ float max64(const float (&x)[64])
     return m[0];
 }
 
+__device__ __forceinline__ void named_bar(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
                 const __grid_constant__ CUtensorMap tm_vc, const AttnArgs a)
@@ -181,12 +221,19 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t *bar_q = bars, *bar_done = bars + 1;
     uint64_t *k_full = bars + 2, *k_empty = k_full + kKS;
     uint64_t *v_full = k_empty + kKS, *v_empty = v_full + kVS;
-    uint64_t *s_full = v_empty + kVS, *s_free = s_full + 1, *p_full = s_full + 2, *p_free = s_full + 4;
+    uint64_t *s_full = v_empty + kVS, *s_free = s_full + 1;
+    uint64_t *p_full = s_free + 1;            // [half * 2 + buffer]
+    uint64_t *p_free = p_full + 4;            // [half * 2 + buffer]
     volatile int32_t *kkind = reinterpret_cast<volatile int32_t *>(sm + L::kOffKind);
     volatile TileInfo *info = reinterpret_cast<volatile TileInfo *>(sm + L::kOffInfo);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kOffMisc);
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(sm + L::kOffMisc + 4);
+    float2 *ml = reinterpret_cast<float2 *>(sm + L::kOffML);   // [2 halves][128] (m, l)
     uint32_t *kept = reinterpret_cast<uint32_t *>(sm + L::kOffMask);
+#ifdef BSA_TRACE
+    long long *trace_sm = reinterpret_cast<long long *>(sm + L::kOffTrace);
+    for (int i = threadIdx.x; i < kTraceTiles * kTraceEvents; i += blockDim.x) trace_sm[i] = 0;
+#endif
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -200,19 +247,19 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(&v_empty[s], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(s_free, 4);
-        for (int i = 0; i < 2; ++i) {
+        mbar_init(s_free, 8);
+        for (int i = 0; i < 4; ++i) {
             mbar_init(&p_full[i], 4);
             mbar_init(&p_free[i], 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && !dense) {
+    if (warp == 8 && !dense) {
         // kept-block bitmasks of the tile's query blocks, from the CSR lists
         for (int w = lane; w < 2 * a.nW; w += 32) kept[w] = 0u;
         __syncwarp();
@@ -233,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             prefetch_tmap(&tm_q);
@@ -247,56 +294,77 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int dc = 0; dc < D / 64; ++dc)
                 tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
             int j = 0;
-            int kiss[kKS] = {}, viss[kVS] = {};
-            auto push = [&](int kind, int blk, uint32_t who, int ncols, float last_bias, uint64_t m0,
-                            uint64_t m1) -> bool {
+            // half h of the tile lands at row offset 64 h of every channel chunk
+            auto load_half = [&](uint8_t *dst, int kind, int blk, const CUtensorMap *tm_x, const CUtensorMap *tm_c,
+                                 uint64_t *bar) {
+                for (int dc = 0; dc < D / 64; ++dc) {
+                    uint8_t *d = dst + dc * (kTK * 128);
+                    if (kind == TILE_EXACT)
+                        tma_load_4d(d, tm_x, bar, dc * 64, h, blk * kBK, b);
+                    else
+                        tma_load_3d(d, tm_c, bar, dc * 64, blk * kBK, bh);
+                }
+            };
+            auto push = [&](int kind, const int (&blk)[2], const uint32_t (&who)[2], const int (&nc)[2],
+                            const int (&pcol)[2], float last_bias, const uint64_t (&cm)[2][2]) -> bool {
                 const int ks = j % kKS, vs = j % kVS;
                 if (j >= kKS && !mbar_wait(&k_empty[ks], ((j / kKS) - 1) & 1, abort_flag, a.status, 10))
                     return false;
                 kkind[ks] = kind;
-                uint8_t *kd = sm + L::kOffK + ks * L::kKVBytes;
-                if (kind == TILE_EXACT) {
-                    mbar_expect_tx(&k_full[ks], L::kKVBytes);
-                    for (int dc = 0; dc < D / 64; ++dc)
-                        tma_load_4d(kd + dc * (kBK * 128), &tm_k, &k_full[ks], dc * 64, h, blk * kBK, b);
-                } else if (kind == TILE_CENT) {
-                    mbar_expect_tx(&k_full[ks], L::kKVBytes);
-                    for (int dc = 0; dc < D / 64; ++dc)
-                        tma_load_3d(kd + dc * (kBK * 128), &tm_kc, &k_full[ks], dc * 64, blk * kBK, bh);
-                } else {
+                TRACE(0, j);
+                uint8_t *kd = sm + L::kOffK + ks * L::kTileBytes;
+                if (kind == TILE_END) {
                     mbar_arrive(&k_full[ks]);
+                } else {
+                    mbar_expect_tx(&k_full[ks], L::kTileBytes);
+                    load_half(kd, kind, blk[0], &tm_k, &tm_kc, &k_full[ks]);
+                    load_half(kd + L::kHalfBytes, kind, blk[1], &tm_k, &tm_kc, &k_full[ks]);
                 }
-                kiss[ks]++;
                 if (j >= kVS && !mbar_wait(&v_empty[vs], ((j / kVS) - 1) & 1, abort_flag, a.status, 11))
                     return false;
+                TRACE(1, j);
                 info[vs].kind = kind;
-                info[vs].blk = blk;
-                info[vs].who = who;
-                info[vs].ncols = ncols;
-                info[vs].last_bias = last_bias;
-                info[vs].cmask[0] = m0;
-                info[vs].cmask[1] = m1;
-                uint8_t *vd = sm + L::kOffV + vs * L::kKVBytes;
-                if (kind == TILE_EXACT) {
-                    mbar_expect_tx(&v_full[vs], L::kKVBytes);
-                    for (int dc = 0; dc < D / 64; ++dc)
-                        tma_load_4d(vd + dc * (kBK * 128), &tm_v, &v_full[vs], dc * 64, h, blk * kBK, b);
-                } else if (kind == TILE_CENT) {
-                    mbar_expect_tx(&v_full[vs], L::kKVBytes);
-                    for (int dc = 0; dc < D / 64; ++dc)
-                        tma_load_3d(vd + dc * (kBK * 128), &tm_vc, &v_full[vs], dc * 64, blk * kBK, bh);
-                } else {
-                    mbar_arrive(&v_full[vs]);
+                for (int x = 0; x < 2; ++x) {
+                    info[vs].blk[x] = blk[x];
+                    info[vs].who[x] = who[x];
+                    info[vs].ncols[x] = nc[x];
+                    info[vs].pcol[x] = pcol[x];
+                    info[vs].cmask[x][0] = cm[x][0];
+                    info[vs].cmask[x][1] = cm[x][1];
                 }
-                viss[vs]++;
+                info[vs].last_bias = last_bias;
+                uint8_t *vd = sm + L::kOffV + vs * L::kTileBytes;
+                if (kind == TILE_END) {
+                    mbar_arrive(&v_full[vs]);
+                } else {
+                    mbar_expect_tx(&v_full[vs], L::kTileBytes);
+                    load_half(vd, kind, blk[0], &tm_v, &tm_vc, &v_full[vs]);
+                    load_half(vd + L::kHalfBytes, kind, blk[1], &tm_v, &tm_vc, &v_full[vs]);
+                }
                 ++j;
                 return true;
             };
+            const uint64_t zero2[2][2] = {{0, 0}, {0, 0}};
+            const int none[2] = {-1, -1};
             bool ok = true;
-            const int last_n = a.N - (a.nKB - 1) * kBK;
+            // exact tiles: pairs of key blocks; an odd last tile repeats its block
+            // in the empty half (a valid load) with no active column
+            int pend = -1;
+            uint32_t pend_who = 0;
+            auto emit_block = [&](int blk, uint32_t who) {
+                if (pend < 0) {
+                    pend = blk;
+                    pend_who = who;
+                    return;
+                }
+                const int bl[2] = {pend, blk};
+                const uint32_t wh[2] = {pend_who, who};
+                const int nc[2] = {min(kBK, a.N - pend * kBK), min(kBK, a.N - blk * kBK)};
+                ok = push(TILE_EXACT, bl, wh, nc, none, 0.f, zero2);
+                pend = -1;
+            };
             if (dense) {
-                for (int blk = kb0; blk < kb1 && ok; ++blk)
-                    ok = push(TILE_EXACT, blk, 3u, min(kBK, a.N - blk * kBK), 0.f, 0, 0);
+                for (int blk = kb0; blk < kb1 && ok; ++blk) emit_block(blk, 3u);
             } else {
                 const uint32_t *k0 = kept, *k1 = kept + a.nW;
                 for (int w = 0; w < a.nW && ok; ++w) {
@@ -304,99 +372,156 @@ __global__ void __launch_bounds__(kThreads, 2)
                     while (u && ok) {
                         const int bit = __ffs(u) - 1;
                         u &= u - 1;
-                        const int blk = w * 32 + bit;
-                        const uint32_t who = ((k0[w] >> bit) & 1u) | (((k1[w] >> bit) & 1u) << 1);
-                        ok = push(TILE_EXACT, blk, who, min(kBK, a.N - blk * kBK), 0.f, 0, 0);
-                    }
-                }
-                if (a.centroid) {
-                    const int nchunk = (a.nKB + kBK - 1) / kBK;
-                    for (int cc = 0; cc < nchunk && ok; ++cc) {
-                        const int nb = min(kBK, a.nKB - cc * kBK);
-                        const uint64_t valid = nb == 64 ? ~0ull : ((1ull << nb) - 1ull);
-                        auto words = [&](const uint32_t *k) -> uint64_t {
-                            const int w0 = 2 * cc;
-                            const uint64_t lo = w0 < a.nW ? k[w0] : 0u;
-                            const uint64_t hi = w0 + 1 < a.nW ? k[w0 + 1] : 0u;
-                            return lo | (hi << 32);
-                        };
-                        const uint64_t m0 = valid & ~words(k0);
-                        const uint64_t m1 = nq > 1 ? (valid & ~words(k1)) : 0ull;
-                        if ((m0 | m1) == 0ull) continue;
-                        const int lastcol = (a.nKB - 1) - cc * kBK;
-                        const bool partial = last_n < kBK && lastcol < kBK;
-                        ok = push(TILE_CENT, cc, 0u, partial ? lastcol : -1,
-                                  partial ? log2f((float)last_n) : 0.f, m0, m1);
+                        emit_block(w * 32 + bit, ((k0[w] >> bit) & 1u) | (((k1[w] >> bit) & 1u) << 1));
                     }
                 }
             }
-            if (ok) ok = push(TILE_END, 0, 0u, 0, 0.f, 0, 0);
-            // no TMA write may still be in flight when the CTA exits
+            if (ok && pend >= 0) {
+                const int bl[2] = {pend, pend};
+                const uint32_t wh[2] = {pend_who, 0u};
+                const int nc[2] = {min(kBK, a.N - pend * kBK), 0};
+                ok = push(TILE_EXACT, bl, wh, nc, none, 0.f, zero2);
+                pend = -1;
+            }
+            if (!dense && a.centroid && ok) {
+                const int last_n = a.N - (a.nKB - 1) * kBK;
+                const int nchunk = (a.nKB + kBK - 1) / kBK;
+                const uint32_t *k0 = kept, *k1 = kept + a.nW;
+                auto cmask = [&](const uint32_t *k, int cc) -> uint64_t {
+                    if (cc >= nchunk) return 0ull;
+                    const int nb = min(kBK, a.nKB - cc * kBK);
+                    const uint64_t valid = nb == 64 ? ~0ull : ((1ull << nb) - 1ull);
+                    const int w0 = 2 * cc;
+                    const uint64_t lo = w0 < a.nW ? k[w0] : 0u;
+                    const uint64_t hi = w0 + 1 < a.nW ? k[w0 + 1] : 0u;
+                    return valid & ~(lo | (hi << 32));
+                };
+                for (int cc = 0; cc < nchunk && ok; cc += 2) {
+                    uint64_t cm[2][2];
+                    int bl[2], pc[2];
+                    for (int x = 0; x < 2; ++x) {
+                        const int c = cc + x;
+                        cm[0][x] = cmask(k0, c);
+                        cm[1][x] = nq > 1 ? cmask(k1, c) : 0ull;
+                        bl[x] = c < nchunk ? c : cc;          // an empty half repeats a valid chunk
+                        const int lastcol = (a.nKB - 1) - c * kBK;
+                        pc[x] = (c < nchunk && last_n < kBK && lastcol >= 0 && lastcol < kBK) ? lastcol : -1;
+                    }
+                    if ((cm[0][0] | cm[0][1] | cm[1][0] | cm[1][1]) == 0ull) continue;
+                    const uint32_t wh[2] = {0u, 0u};
+                    const int nc[2] = {0, 0};
+                    ok = push(TILE_CENT, bl, wh, nc, pc, last_n < kBK ? log2f((float)last_n) : 0.f, cm);
+                }
+            }
+            if (ok) {
+                const int bl[2] = {0, 0};
+                const uint32_t wh[2] = {0u, 0u};
+                const int nc[2] = {0, 0};
+                ok = push(TILE_END, bl, wh, nc, none, 0.f, zero2);
+            }
+            // no TMA write may still be in flight when the CTA exits: wait for the
+            // last phase every slot was armed with
             volatile int32_t no_abort = 0;
-            for (int s = 0; s < kKS; ++s)
-                if (kiss[s] > 0) mbar_wait(&k_full[s], (kiss[s] - 1) & 1, &no_abort, a.status, 12);
-            for (int s = 0; s < kVS; ++s)
-                if (viss[s] > 0) mbar_wait(&v_full[s], (viss[s] - 1) & 1, &no_abort, a.status, 13);
+            for (int s = 0; s < kKS; ++s) {
+                const int n = (j - s + kKS - 1) / kKS;
+                if (n > 0) mbar_wait(&k_full[s], (n - 1) & 1, &no_abort, a.status, 12);
+            }
+            for (int s = 0; s < kVS; ++s) {
+                const int n = (j - s + kVS - 1) / kVS;
+                if (n > 0) mbar_wait(&v_full[s], (n - 1) & 1, &no_abort, a.status, 13);
+            }
             mbar_wait(bar_q, 0, &no_abort, a.status, 14);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16_f32(kM, kBK, 0, 0);
+            const uint32_t idesc_s = idesc_bf16_f32(kM, kTK, 0, 0);
             const uint32_t idesc_o = idesc_bf16_f32(kM, D, 0, 1);
             const uint32_t q_addr = smem_u32(sm + L::kOffQ);
             const uint32_t k_addr = smem_u32(sm + L::kOffK);
             const uint32_t v_addr = smem_u32(sm + L::kOffV);
-            auto issue_pv = [&](int t) -> bool {
-                const int pb = t & 1, vs = t % kVS;
-                if (!mbar_wait(&v_full[vs], (t / kVS) & 1, abort_flag, a.status, 20)) return false;
-                if (!mbar_wait(&p_full[pb], (t >> 1) & 1, abort_flag, a.status, 21)) return false;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kBK / 16; ++ks) {
-                    const uint64_t bd = sdesc_sw128(v_addr + vs * L::kKVBytes + ks * 2048, kBK * 128, 1024);
-                    umma_bf16_ts(tmem + kColO, tmem + kColP + 32 * pb + 8 * ks, bd, idesc_o,
-                                 (t > 0 || ks > 0) ? 1u : 0u);
-                }
-                umma_commit(&v_empty[vs]);
-                umma_commit(&p_free[pb]);
-                return true;
-            };
             bool ok = mbar_wait(bar_q, 0, abort_flag, a.status, 22);
             tc_fence_after();
-            int j = 0;
-            while (ok) {
-                const int ks = j % kKS;
-                if (!(ok = mbar_wait(&k_full[ks], (j / kKS) & 1, abort_flag, a.status, 23))) break;
-                tc_fence_after();
-                if (kkind[ks] == TILE_END) break;
-                if (j >= 1 && !(ok = mbar_wait(s_free, (j - 1) & 1, abort_flag, a.status, 24))) break;
-                tc_fence_after();
+            // Event loop: S of the next tile is issued as soon as both halves have
+            // read the current S; O_h += P_h V_h as soon as half h's P is in.
+            int ns = 0, T = -1;
+            int np[2] = {0, 0};
+            long long idle_since = clock64();
+            while (ok && (T < 0 || np[0] < T || np[1] < T)) {
+                bool progressed = false;
+                if (T < 0) {
+                    const int ks = ns % kKS;
+                    if (mbar_test(&k_full[ks], (ns / kKS) & 1) && (ns < 1 || mbar_test(s_free, (ns - 1) & 1))) {
+                        tc_fence_after();
+                        if (kkind[ks] == TILE_END) {
+                            T = ns;
+                        } else {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad =
-                        sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(
-                        k_addr + ks * L::kKVBytes + (kk >> 2) * (kBK * 128) + (kk & 3) * 32, 16, 1024);
-                    umma_bf16(tmem + kColS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint64_t ad =
+                                    sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+                                const uint64_t bd = sdesc_sw128(
+                                    k_addr + ks * L::kTileBytes + (kk >> 2) * (kTK * 128) + (kk & 3) * 32, 16, 1024);
+                                umma_bf16(tmem + kColS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                            }
+                            umma_commit(s_full);
+                            umma_commit(&k_empty[ks]);
+                            TRACE(2, ns);
+                            ++ns;
+                        }
+                        progressed = true;
+                    }
                 }
-                umma_commit(s_full);
-                umma_commit(&k_empty[ks]);
-                if (j >= 1 && !(ok = issue_pv(j - 1))) break;
-                ++j;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int t = np[hf];
+                    if (t >= ns) continue;
+                    const int pb = t & 1, vs = t % kVS;
+                    if (mbar_test(&p_full[2 * hf + pb], (t >> 1) & 1) && mbar_test(&v_full[vs], (t / kVS) & 1)) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < kBK / 16; ++ks) {
+                            const uint64_t bd = sdesc_sw128(
+                                v_addr + vs * L::kTileBytes + hf * L::kHalfBytes + ks * 2048, kTK * 128, 1024);
+                            umma_bf16_ts(tmem + kColO + 128 * hf, tmem + kColP + 64 * hf + 32 * pb + 8 * ks, bd,
+                                         idesc_o, (t > 0 || ks > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&p_free[2 * hf + pb]);
+                        // the V slot is free once both halves used it; the later half releases it
+                        if (np[1 - hf] > t) umma_commit(&v_empty[vs]);
+                        if (hf == 0) TRACE(3, t);
+                        np[hf] = t + 1;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    idle_since = clock64();
+                } else if (*abort_flag) {
+                    ok = false;
+                } else if (clock64() - idle_since > kWaitCycles) {
+                    *abort_flag = 1;
+                    report(a.status, BSA_DEV_TIMEOUT, 26);
+                    ok = false;
+                }
             }
-            if (ok && j >= 1) ok = issue_pv(j - 1);
-            if (ok) umma_commit(s_full);      // end-of-list marker for the softmax warps
+            // end-of-list marker for the softmax warps, once S is free again
+            if (ok && T >= 1) ok = mbar_wait(s_free, (T - 1) & 1, abort_flag, a.status, 27);
+            if (ok) umma_commit(s_full);
             umma_commit(bar_done);
             volatile int32_t no_abort = 0;
             mbar_wait(bar_done, 0, &no_abort, a.status, 25);
         }
     } else {
         // ---------------------------------------------------------- softmax
-        const int r = threadIdx.x;                               // tile row == TMEM lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // warpgroup hf owns half hf of every tile (one key block) and keeps its own
+        // online softmax state and accumulator O_hf
+        const int hf = warp >> 2;
+        const int r = threadIdx.x & 127;                         // tile row == TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const int qsel = (a.Bq == 64 && !dense) ? (r >> 6) : 0;
         const float scale = a.scale_log2;
+        const uint32_t col_o = kColO + 128 * hf;
+        uint64_t *pf = p_full + 2 * hf, *pe = p_free + 2 * hf;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         int j = 0;
@@ -408,161 +533,193 @@ __global__ void __launch_bounds__(kThreads, 2)
             tc_fence_after();
             const int kind = info[vs].kind;
             if (kind == TILE_END) break;
+            if (r == 0) TRACE(4 + 3 * hf, j);
             float s[64];
-            tmem_ld32(tmem + lane_base + kColS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-            tmem_ld32(tmem + lane_base + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+            tmem_ld32(tmem + lane_base + kColS + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+            tmem_ld32(tmem + lane_base + kColS + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(s_free);
+            if (r == 0) TRACE(5 + 3 * hf, j);
 
-            bool fast = false;
+            // 0: skip (no active column), 1: all 64 columns active, 2: masked / biased
+            int mode;
             if (kind == TILE_EXACT) {
-                const bool act = (info[vs].who >> qsel) & 1u;
-                const int nc = act ? info[vs].ncols : 0;
-                fast = nc == kBK;
-                if (!fast) {
+                const bool act = (info[vs].who[hf] >> qsel) & 1u;
+                const int nc = act ? info[vs].ncols[hf] : 0;
+                if (nc >= kBK) {
+                    mode = 1;
+                } else if (nc <= 0) {
+                    mode = 0;
+                } else {
+                    mode = 2;
 #pragma unroll
                     for (int c = 0; c < 64; ++c) s[c] = c < nc ? s[c] * scale : -INFINITY;
                 }
             } else {
-                const uint64_t msk = info[vs].cmask[qsel];
-                const int pc = info[vs].ncols;
+                const uint64_t msk = info[vs].cmask[qsel][hf];
+                const int pc = info[vs].pcol[hf];
                 const float pbias = info[vs].last_bias;
+                mode = msk ? 2 : 0;
+                if (msk) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float bias = c == pc ? pbias : 6.0f;       // log2(64) for full blocks
-                    s[c] = ((msk >> c) & 1ull) ? fmaf(s[c], scale, bias) : -INFINITY;
+                    for (int c = 0; c < 64; ++c) {
+                        const float bias = c == pc ? pbias : 6.0f;       // log2(64) for full blocks
+                        s[c] = ((msk >> c) & 1ull) ? fmaf(s[c], scale, bias) : -INFINITY;
+                    }
                 }
             }
-            const float mt = fast ? max64(s) * scale : max64(s);
-            float alpha = 1.f;
-            bool rescale = false;
-            if (mt > m_ref) {
-                if (m_ref == -INFINITY) {
-                    m_ref = mt;
-                } else if (mt > m_ref + kRescaleLog2) {
-                    alpha = ex2(m_ref - mt);
-                    l *= alpha;
-                    m_ref = mt;
-                    rescale = true;
-                }
-            }
-            const float mref = m_ref == -INFINITY ? 0.f : m_ref;
             uint32_t pk[32];
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            if (fast) {
-                const float nm = -mref;
+            bool rescale = false;
+            float alpha = 1.f;
+            if (mode == 0) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2(fmaf(s[2 * c], scale, nm));
-                    const float p1 = ex2(fmaf(s[2 * c + 1], scale, nm));
-                    acc[c & 3] += p0 + p1;
-                    pk[c] = pack_bf16x2(p0, p1);
-                }
+                for (int c = 0; c < 32; ++c) pk[c] = 0u;
             } else {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2(s[2 * c] - mref);
-                    const float p1 = ex2(s[2 * c + 1] - mref);
-                    acc[c & 3] += p0 + p1;
-                    pk[c] = pack_bf16x2(p0, p1);
+                const float mt = mode == 1 ? max64(s) * scale : max64(s);
+                if (mt > m_ref) {
+                    if (m_ref == -INFINITY) {
+                        m_ref = mt;
+                    } else if (mt > m_ref + kRescaleLog2) {
+                        alpha = ex2(m_ref - mt);
+                        l *= alpha;
+                        m_ref = mt;
+                        rescale = true;
+                    }
                 }
+                const float mref = m_ref == -INFINITY ? 0.f : m_ref;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                if (mode == 1) {
+                    const float nm = -mref;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float p0 = ex2(fmaf(s[2 * c], scale, nm));
+                        const float p1 = ex2(fmaf(s[2 * c + 1], scale, nm));
+                        acc[c & 3] += p0 + p1;
+                        pk[c] = pack_bf16x2(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const float p0 = ex2(s[2 * c] - mref);
+                        const float p1 = ex2(s[2 * c + 1] - mref);
+                        acc[c & 3] += p0 + p1;
+                        pk[c] = pack_bf16x2(p0, p1);
+                    }
+                }
+                l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
-            l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            if (r == 0) TRACE(10 + 3 * hf, j);
             if (j >= 2) {
-                ok = mbar_wait(&p_free[j & 1], ((j >> 1) - 1) & 1, abort_flag, a.status, 32);
+                ok = mbar_wait(&pe[j & 1], ((j >> 1) - 1) & 1, abort_flag, a.status, 32);
                 if (!(ok = __all_sync(0xffffffffu, ok))) break;
             }
-            tmem_st32(tmem + lane_base + kColP + 32 * (j & 1), pk);
+            if (r == 0) TRACE(11 + 3 * hf, j);
+            tmem_st32(tmem + lane_base + kColP + 64 * hf + 32 * (j & 1), pk);
             if (__any_sync(0xffffffffu, rescale)) {
                 // the accumulator must hold every earlier P V product before it is scaled
-                ok = mbar_wait(&p_free[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status, 33);
+                ok = mbar_wait(&pe[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status, 33);
                 if (!(ok = __all_sync(0xffffffffu, ok))) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t o[32];
-                    tmem_ld32(tmem + lane_base + kColO + cc * 32, o);
+                    tmem_ld32(tmem + lane_base + col_o + cc * 32, o);
                     tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(tmem + lane_base + kColO + cc * 32, o);
+                    tmem_st32(tmem + lane_base + col_o + cc * 32, o);
                 }
             }
             tmem_st_wait();
+            if (r == 0) TRACE(12 + 3 * hf, j);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[j & 1]);
+            if (lane == 0) mbar_arrive(&pf[j & 1]);
+            if (r == 0) TRACE(6 + 3 * hf, j);
         }
         const int T = j;
-        if (ok && T >= 1)
-            ok = mbar_wait(&p_free[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, a.status, 34);
+        if (ok && T >= 1) ok = mbar_wait(&pe[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, a.status, 34);
         ok = __all_sync(0xffffffffu, ok);
+        // ------------------------------------------------------ epilogue
+        // merge the halves: O = (wA O_A + wB O_B) / (wA lA + wB lB), w = 2^(m_half - m)
+        const bool have = T >= 1 && l > 0.f;
+        ml[hf * kM + r] = make_float2(have ? m_ref : -INFINITY, have ? l : 0.f);
+        named_bar(1, 256);
+        const float2 A = ml[r], Bv = ml[kM + r];
+        const float m = fmaxf(A.x, Bv.x);
+        const float wA = A.x > -INFINITY ? ex2(A.x - m) : 0.f;
+        const float wB = Bv.x > -INFINITY ? ex2(Bv.x - m) : 0.f;
+        const float lt = wA * A.y + wB * Bv.y;
         tc_fence_after();
         if (ok) {
             const bool row_ok = r < nvalid;
             const int n = row0 + r;
-            const bool have_o = T >= 1 && l > 0.f;
-            if (dense && a.dense_split > 1) {
-                // unnormalised partial in the frame of m_ref, merged by combine_kernel
-                float *po = a.part_o + (pidx * kM + r) * D;
+            const bool split = dense && a.dense_split > 1;
+            // a sparse item leaves rows of the dense range to the dense items
+            const bool mine = row_ok && (dense || n < a.dense_begin || n >= a.dense_end);
+            const float inv = split ? 1.f : (lt > 0.f ? 1.f / lt : 0.f);
+            const float cA = wA * inv, cB = wB * inv;
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    __syncwarp();
-                    tmem_ld32(tmem + lane_base + kColO + cc * 32, o);
-                    tmem_ld_wait();
-                    float4 *dst = reinterpret_cast<float4 *>(po + cc * 32);
+            for (int cc = hf * (D / 64); cc < (hf + 1) * (D / 64); ++cc) {
+                uint32_t oa[32], ob[32];
+                __syncwarp();
+                tmem_ld32(tmem + lane_base + kColO + cc * 32, oa);
+                tmem_ld32(tmem + lane_base + kColO + 128 + cc * 32, ob);
+                tmem_ld_wait();
+                if (!(split ? row_ok : mine)) continue;
+                float v[32];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        dst[e] = have_o ? make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                                                      __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]))
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int e = 0; e < 32; ++e) {
+                    const float xa = cA > 0.f ? cA * __uint_as_float(oa[e]) : 0.f;
+                    const float xb = cB > 0.f ? cB * __uint_as_float(ob[e]) : 0.f;
+                    v[e] = xa + xb;
                 }
-                float *ml = a.part_ml + (pidx * kM + r) * 2;
-                ml[0] = have_o ? m_ref : -INFINITY;
-                ml[1] = have_o ? l : 0.f;
-            } else {
-                // a sparse item leaves rows of the dense range to the dense items
-                const bool mine = row_ok && (dense || n < a.dense_begin || n >= a.dense_end);
-                const float inv_l = have_o ? 1.f / l : 0.f;
-#pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    __syncwarp();
-                    tmem_ld32(tmem + lane_base + kColO + cc * 32, o);
-                    tmem_ld_wait();
-                    if (!mine) continue;
-                    float v[32];
+                if (split) {
+                    // unnormalised partial in the frame of m, merged by combine_kernel
+                    float4 *dst = reinterpret_cast<float4 *>(a.part_o + (pidx * kM + r) * D + cc * 32);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = have_o ? __uint_as_float(o[e]) * inv_l : 0.f;
-                    const int64_t off = (int64_t)b * a.sb + (int64_t)n * a.sn + (int64_t)h * a.sh + cc * 32;
-                    if (a.out_f32) {
-                        float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + off);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-                    } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + off);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]),
-                                                pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
-                                                pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
-                                                pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
-                    }
+                    for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+                    continue;
                 }
-                if (mine && a.lse != nullptr)
-                    a.lse[(int64_t)bh * a.N + n] =
-                        have_o ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+                const int64_t off = (int64_t)b * a.sb + (int64_t)n * a.sn + (int64_t)h * a.sh + cc * 32;
+                if (a.out_f32) {
+                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + off);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+                } else {
+                    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(a.out) + off);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]), pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
+                                            pack_bf16x2(v[8 * e + 4], v[8 * e + 5]),
+                                            pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
+                }
+            }
+            if (hf == 0) {
+                if (split) {
+                    float *pm = a.part_ml + (pidx * kM + r) * 2;
+                    pm[0] = lt > 0.f ? m : -INFINITY;
+                    pm[1] = lt;
+                } else if (mine && a.lse != nullptr) {
+                    a.lse[(int64_t)bh * a.N + n] = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+                }
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+#ifdef BSA_TRACE
+    {
+        const int c = (int)blockIdx.x - a.trace_base;
+        if (a.trace != nullptr && c >= 0 && c < kTraceCtas)
+            for (int i = threadIdx.x; i < kTraceTiles * kTraceEvents; i += blockDim.x)
+                a.trace[(int64_t)c * kTraceTiles * kTraceEvents + i] = trace_sm[i];
+    }
+#endif
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -699,6 +856,16 @@ cudaError_t launch_attn_kernel(const CUtensorMap &tq, const CUtensorMap &tk, con
 
 }  // namespace
 
+#ifdef BSA_TRACE
+long long *g_trace = nullptr;
+int g_trace_base = 0;
+extern "C" __attribute__((visibility("default"))) void bsa_debug_set_trace(void *p, int base)
+{
+    g_trace = static_cast<long long *>(p);
+    g_trace_base = base;
+}
+#endif
+
 // Key-chunk split of the dense rows: enough items to cover the GPU, chunks of
 // at least 256 key blocks, bounded by `max_partials` partial tiles.
 int dense_split_for(const Dims &D, int nrows, int64_t max_partials)
@@ -782,6 +949,13 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     a.centroid = p.centroid;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D.d));
     a.status = reinterpret_cast<int32_t *>(ws + L.status);
+#ifdef BSA_TRACE
+    a.trace = g_trace;
+    a.trace_base = g_trace_base;
+#else
+    a.trace = nullptr;
+    a.trace_base = 0;
+#endif
     a.n_sparse = dense_only ? 0 : (int)ceil_div(D.N, kM);
     a.skip_begin = row_begin;
     a.skip_end = row_end;
