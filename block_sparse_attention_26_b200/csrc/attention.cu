@@ -27,15 +27,17 @@
 // the tile's half h -- one key block -- with its own online softmax state and
 // its own accumulator O_h; the halves are merged in the epilogue.
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3, 4-7  softmax warpgroups h = 0, 1: thread r owns query row r
 //              (TMEM lane r).  Read S from TMEM, mask, online softmax in the log2
 //              domain with a lazily updated reference max (the accumulator is
 //              rescaled only when the row max grows by more than 2^8), write P
 //              (bf16) into TMEM, and run the epilogue.
-//   warp 8     producer: builds the tile list; TMA loads of K and V tiles (or of
-//              bf16 centroid tiles) into separate rings; a K slot is released as
-//              soon as its S product is done.
+//   warps 8, 10  K and V producers: each builds the same tile list and TMA-loads
+//              its K (resp. V) tiles (or bf16 centroid tiles) into its own ring,
+//              so K prefetch never waits for V slots; a K slot is released as
+//              soon as its S product is done, the V producer also publishes each
+//              tile's masks to the softmax warps.
 //   warp 9     MMA issuer (one thread, event loop): S = Q K^T (A and B from
 //              shared memory) runs ahead of the softmax; O_h += P_h V_h (A = P_h
 //              from TMEM) is issued as soon as half h of a tile's P is in.
@@ -56,7 +58,7 @@ constexpr int kBK = 64;        // keys per key block
 constexpr int kTK = 128;       // keys per tile (two blocks)
 constexpr int kKS = 2;         // K ring depth (tiles)
 constexpr int kVS = 3;         // V ring depth (tiles)
-constexpr int kThreads = 320;  // 2 softmax warpgroups + producer warp + MMA warp
+constexpr int kThreads = 352;  // 2 softmax warpgroups + K producer + MMA + V producer
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;          // S, 128 columns
@@ -280,23 +282,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
-        // ---------------------------------------------------------- producer
+    if (warp == 8 || warp == 10) {
+        // ---------------------------------------------------------- producers
         if (lane == 0) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-            if (!dense && a.centroid) {
-                prefetch_tmap(&tm_kc);
-                prefetch_tmap(&tm_vc);
+            const bool is_k = warp == 8;
+            if (is_k) {
+                prefetch_tmap(&tm_q);
+                prefetch_tmap(&tm_k);
+                if (!dense && a.centroid) prefetch_tmap(&tm_kc);
+                mbar_expect_tx(bar_q, L::kQBytes);
+                for (int dc = 0; dc < D / 64; ++dc)
+                    tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
+            } else {
+                prefetch_tmap(&tm_v);
+                if (!dense && a.centroid) prefetch_tmap(&tm_vc);
             }
-            mbar_expect_tx(bar_q, L::kQBytes);
-            for (int dc = 0; dc < D / 64; ++dc)
-                tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
+            const CUtensorMap *tm_x = is_k ? &tm_k : &tm_v;
+            const CUtensorMap *tm_c = is_k ? &tm_kc : &tm_vc;
+            const int depth = is_k ? kKS : kVS;
+            uint64_t *full = is_k ? k_full : v_full;
+            uint64_t *empty = is_k ? k_empty : v_empty;
+            uint8_t *ring = sm + (is_k ? L::kOffK : L::kOffV);
             int j = 0;
-            // half h of the tile lands at row offset 64 h of every channel chunk
-            auto load_half = [&](uint8_t *dst, int kind, int blk, const CUtensorMap *tm_x, const CUtensorMap *tm_c,
-                                 uint64_t *bar) {
+            // half x of the tile lands at row offset 64 x of every channel chunk
+            auto load_half = [&](uint8_t *dst, int kind, int blk, uint64_t *bar) {
                 for (int dc = 0; dc < D / 64; ++dc) {
                     uint8_t *d = dst + dc * (kTK * 128);
                     if (kind == TILE_EXACT)
@@ -307,39 +316,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto push = [&](int kind, const int (&blk)[2], const uint32_t (&who)[2], const int (&nc)[2],
                             const int (&pcol)[2], float last_bias, const uint64_t (&cm)[2][2]) -> bool {
-                const int ks = j % kKS, vs = j % kVS;
-                if (j >= kKS && !mbar_wait(&k_empty[ks], ((j / kKS) - 1) & 1, abort_flag, a.status, 10))
+                const int s = j % depth;
+                if (j >= depth && !mbar_wait(&empty[s], ((j / depth) - 1) & 1, abort_flag, a.status, is_k ? 10 : 11))
                     return false;
-                kkind[ks] = kind;
-                TRACE(0, j);
-                uint8_t *kd = sm + L::kOffK + ks * L::kTileBytes;
-                if (kind == TILE_END) {
-                    mbar_arrive(&k_full[ks]);
+                if (is_k) {
+                    kkind[s] = kind;
+                    TRACE(0, j);
                 } else {
-                    mbar_expect_tx(&k_full[ks], L::kTileBytes);
-                    load_half(kd, kind, blk[0], &tm_k, &tm_kc, &k_full[ks]);
-                    load_half(kd + L::kHalfBytes, kind, blk[1], &tm_k, &tm_kc, &k_full[ks]);
+                    TRACE(1, j);
+                    info[s].kind = kind;
+                    for (int x = 0; x < 2; ++x) {
+                        info[s].blk[x] = blk[x];
+                        info[s].who[x] = who[x];
+                        info[s].ncols[x] = nc[x];
+                        info[s].pcol[x] = pcol[x];
+                        info[s].cmask[x][0] = cm[x][0];
+                        info[s].cmask[x][1] = cm[x][1];
+                    }
+                    info[s].last_bias = last_bias;
                 }
-                if (j >= kVS && !mbar_wait(&v_empty[vs], ((j / kVS) - 1) & 1, abort_flag, a.status, 11))
-                    return false;
-                TRACE(1, j);
-                info[vs].kind = kind;
-                for (int x = 0; x < 2; ++x) {
-                    info[vs].blk[x] = blk[x];
-                    info[vs].who[x] = who[x];
-                    info[vs].ncols[x] = nc[x];
-                    info[vs].pcol[x] = pcol[x];
-                    info[vs].cmask[x][0] = cm[x][0];
-                    info[vs].cmask[x][1] = cm[x][1];
-                }
-                info[vs].last_bias = last_bias;
-                uint8_t *vd = sm + L::kOffV + vs * L::kTileBytes;
+                uint8_t *dst = ring + s * L::kTileBytes;
                 if (kind == TILE_END) {
-                    mbar_arrive(&v_full[vs]);
+                    mbar_arrive(&full[s]);
                 } else {
-                    mbar_expect_tx(&v_full[vs], L::kTileBytes);
-                    load_half(vd, kind, blk[0], &tm_v, &tm_vc, &v_full[vs]);
-                    load_half(vd + L::kHalfBytes, kind, blk[1], &tm_v, &tm_vc, &v_full[vs]);
+                    mbar_expect_tx(&full[s], L::kTileBytes);
+                    load_half(dst, kind, blk[0], &full[s]);
+                    load_half(dst + L::kHalfBytes, kind, blk[1], &full[s]);
                 }
                 ++j;
                 return true;
@@ -422,15 +424,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // no TMA write may still be in flight when the CTA exits: wait for the
             // last phase every slot was armed with
             volatile int32_t no_abort = 0;
-            for (int s = 0; s < kKS; ++s) {
-                const int n = (j - s + kKS - 1) / kKS;
-                if (n > 0) mbar_wait(&k_full[s], (n - 1) & 1, &no_abort, a.status, 12);
+            for (int s = 0; s < depth; ++s) {
+                const int n = (j - s + depth - 1) / depth;
+                if (n > 0) mbar_wait(&full[s], (n - 1) & 1, &no_abort, a.status, 12);
             }
-            for (int s = 0; s < kVS; ++s) {
-                const int n = (j - s + kVS - 1) / kVS;
-                if (n > 0) mbar_wait(&v_full[s], (n - 1) & 1, &no_abort, a.status, 13);
-            }
-            mbar_wait(bar_q, 0, &no_abort, a.status, 14);
+            if (is_k) mbar_wait(bar_q, 0, &no_abort, a.status, 14);
         }
     } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
