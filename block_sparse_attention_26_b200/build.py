@@ -1,6 +1,8 @@
 """Build libbsa.so (sm_100a) in-tree with nvcc.
 
-    python -m block_sparse_attention_26_b200.build [--force]
+    python block_sparse_attention_26_b200/build.py [--force]
+
+(Run it by path: importing the package loads the library it builds.)
 """
 from __future__ import annotations
 
