@@ -51,7 +51,7 @@ class BsaError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libbsa.so not built at {LIB_PATH}; run block_sparse_attention_26_b200.build")
+        raise ImportError(f"libbsa.so not built at {LIB_PATH}; run python block_sparse_attention_26_b200/build.py")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     PP = ctypes.POINTER(bsa_params)
@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
     lib.bsa_workspace_size.argtypes = [PP, ctypes.POINTER(SZ), ctypes.POINTER(I64)]
     lib.bsa_pool.argtypes = [PP, P, P, P, P, P, P, P, P]
     lib.bsa_select.argtypes = [PP, P, P, P, P, P, I64, P, P, P, P, SZ, P]
+    lib.bsa_select_static.argtypes = [PP, P, P, P, P, I64, P, P]
     lib.bsa_attention.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.bsa_dense_ref_rows.argtypes = [PP, P, P, P, I32, I32, P, P, P, SZ, P]
     lib.bsa_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
@@ -67,16 +68,16 @@ def _load() -> ctypes.CDLL:
     lib.bsa_status_string.restype = ctypes.c_char_p
     lib.bsa_last_error.argtypes = []
     lib.bsa_last_error.restype = ctypes.c_char_p
-    for f in ("bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_attention", "bsa_dense_ref_rows",
-              "bsa_device_status"):
+    for f in ("bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_select_static", "bsa_attention",
+              "bsa_dense_ref_rows", "bsa_device_status"):
         getattr(lib, f).restype = I32
     return lib
 
 
 lib = _load()
 
-EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_attention",
-            "bsa_dense_ref_rows", "bsa_device_status", "bsa_status_string", "bsa_last_error")
+EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_select_static",
+            "bsa_attention", "bsa_dense_ref_rows", "bsa_device_status", "bsa_status_string", "bsa_last_error")
 
 
 def _check(status: int, where: str):
@@ -156,6 +157,12 @@ def bsa_select(p, qbar, kbar, k, row_ptr, col_idx, kept_count, extra_idx, extra_
     _check(lib.bsa_select(ctypes.byref(p), _ptr(qbar), _ptr(kbar), _ptr(k), _ptr(row_ptr), _ptr(col_idx),
                           cap, _ptr(kept_count), _ptr(extra_idx), _ptr(extra_count), _ptr(ws),
                           ws.numel() * ws.element_size(), _stream(stream)), "bsa_select")
+
+
+def bsa_select_static(p, qbar, kbar, row_ptr, col_idx, kept_count, stream=None):
+    cap = 0 if col_idx is None else col_idx.numel()
+    _check(lib.bsa_select_static(ctypes.byref(p), _ptr(qbar), _ptr(kbar), _ptr(row_ptr), _ptr(col_idx), cap,
+                                 _ptr(kept_count), _stream(stream)), "bsa_select_static")
 
 
 def bsa_attention(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra_idx, extra_count, out,

@@ -217,6 +217,28 @@ bsa_status bsa_select(const bsa_params *p, const float *qbar, const float *kbar,
                      "bsa_select");
 }
 
+bsa_status bsa_select_static(const bsa_params *p, const float *qbar, const float *kbar, int64_t *row_ptr,
+                             int32_t *col_idx, int64_t col_capacity, int32_t *kept_count, void *stream)
+{
+    g_err[0] = 0;
+    TRY(check_params(p));
+    TRY(check_tensor(qbar, "qbar"));
+    TRY(check_tensor(kbar, "kbar"));
+    if (row_ptr == nullptr || kept_count == nullptr) FAIL(BSA_ERR_INVALID_ARG, "row_ptr / kept_count is NULL");
+    if (col_capacity < 0) FAIL(BSA_ERR_INVALID_ARG, "col_capacity < 0");
+    if (col_capacity > 0 && col_idx == nullptr) FAIL(BSA_ERR_INVALID_ARG, "col_idx is NULL");
+    if (p->extra_tokens > 0) FAIL(BSA_ERR_UNSUPPORTED, "bsa_select_static does not pick extra tokens");
+    WsLayout L;
+    size_t need = 0;
+    if (!static_select_layout(*p, &L, &need))
+        FAIL(BSA_ERR_CAPACITY, "bsa_select_static: this problem needs %zu bytes of scratch, the static array holds %zu",
+             need, static_scratch_bytes());
+    const Dims D = dims_of(*p);
+    return from_cuda(launch_select_static(*p, D, qbar, kbar, row_ptr, col_idx, col_capacity, kept_count, L,
+                                          (cudaStream_t)stream),
+                     "bsa_select_static");
+}
+
 bsa_status bsa_attention(const bsa_params *p, const void *q, const void *k, const void *v, const float *kbar,
                          const float *vbar, const int32_t *blk_count, const int64_t *row_ptr,
                          const int32_t *col_idx, const int32_t *extra_idx, const int32_t *extra_count,

@@ -61,6 +61,13 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
                              int row_begin, int row_end, char *ws, const WsLayout &L,
                              cudaStream_t st);
 
+// Selection with the library's static scratch array instead of a workspace.
+bool static_select_layout(const bsa_params &p, WsLayout *L, size_t *need);
+cudaError_t launch_select_static(const bsa_params &p, const Dims &D, const float *qbar, const float *kbar,
+                                 int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                                 int32_t *kept_count, const WsLayout &L, cudaStream_t st);
+size_t static_scratch_bytes();
+
 // Thread-local host error text.
 void set_error(const char *fmt, ...);
 

@@ -21,6 +21,8 @@
 //   expand_kernel  bitmask -> ascending CSR column lists (popc prefix per warp).
 #include <math.h>
 
+#include <atomic>
+
 #include "bsa_device.cuh"
 #include "bsa_internal.h"
 
@@ -333,5 +335,82 @@ cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar,
                                       kept_count, status);
     return cudaGetLastError();
 }
+
+// ---------------------------------------------------------------------------
+// Selection without caller-provided scratch.
+//
+// Some callers cannot allocate device memory at all: code that runs inside a
+// host framework owning every allocation, a plugin that may not call
+// cudaMalloc on its host's streams, or a process whose allocator is locked
+// while it serves requests.  For them bsa_select_static() keeps the selection
+// scratch (block scores, kept-block bitmasks, per-row counts and the status
+// word) in the file-scope device array below instead of a workspace.  The
+// array has a fixed size; every GPU that loads the library holds it until the
+// process exits.
+constexpr size_t kStaticScratchBytes = (size_t)32 << 20;   // 32 MiB
+static __device__ __align__(256) unsigned char g_select_scratch[kStaticScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<char *> g_static_base[kMaxDevices];
+
+// Device address of g_select_scratch on the current device (looked up once per
+// device; the host-side symbol is only a stand-in and must never be passed to
+// a kernel).
+cudaError_t static_scratch(char **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    char *p = g_static_base[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        void *addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_select_scratch);
+        if (e != cudaSuccess) return e;
+        p = static_cast<char *>(addr);
+        g_static_base[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+// Layout of the selection scratch inside the static array; false if it does not fit.
+bool static_select_layout(const bsa_params &p, WsLayout *L, size_t *need)
+{
+    const Dims D = dims_of(p);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + bytes, 256);
+        return at;
+    };
+    *L = WsLayout();
+    L->status = take(sizeof(int32_t) * 2);
+    L->scores = take((size_t)D.rows * D.nKB * sizeof(float));
+    L->bitmask = take((size_t)D.rows * D.nW * sizeof(uint32_t));
+    L->counts = take((size_t)D.rows * sizeof(int32_t));
+    L->total = off;
+    *need = off;
+    return off <= kStaticScratchBytes;
+}
+
+cudaError_t launch_select_static(const bsa_params &p, const Dims &D, const float *qbar, const float *kbar,
+                                 int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                                 int32_t *kept_count, const WsLayout &L, cudaStream_t st)
+{
+    char *base = nullptr;
+    cudaError_t e = static_scratch(&base);
+    if (e != cudaSuccess) return e;
+    // the status word is the only region read before it is written
+    e = cudaMemsetAsync(base + L.status, 0, sizeof(int32_t) * 2, st);
+    if (e != cudaSuccess) return e;
+    return launch_select(p, D, qbar, kbar, row_ptr, col_idx, col_capacity, kept_count, base, L, st);
+}
+
+size_t static_scratch_bytes() { return kStaticScratchBytes; }
 
 }  // namespace bsa

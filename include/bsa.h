@@ -134,6 +134,28 @@ BSA_API bsa_status bsa_select(const bsa_params *p, const float *qbar, const floa
                       int32_t *kept_count, int32_t *extra_idx, int32_t *extra_count,
                       void *ws, size_t ws_bytes, void *stream);
 
+/* bsa_select without a workspace, for callers that cannot allocate device
+ * memory: a process whose allocator is owned by a host framework, a plugin
+ * that may not call cudaMalloc, a server that must not allocate while it
+ * serves.  The pages describe no such variant; it is a deployment convenience.
+ *   Arguments as for bsa_select (extra tokens are not picked: p->extra_tokens
+ *   must be 0).  The scratch lives in a 32 MiB device array inside the library
+ *   (every GPU that loads the library holds it until the process exits); a
+ *   problem whose selection scratch -- rows*nKB*4 + rows*ceil(nKB/32)*4 +
+ *   rows*4 bytes plus alignment -- exceeds it is rejected with
+ *   BSA_ERR_CAPACITY before anything is launched.
+ *   The first call on a device looks the array's device address up (one
+ *   cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   All calls share the one array: calls whose work overlaps on the GPU (on
+ *   different streams) race; serialise them.  The array keeps the last call's
+ *   contents, and each call clears what must start at zero.
+ *   A CSR overflow shows as row_ptr[rows] > col_capacity (the status word of
+ *   this variant is not reported). */
+BSA_API bsa_status bsa_select_static(const bsa_params *p, const float *qbar, const float *kbar,
+                                     int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
+                                     int32_t *kept_count, void *stream);
+
 /* Step 3, fine pass ([STAR] "Sol": exact kept blocks + centroids of the
  * others in one FP32 online softmax; [DOC] sink_conditioning).
  *   q, k, v        : [B, N, H, d] inputs.
