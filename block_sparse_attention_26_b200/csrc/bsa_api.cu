@@ -61,6 +61,12 @@ WsLayout ws_layout(const bsa_params &p)
     L.q16 = take(in16);
     L.k16 = take(in16);
     L.v16 = take(in16);
+    const bool ex = D.E > 0;
+    L.ex_theta = take(ex ? (size_t)D.rows * 4 : 0);
+    L.ex_buf = take(ex ? (size_t)D.rows * extra_buffer_capacity() * 8 : 0);
+    L.ex_cnt = take(ex ? (size_t)D.rows * 4 : 0);
+    L.ex_ovf = take(ex ? (size_t)(D.rows + 1) * 4 : 0);
+    L.ex_scratch = take(ex ? (size_t)148 * D.N * 4 : 0);
     L.part_tiles = dense_partial_tiles(D, p.dense_row_end - p.dense_row_begin);
     L.part_o = take((size_t)L.part_tiles * 128 * D.d * sizeof(float));
     L.part_ml = take((size_t)L.part_tiles * 128 * 2 * sizeof(float));
@@ -204,17 +210,21 @@ bsa_status bsa_select(const bsa_params *p, const float *qbar, const float *kbar,
     if (col_capacity < 0) FAIL(BSA_ERR_INVALID_ARG, "col_capacity < 0");
     if (col_capacity > 0 && col_idx == nullptr) FAIL(BSA_ERR_INVALID_ARG, "col_idx is NULL");
     if (p->extra_tokens > 0) {
-        (void)k;
-        (void)extra_idx;
-        (void)extra_count;
-        FAIL(BSA_ERR_UNSUPPORTED, "extra_tokens > 0 is not available in this build yet");
+        if (p->dtype != BSA_DT_BF16) FAIL(BSA_ERR_UNSUPPORTED, "extra tokens need bf16 inputs");
+        TRY(check_tensor(k, "k"));
+        if (extra_idx == nullptr || extra_count == nullptr) FAIL(BSA_ERR_INVALID_ARG, "extra_idx / extra_count is NULL");
     }
     TRY(check_ws(p, ws, ws_bytes));
     const Dims D = dims_of(*p);
     const WsLayout L = ws_layout(*p);
-    return from_cuda(launch_select(*p, D, qbar, kbar, row_ptr, col_idx, col_capacity, kept_count,
-                                   static_cast<char *>(ws), L, (cudaStream_t)stream),
-                     "bsa_select");
+    TRY(from_cuda(launch_select(*p, D, qbar, kbar, row_ptr, col_idx, col_capacity, kept_count,
+                                static_cast<char *>(ws), L, (cudaStream_t)stream),
+                  "bsa_select"));
+    if (p->extra_tokens > 0)
+        TRY(from_cuda(launch_extra(*p, D, qbar, k, extra_idx, extra_count, static_cast<char *>(ws), L,
+                                   (cudaStream_t)stream),
+                      "bsa_select (extra tokens)"));
+    return BSA_OK;
 }
 
 bsa_status bsa_select_static(const bsa_params *p, const float *qbar, const float *kbar, int64_t *row_ptr,

@@ -33,6 +33,11 @@ struct WsLayout {
     size_t cbias;          // [rows, nKB_pad] f32 per-row centroid bias overrides (extra tokens)
     size_t xk16, xv16;     // [rows, E, d] bf16 modified centroids (extra tokens)
     size_t q16, k16, v16;  // [B, N, H, d] bf16 copies of f32 inputs (attention, f32 only)
+    size_t ex_theta;       // [rows] f32 extra-token score bounds
+    size_t ex_buf;         // [rows, 1024] u64 surviving (score, token) pairs
+    size_t ex_cnt;         // [rows] i32 survivors per row
+    size_t ex_ovf;         // [1 + rows] i32 overflowed rows
+    size_t ex_scratch;     // [148, N] u32 fallback keys
     size_t part_o;         // [part_tiles, 128, d] f32 dense-row partial outputs
     size_t part_ml;        // [part_tiles, 128, 2] f32 dense-row partial (max, sum)
     int64_t part_tiles;    // capacity of the partial buffers, in 128-row tiles
@@ -67,6 +72,11 @@ cudaError_t launch_select_static(const bsa_params &p, const Dims &D, const float
                                  int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
                                  int32_t *kept_count, const WsLayout &L, cudaStream_t st);
 size_t static_scratch_bytes();
+
+// Extra tokens (E > 0): survivor buffer capacity per row, and the launch.
+int64_t extra_buffer_capacity();
+cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, const void *k,
+                         int32_t *extra_idx, int32_t *extra_count, char *ws, const WsLayout &L, cudaStream_t st);
 
 // Thread-local host error text.
 void set_error(const char *fmt, ...);

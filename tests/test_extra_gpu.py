@@ -1,0 +1,91 @@
+"""GPU parity of the extra-token selection ("BlockSparseAttention - ComfyUI
+Built-in Node Documentation", general inputs, extra_tokens) against the CPU
+oracle.
+
+The GPU ranks tokens by tensor-core dot products (fp32 accumulation), the
+oracle by fp64 dot products: the selected sets must agree except for tokens
+whose oracle score lies within a relative 1e-4 of the row's E-th score
+(near-ties at the cut), which are counted.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_26_b200 as bsa
+import oracle
+from workloads import CONFIGS, Workload, make_qkv, sample_heads, sample_query_blocks
+
+pytestmark = pytest.mark.gpu
+
+BAND = 1e-4
+
+
+def _gpu_select(w, q, k, v):
+    p = bsa.params_for(w, q)
+    buf = bsa.Buffers(p, q.device)
+    bsa.bsa_pool(p, q, k, v, buf.qbar, buf.kbar, buf.vbar, buf.blk_count)
+    bsa.bsa_select(p, buf.qbar, buf.kbar, k, buf.row_ptr, buf.col_idx, buf.kept_count, buf.extra_idx,
+                   buf.extra_count, buf.ws)
+    assert bsa.bsa_device_status(buf.ws) == 0
+    return p, buf
+
+
+def _row_all_dense(w, r):
+    i = r % w.nQB
+    lo, hi = i * w.q_block, min(w.N, (i + 1) * w.q_block)
+    return lo >= w.dense_rows[0] and hi <= w.dense_rows[1]
+
+
+def _check_rows(w, res, kc, gpu_idx, gpu_cnt, rows):
+    """Compare GPU extras with the oracle's on `rows`; returns the exempted count."""
+    ex, ec, _ = oracle.extra_tokens(res.qbar, oracle.as_raw(kc), res.keep, w.q_block, w.k_block,
+                                    w.extra_tokens, rows)
+    K = kc.double().numpy()
+    exempt = 0
+    for n, r in enumerate(rows):
+        if _row_all_dense(w, r):
+            assert gpu_cnt[r] == 0
+            continue
+        a = set(ex[n, :ec[n]].tolist())
+        g_list = gpu_idx[r, :gpu_cnt[r]].tolist()
+        assert g_list == sorted(g_list), f"row {r}: not ascending"
+        g = set(g_list)
+        assert len(g) == gpu_cnt[r] == ec[n], (r, len(g), gpu_cnt[r], ec[n])
+        diff = a ^ g
+        if not diff:
+            continue
+        b, h, i = r // (w.H * w.nQB), (r // w.nQB) % w.H, r % w.nQB
+        qt = torch.from_numpy(res.qbar[b, h, i]).to(torch.bfloat16).double().numpy()
+        sc = lambda t: float(K[b, t, h] @ qt) / math.sqrt(w.d)
+        t_e = min(sc(t) for t in a)              # the oracle's E-th score
+        for t in diff:
+            assert abs(sc(t) - t_e) <= BAND * (1.0 + abs(t_e)), (r, t, sc(t), t_e)
+        exempt += len(diff)
+    return exempt
+
+
+@pytest.mark.parametrize("E", [64, 256])
+def test_extra_tokens_small(E):
+    w = Workload("extra_small", B=1, H=2, N=2120, d=128, dtype="bf16", method="sol", q_block=64,
+                 k_block=64, tau=1.3, prefix_len=200, dense_rows=(72, 200), extra_tokens=E,
+                 grid=(3, 16, 40), seed=51)
+    qc, kc, vc = make_qkv(w, "cpu")
+    p, buf = _gpu_select(w, qc.cuda(), kc.cuda(), vc.cuda())
+    res = oracle.routing(w, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc), with_extra=False)
+    exempt = _check_rows(w, res, kc, buf.extra_idx.cpu().numpy(), buf.extra_count.cpu().numpy(),
+                         list(range(w.rows)))
+    assert exempt <= w.rows * E // 1000 + 2, exempt
+
+
+def test_extra_tokens_full_size_sampled():
+    w = CONFIGS["sol_sinks"]
+    q, k, v = make_qkv(w, "cuda")
+    p, buf = _gpu_select(w, q, k, v)
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    res = oracle.routing(w, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc), with_extra=False)
+    rows = [(0 * w.H + h) * w.nQB + i for h in sample_heads(w)[:2] for i in sample_query_blocks(w, 16)]
+    exempt = _check_rows(w, res, kc, buf.extra_idx.cpu().numpy(), buf.extra_count.cpu().numpy(), rows)
+    print(f"sol_sinks: {len(rows)} sampled rows, exempted tokens {exempt}")
+    assert exempt <= len(rows) * 2
