@@ -65,7 +65,8 @@ constexpr uint32_t kColS = 0;          // S, 128 columns
 constexpr uint32_t kColP = 128;        // P of half h, buffer b at kColP + 64 h + 32 b
 constexpr uint32_t kColO = 256;        // O of half h at kColO + 128 h
 
-enum : int32_t { TILE_EXACT = 0, TILE_CENT = 1, TILE_END = 2 };
+enum : int32_t { TILE_EXACT = 0, TILE_CENT = 1, TILE_END = 2, TILE_GATHER = 3 };
+constexpr int kMaxE = 256;     // extra tokens per query block (the node's range is 0..256)
 
 #ifdef BSA_TRACE
 // Per-tile clock64() stamps of a few CTAs (development builds only), kept in
@@ -114,6 +115,16 @@ struct AttnArgs {
     int32_t *status;
     long long *trace;            // development builds: per-tile timestamps
     int trace_base;
+    // extra tokens (E > 0): gathered as exact keys; the blocks they came from keep a
+    // centroid over their remaining tokens (per query block)
+    int E, Ecap;
+    const int32_t *extra_idx;    // [rows, E] ascending token indices
+    const int32_t *extra_count;  // [rows]
+    const __nv_bfloat16 *kx, *vx;              // K and V inputs (bf16), output strides
+    const __nv_bfloat16 *xk16, *xv16;          // [rows, Ecap, d] modified centroids
+    const float *xbias;                        // [rows, Ecap] log2 of their token counts
+    const int32_t *xcnt;                       // [rows] modified centroids per row
+    const uint32_t *xaff;                      // [rows, nW] blocks that gave extra tokens
 };
 
 template <int D>
@@ -132,12 +143,16 @@ struct Lay {
     static constexpr int kNumBar = 2 + 2 * kKS + 2 * kVS + 2 + 8;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
     static constexpr int kOffML = kOffMisc + 16;                 // [2][128] (m, l) per half
-    static constexpr int kOffTrace = kOffML + 2 * kM * 8;
-    static constexpr int kOffMask = kOffTrace + kTraceBytes;
+    static constexpr int kOffBias = kOffML + 2 * kM * 8;         // [VS][128] per-column bias (gathers)
+    static constexpr int kOffCodes = kOffBias + kVS * kTK * 4;   // [2 producers][128] gathered rows
+    static constexpr int kOffSBias = kOffCodes + 2 * kTK * 4;    // [128] staged bias of the next gather
+    static constexpr int kOffExt = kOffSBias + kTK * 4;          // [2][kMaxE] extra tokens + [4] counts
+    static constexpr int kOffTrace = kOffExt + 2 * kMaxE * 4 + 16;
+    static constexpr int kOffMask = kOffTrace + kTraceBytes;     // kept [2][nW], then affected [2][nW]
     // at least 116 KB so that a single CTA owns an SM (it allocates all 512 TMEM columns)
     static size_t bytes(int nW)
     {
-        const size_t b = (size_t)kOffMask + 2 * (size_t)nW * 4 + 1024;
+        const size_t b = (size_t)kOffMask + 4 * (size_t)nW * 4 + 1024;
         return b < 116 * 1024 ? 116 * 1024 : b;
     }
 };
@@ -232,6 +247,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(sm + L::kOffMisc + 4);
     float2 *ml = reinterpret_cast<float2 *>(sm + L::kOffML);   // [2 halves][128] (m, l)
     uint32_t *kept = reinterpret_cast<uint32_t *>(sm + L::kOffMask);
+    uint32_t *aff = kept + 2 * a.nW;                            // blocks that gave extra tokens
+    float *bias_sm = reinterpret_cast<float *>(sm + L::kOffBias);
+    int32_t *ext = reinterpret_cast<int32_t *>(sm + L::kOffExt); // [2][kMaxE]
+    int32_t *ext_n = ext + 2 * kMaxE;                            // [2] extra tokens, [2..3] modified centroids
 #ifdef BSA_TRACE
     long long *trace_sm = reinterpret_cast<long long *>(sm + L::kOffTrace);
     for (int i = threadIdx.x; i < kTraceTiles * kTraceEvents; i += blockDim.x) trace_sm[i] = 0;
@@ -262,9 +281,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     if (warp == 8 && !dense) {
-        // kept-block bitmasks of the tile's query blocks, from the CSR lists
-        for (int w = lane; w < 2 * a.nW; w += 32) kept[w] = 0u;
+        // kept-block bitmasks of the tile's query blocks, from the CSR lists; with
+        // extra tokens also their lists and the blocks they came from
+        for (int w = lane; w < 4 * a.nW; w += 32) kept[w] = 0u;
+        if (lane < 4) ext_n[lane] = 0;
         __syncwarp();
+        if (a.E > 0) {
+            for (int q = 0; q < nq; ++q) {
+                const int64_t rq = rbase + q;
+                const int n = min(a.extra_count[rq], a.E);
+                for (int e = lane; e < n; e += 32) ext[q * kMaxE + e] = a.extra_idx[rq * a.E + e];
+                for (int w = lane; w < a.nW; w += 32) aff[q * a.nW + w] = a.xaff[rq * a.nW + w];
+                if (lane == 0) {
+                    ext_n[q] = n;
+                    ext_n[2 + q] = a.xcnt[rq];
+                }
+            }
+        }
         for (int q = 0; q < nq; ++q) {
             const int64_t p0 = a.row_ptr[rbase + q], p1 = a.row_ptr[rbase + q + 1];
             for (int64_t p = p0 + lane; p < p1; p += 32) {
@@ -284,8 +317,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 8 || warp == 10) {
         // ---------------------------------------------------------- producers
+        // Every lane walks the same tile list; lane 0 waits on the ring, issues the
+        // TMA loads and publishes tile metadata; all lanes copy gathered rows.
+        const bool is_k = warp == 8;
         if (lane == 0) {
-            const bool is_k = warp == 8;
             if (is_k) {
                 prefetch_tmap(&tm_q);
                 prefetch_tmap(&tm_k);
@@ -297,28 +332,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                 prefetch_tmap(&tm_v);
                 if (!dense && a.centroid) prefetch_tmap(&tm_vc);
             }
-            const CUtensorMap *tm_x = is_k ? &tm_k : &tm_v;
-            const CUtensorMap *tm_c = is_k ? &tm_kc : &tm_vc;
-            const int depth = is_k ? kKS : kVS;
-            uint64_t *full = is_k ? k_full : v_full;
-            uint64_t *empty = is_k ? k_empty : v_empty;
-            uint8_t *ring = sm + (is_k ? L::kOffK : L::kOffV);
-            int j = 0;
-            // half x of the tile lands at row offset 64 x of every channel chunk
-            auto load_half = [&](uint8_t *dst, int kind, int blk, uint64_t *bar) {
-                for (int dc = 0; dc < D / 64; ++dc) {
-                    uint8_t *d = dst + dc * (kTK * 128);
-                    if (kind == TILE_EXACT)
-                        tma_load_4d(d, tm_x, bar, dc * 64, h, blk * kBK, b);
-                    else
-                        tma_load_3d(d, tm_c, bar, dc * 64, blk * kBK, bh);
-                }
-            };
-            auto push = [&](int kind, const int (&blk)[2], const uint32_t (&who)[2], const int (&nc)[2],
-                            const int (&pcol)[2], float last_bias, const uint64_t (&cm)[2][2]) -> bool {
-                const int s = j % depth;
-                if (j >= depth && !mbar_wait(&empty[s], ((j / depth) - 1) & 1, abort_flag, a.status, is_k ? 10 : 11))
-                    return false;
+        }
+        const CUtensorMap *tm_x = is_k ? &tm_k : &tm_v;
+        const CUtensorMap *tm_c = is_k ? &tm_kc : &tm_vc;
+        const int depth = is_k ? kKS : kVS;
+        uint64_t *full = is_k ? k_full : v_full;
+        uint64_t *empty = is_k ? k_empty : v_empty;
+        uint8_t *ring = sm + (is_k ? L::kOffK : L::kOffV);
+        uint32_t *codes = reinterpret_cast<uint32_t *>(sm + L::kOffCodes) + (is_k ? 0 : kTK);
+        float *stage_bias = reinterpret_cast<float *>(sm + L::kOffSBias);
+        const __nv_bfloat16 *src_x = is_k ? a.kx : a.vx;
+        const __nv_bfloat16 *src_c = is_k ? a.xk16 : a.xv16;
+        int j = 0;
+        // half x of the tile lands at row offset 64 x of every channel chunk
+        auto load_half = [&](uint8_t *dst, int kind, int blk, uint64_t *bar) {
+            for (int dc = 0; dc < D / 64; ++dc) {
+                uint8_t *d = dst + dc * (kTK * 128);
+                if (kind == TILE_EXACT)
+                    tma_load_4d(d, tm_x, bar, dc * 64, h, blk * kBK, b);
+                else
+                    tma_load_3d(d, tm_c, bar, dc * 64, blk * kBK, bh);
+            }
+        };
+        // row address of a gathered column: an extra token of this head, or a
+        // modified centroid (bit 31 set; query block in bit 30, entry in bits 0-29)
+        auto row_src = [&](uint32_t code) -> const __nv_bfloat16 * {
+            if (code & 0x80000000u) {
+                const int q = (code >> 30) & 1, e = (int)(code & 0x3fffffffu);
+                return src_c + ((rbase + q) * a.Ecap + e) * D;
+            }
+            return src_x + (int64_t)b * a.sb + (int64_t)code * a.sn + (int64_t)h * a.sh;
+        };
+        auto push = [&](int kind, const int (&blk)[2], const uint32_t (&who)[2], const int (&nc)[2],
+                        const int (&pcol)[2], float last_bias, const uint64_t (&cm)[2][2]) -> bool {
+            const int s = j % depth;
+            if (j >= depth) {
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(&empty[s], ((j / depth) - 1) & 1, abort_flag, a.status, is_k ? 10 : 11);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+            }
+            if (lane == 0) {
                 if (is_k) {
                     kkind[s] = kind;
                     TRACE(0, j);
@@ -335,7 +388,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     info[s].last_bias = last_bias;
                 }
-                uint8_t *dst = ring + s * L::kTileBytes;
+            }
+            uint8_t *dst = ring + s * L::kTileBytes;
+            if (kind == TILE_GATHER && !is_k)
+                for (int c = lane; c < kTK; c += 32) bias_sm[s * kTK + c] = stage_bias[c];
+            if (kind == TILE_GATHER) {
+                // 128 rows from arbitrary addresses, written in the 128-byte-swizzled
+                // layout the tensor core reads; completion through the barrier
+                const uint32_t base = smem_u32(dst);
+                for (int t = lane; t < kTK * (D / 8); t += 32) {
+                    const int c = t / (D / 8), k16 = t % (D / 8);
+                    const int dc = k16 >> 3, c16 = k16 & 7;
+                    const uint32_t sa = base + dc * (kTK * 128) + (c >> 3) * 1024 + (c & 7) * 128 +
+                                        ((c16 ^ (c & 7)) << 4);
+                    const __nv_bfloat16 *ga = row_src(codes[c]) + k16 * 8;
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(ga) : "memory");
+                }
+                asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[s]);
+            } else if (lane == 0) {
                 if (kind == TILE_END) {
                     mbar_arrive(&full[s]);
                 } else {
@@ -343,84 +416,141 @@ __global__ void __launch_bounds__(kThreads, 1)
                     load_half(dst, kind, blk[0], &full[s]);
                     load_half(dst + L::kHalfBytes, kind, blk[1], &full[s]);
                 }
-                ++j;
-                return true;
-            };
-            const uint64_t zero2[2][2] = {{0, 0}, {0, 0}};
-            const int none[2] = {-1, -1};
-            bool ok = true;
-            // exact tiles: pairs of key blocks; an odd last tile repeats its block
-            // in the empty half (a valid load) with no active column
-            int pend = -1;
-            uint32_t pend_who = 0;
-            auto emit_block = [&](int blk, uint32_t who) {
-                if (pend < 0) {
-                    pend = blk;
-                    pend_who = who;
-                    return;
+            }
+            ++j;
+            return true;
+        };
+        const uint64_t zero2[2][2] = {{0, 0}, {0, 0}};
+        const int none[2] = {-1, -1};
+        bool ok = true;
+        // exact tiles: pairs of key blocks; an odd last tile repeats its block
+        // in the empty half (a valid load) with no active column
+        int pend = -1;
+        uint32_t pend_who = 0;
+        auto emit_block = [&](int blk, uint32_t who) {
+            if (pend < 0) {
+                pend = blk;
+                pend_who = who;
+                return;
+            }
+            const int bl[2] = {pend, blk};
+            const uint32_t wh[2] = {pend_who, who};
+            const int nc[2] = {min(kBK, a.N - pend * kBK), min(kBK, a.N - blk * kBK)};
+            ok = push(TILE_EXACT, bl, wh, nc, none, 0.f, zero2);
+            pend = -1;
+        };
+        if (dense) {
+            for (int blk = kb0; blk < kb1 && ok; ++blk) emit_block(blk, 3u);
+        } else {
+            const uint32_t *k0 = kept, *k1 = kept + a.nW;
+            for (int w = 0; w < a.nW && ok; ++w) {
+                uint32_t u = k0[w] | k1[w];
+                while (u && ok) {
+                    const int bit = __ffs(u) - 1;
+                    u &= u - 1;
+                    emit_block(w * 32 + bit, ((k0[w] >> bit) & 1u) | (((k1[w] >> bit) & 1u) << 1));
                 }
-                const int bl[2] = {pend, blk};
-                const uint32_t wh[2] = {pend_who, who};
-                const int nc[2] = {min(kBK, a.N - pend * kBK), min(kBK, a.N - blk * kBK)};
-                ok = push(TILE_EXACT, bl, wh, nc, none, 0.f, zero2);
-                pend = -1;
-            };
-            if (dense) {
-                for (int blk = kb0; blk < kb1 && ok; ++blk) emit_block(blk, 3u);
-            } else {
-                const uint32_t *k0 = kept, *k1 = kept + a.nW;
-                for (int w = 0; w < a.nW && ok; ++w) {
-                    uint32_t u = k0[w] | k1[w];
-                    while (u && ok) {
-                        const int bit = __ffs(u) - 1;
-                        u &= u - 1;
-                        emit_block(w * 32 + bit, ((k0[w] >> bit) & 1u) | (((k1[w] >> bit) & 1u) << 1));
+            }
+        }
+        if (ok && pend >= 0) {
+            const int bl[2] = {pend, pend};
+            const uint32_t wh[2] = {pend_who, 0u};
+            const int nc[2] = {min(kBK, a.N - pend * kBK), 0};
+            ok = push(TILE_EXACT, bl, wh, nc, none, 0.f, zero2);
+            pend = -1;
+        }
+        if (!dense && a.E > 0 && ok) {
+            // gathered tiles: the union of the two query blocks' extra tokens (in
+            // token order), then each query block's modified centroids
+            const int n0 = ext_n[0], n1 = ext_n[1], m0 = ext_n[2], m1 = ext_n[3];
+            int i0 = 0, i1 = 0, e0 = 0, e1 = 0;
+            const int none2[2] = {-1, -1};
+            const int nc0[2] = {0, 0};
+            const uint32_t wh0[2] = {0u, 0u};
+            while (ok && (i0 < n0 || i1 < n1 || e0 < m0 || e1 < m1)) {
+                uint64_t cm[2][2] = {{0, 0}, {0, 0}};
+                int c = 0;
+                if (lane == 0) {
+                    float *bias = stage_bias;
+                    for (; c < kTK && (i0 < n0 || i1 < n1 || e0 < m0 || e1 < m1); ++c) {
+                        uint32_t code, who;
+                        float bs = 0.f;
+                        if (i0 < n0 || i1 < n1) {
+                            const int t0 = i0 < n0 ? ext[i0] : INT_MAX, t1 = i1 < n1 ? ext[kMaxE + i1] : INT_MAX;
+                            const int t = min(t0, t1);
+                            who = (t0 == t ? 1u : 0u) | (t1 == t ? 2u : 0u);
+                            i0 += t0 == t;
+                            i1 += t1 == t;
+                            code = (uint32_t)t;
+                        } else if (e0 < m0) {
+                            code = 0x80000000u | (uint32_t)e0;
+                            bs = a.xbias[rbase * a.Ecap + e0];
+                            who = 1u;
+                            ++e0;
+                        } else {
+                            code = 0xC0000000u | (uint32_t)e1;
+                            bs = a.xbias[(rbase + 1) * a.Ecap + e1];
+                            who = 2u;
+                            ++e1;
+                        }
+                        codes[c] = code;
+                        if (!is_k) bias[c] = bs;
+                        if (who & 1u) cm[0][c >> 6] |= 1ull << (c & 63);
+                        if (who & 2u) cm[1][c >> 6] |= 1ull << (c & 63);
+                    }
+                    for (int p = c; p < kTK; ++p) {
+                        codes[p] = codes[0];            // a valid row; no column active
+                        if (!is_k) bias[p] = 0.f;
                     }
                 }
+                // the list state lives in lane 0: broadcast it
+                i0 = __shfl_sync(0xffffffffu, i0, 0);
+                i1 = __shfl_sync(0xffffffffu, i1, 0);
+                e0 = __shfl_sync(0xffffffffu, e0, 0);
+                e1 = __shfl_sync(0xffffffffu, e1, 0);
+                for (int x = 0; x < 2; ++x)
+                    for (int y = 0; y < 2; ++y) cm[x][y] = __shfl_sync(0xffffffffu, cm[x][y], 0);
+                __syncwarp();
+                ok = push(TILE_GATHER, none2, wh0, nc0, none2, 0.f, cm);
             }
-            if (ok && pend >= 0) {
-                const int bl[2] = {pend, pend};
-                const uint32_t wh[2] = {pend_who, 0u};
-                const int nc[2] = {min(kBK, a.N - pend * kBK), 0};
-                ok = push(TILE_EXACT, bl, wh, nc, none, 0.f, zero2);
-                pend = -1;
-            }
-            if (!dense && a.centroid && ok) {
-                const int last_n = a.N - (a.nKB - 1) * kBK;
-                const int nchunk = (a.nKB + kBK - 1) / kBK;
-                const uint32_t *k0 = kept, *k1 = kept + a.nW;
-                auto cmask = [&](const uint32_t *k, int cc) -> uint64_t {
-                    if (cc >= nchunk) return 0ull;
-                    const int nb = min(kBK, a.nKB - cc * kBK);
-                    const uint64_t valid = nb == 64 ? ~0ull : ((1ull << nb) - 1ull);
-                    const int w0 = 2 * cc;
-                    const uint64_t lo = w0 < a.nW ? k[w0] : 0u;
-                    const uint64_t hi = w0 + 1 < a.nW ? k[w0 + 1] : 0u;
-                    return valid & ~(lo | (hi << 32));
-                };
-                for (int cc = 0; cc < nchunk && ok; cc += 2) {
-                    uint64_t cm[2][2];
-                    int bl[2], pc[2];
-                    for (int x = 0; x < 2; ++x) {
-                        const int c = cc + x;
-                        cm[0][x] = cmask(k0, c);
-                        cm[1][x] = nq > 1 ? cmask(k1, c) : 0ull;
-                        bl[x] = c < nchunk ? c : cc;          // an empty half repeats a valid chunk
-                        const int lastcol = (a.nKB - 1) - c * kBK;
-                        pc[x] = (c < nchunk && last_n < kBK && lastcol >= 0 && lastcol < kBK) ? lastcol : -1;
-                    }
-                    if ((cm[0][0] | cm[0][1] | cm[1][0] | cm[1][1]) == 0ull) continue;
-                    const uint32_t wh[2] = {0u, 0u};
-                    const int nc[2] = {0, 0};
-                    ok = push(TILE_CENT, bl, wh, nc, pc, last_n < kBK ? log2f((float)last_n) : 0.f, cm);
+        }
+        if (!dense && a.centroid && ok) {
+            const int last_n = a.N - (a.nKB - 1) * kBK;
+            const int nchunk = (a.nKB + kBK - 1) / kBK;
+            const uint32_t *k0 = kept, *k1 = kept + a.nW, *f0 = aff, *f1 = aff + a.nW;
+            auto cmask = [&](const uint32_t *k, const uint32_t *f, int cc) -> uint64_t {
+                if (cc >= nchunk) return 0ull;
+                const int nb = min(kBK, a.nKB - cc * kBK);
+                const uint64_t valid = nb == 64 ? ~0ull : ((1ull << nb) - 1ull);
+                const int w0 = 2 * cc;
+                const uint64_t lo = w0 < a.nW ? (k[w0] | f[w0]) : 0u;
+                const uint64_t hi = w0 + 1 < a.nW ? (k[w0 + 1] | f[w0 + 1]) : 0u;
+                return valid & ~(lo | (hi << 32));
+            };
+            for (int cc = 0; cc < nchunk && ok; cc += 2) {
+                uint64_t cm[2][2];
+                int bl[2], pc[2];
+                for (int x = 0; x < 2; ++x) {
+                    const int c = cc + x;
+                    cm[0][x] = cmask(k0, f0, c);
+                    cm[1][x] = nq > 1 ? cmask(k1, f1, c) : 0ull;
+                    bl[x] = c < nchunk ? c : cc;          // an empty half repeats a valid chunk
+                    const int lastcol = (a.nKB - 1) - c * kBK;
+                    pc[x] = (c < nchunk && last_n < kBK && lastcol >= 0 && lastcol < kBK) ? lastcol : -1;
                 }
-            }
-            if (ok) {
-                const int bl[2] = {0, 0};
+                if ((cm[0][0] | cm[0][1] | cm[1][0] | cm[1][1]) == 0ull) continue;
                 const uint32_t wh[2] = {0u, 0u};
                 const int nc[2] = {0, 0};
-                ok = push(TILE_END, bl, wh, nc, none, 0.f, zero2);
+                ok = push(TILE_CENT, bl, wh, nc, pc, last_n < kBK ? log2f((float)last_n) : 0.f, cm);
             }
+        }
+        if (ok) {
+            const int bl[2] = {0, 0};
+            const uint32_t wh[2] = {0u, 0u};
+            const int nc[2] = {0, 0};
+            ok = push(TILE_END, bl, wh, nc, none, 0.f, zero2);
+        }
+        if (lane == 0) {
             // no TMA write may still be in flight when the CTA exits: wait for the
             // last phase every slot was armed with
             volatile int32_t no_abort = 0;
@@ -555,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 64; ++c) s[c] = c < nc ? s[c] * scale : -INFINITY;
                 }
-            } else {
+            } else if (kind == TILE_CENT) {
                 const uint64_t msk = info[vs].cmask[qsel][hf];
                 const int pc = info[vs].pcol[hf];
                 const float pbias = info[vs].last_bias;
@@ -566,6 +696,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float bias = c == pc ? pbias : 6.0f;       // log2(64) for full blocks
                         s[c] = ((msk >> c) & 1ull) ? fmaf(s[c], scale, bias) : -INFINITY;
                     }
+                }
+            } else {
+                // gathered columns: extra tokens (bias 0) and modified centroids
+                // (bias log2 of their remaining token count)
+                const uint64_t msk = info[vs].cmask[qsel][hf];
+                const float *bias = bias_sm + vs * kTK + 64 * hf;
+                mode = msk ? 2 : 0;
+                if (msk) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        s[c] = ((msk >> c) & 1ull) ? fmaf(s[c], scale, bias[c]) : -INFINITY;
                 }
             }
             uint32_t pk[32];
@@ -766,6 +907,58 @@ __global__ void __launch_bounds__(128) combine_kernel(AttnArgs a, int d)
         a.lse[(int64_t)bh * a.N + n] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
 }
 
+// Per query block with extra tokens: the blocks they came from, and for each
+// such block that keeps tokens a centroid over its remaining tokens, (n k - sum
+// of the extra keys) / (n - e) in fp64 from the f32 block mean, stored in bf16
+// with bias log2(n - e).  One warp per row.
+__global__ void __launch_bounds__(256) modcent_kernel(const int32_t *__restrict__ extra_idx,
+                                                      const int32_t *__restrict__ extra_count,
+                                                      const float *__restrict__ kbar, const float *__restrict__ vbar,
+                                                      const __nv_bfloat16 *__restrict__ k,
+                                                      const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
+                                                      int64_t sh, int64_t rows, int H, int N, int nQB, int nKB, int nW,
+                                                      int d, int E, int Ecap, __nv_bfloat16 *__restrict__ xk,
+                                                      __nv_bfloat16 *__restrict__ xv, float *__restrict__ xbias,
+                                                      int32_t *__restrict__ xcnt, uint32_t *__restrict__ xaff)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * 8 + warp;
+    if (r >= rows) return;
+    const int bh = (int)(r / nQB);
+    const int b = bh / H, h = bh % H;
+    for (int w = lane; w < nW; w += 32) xaff[r * nW + w] = 0u;
+    __syncwarp();
+    const int n = extra_count[r];
+    const int32_t *ex = extra_idx + r * E;
+    int nent = 0;
+    for (int i = 0; i < n;) {
+        const int blk = ex[i] >> 6;
+        int jend = i;
+        while (jend < n && (ex[jend] >> 6) == blk) ++jend;
+        if (lane == 0) xaff[r * nW + (blk >> 5)] |= 1u << (blk & 31);
+        const int nb = min(64, N - blk * 64);
+        const int rem = nb - (jend - i);
+        if (rem > 0) {
+            const float *kb = kbar + ((int64_t)bh * nKB + blk) * d;
+            const float *vb = vbar + ((int64_t)bh * nKB + blk) * d;
+            for (int c = lane; c < d; c += 32) {
+                double sk = (double)nb * (double)kb[c], sv = (double)nb * (double)vb[c];
+                for (int t = i; t < jend; ++t) {
+                    const int64_t off = (int64_t)b * sb + (int64_t)ex[t] * sn + (int64_t)h * sh + c;
+                    sk -= (double)__bfloat162float(k[off]);
+                    sv -= (double)__bfloat162float(v[off]);
+                }
+                xk[(r * Ecap + nent) * d + c] = __float2bfloat16_rn((float)(sk / rem));
+                xv[(r * Ecap + nent) * d + c] = __float2bfloat16_rn((float)(sv / rem));
+            }
+            if (lane == 0) xbias[r * Ecap + nent] = log2f((float)rem);
+            ++nent;
+        }
+        i = jend;
+    }
+    if (lane == 0) xcnt[r] = nent;
+}
+
 // bf16 copies of f32 centroids: elementwise, grid-stride.
 __global__ void to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst, int64_t n)
 {
@@ -889,8 +1082,6 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
                              const int32_t *extra_count, void *out, float *lse, int dense_only,
                              int row_begin, int row_end, char *ws, const WsLayout &L, cudaStream_t st)
 {
-    (void)extra_idx;
-    (void)extra_count;
     const int BH = D.B * D.H;
     int64_t sb = p.stride_b, sn = p.stride_n, sh = p.stride_h;
     const void *q16 = q, *k16 = k, *v16 = v;
@@ -954,6 +1145,30 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     a.trace = nullptr;
     a.trace_base = 0;
 #endif
+    a.E = dense_only ? 0 : D.E;
+    a.Ecap = D.E > 0 ? std::min(D.E, D.nKB) : 0;
+    a.extra_idx = extra_idx;
+    a.extra_count = extra_count;
+    a.kx = static_cast<const __nv_bfloat16 *>(k16);
+    a.vx = static_cast<const __nv_bfloat16 *>(v16);
+    a.xk16 = reinterpret_cast<const __nv_bfloat16 *>(ws + L.xk16);
+    a.xv16 = reinterpret_cast<const __nv_bfloat16 *>(ws + L.xv16);
+    a.xbias = reinterpret_cast<const float *>(ws + L.xbias);
+    a.xcnt = reinterpret_cast<const int32_t *>(ws + L.xcnt);
+    a.xaff = reinterpret_cast<const uint32_t *>(ws + L.xaff);
+    if (a.E > 0) {
+        // the gathers read rows through the input strides
+        if (p.dtype != BSA_DT_BF16) {
+            set_error("extra tokens need bf16 inputs");
+            return cudaErrorInvalidValue;
+        }
+        modcent_kernel<<<(unsigned)ceil_div(D.rows, 8), 256, 0, st>>>(
+            extra_idx, extra_count, kbar, vbar, static_cast<const __nv_bfloat16 *>(k),
+            static_cast<const __nv_bfloat16 *>(v), sb, sn, sh, D.rows, D.H, D.N, D.nQB, D.nKB, D.nW, D.d, D.E,
+            a.Ecap, reinterpret_cast<__nv_bfloat16 *>(ws + L.xk16), reinterpret_cast<__nv_bfloat16 *>(ws + L.xv16),
+            reinterpret_cast<float *>(ws + L.xbias), reinterpret_cast<int32_t *>(ws + L.xcnt),
+            reinterpret_cast<uint32_t *>(ws + L.xaff));
+    }
     a.n_sparse = dense_only ? 0 : (int)ceil_div(D.N, kM);
     a.skip_begin = row_begin;
     a.skip_end = row_end;

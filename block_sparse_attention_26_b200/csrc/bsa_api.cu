@@ -6,6 +6,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
+
 #include "bsa_internal.h"
 
 namespace bsa {
@@ -54,9 +56,12 @@ WsLayout ws_layout(const bsa_params &p)
     L.counts = take((size_t)D.rows * sizeof(int32_t));
     L.kc16 = take((size_t)BH * D.nKB * D.d * 2);
     L.vc16 = take((size_t)BH * D.nKB * D.d * 2);
-    L.cbias = take(0);
-    L.xk16 = take(0);
-    L.xv16 = take(0);
+    const size_t ecap = D.E > 0 ? (size_t)std::min(D.E, D.nKB) : 0;
+    L.xk16 = take((size_t)D.rows * ecap * D.d * 2);
+    L.xv16 = take((size_t)D.rows * ecap * D.d * 2);
+    L.xbias = take((size_t)D.rows * ecap * 4);
+    L.xcnt = take(D.E > 0 ? (size_t)D.rows * 4 : 0);
+    L.xaff = take(D.E > 0 ? (size_t)D.rows * D.nW * 4 : 0);
     const size_t in16 = p.dtype == BSA_DT_F32 ? (size_t)D.B * D.N * D.H * D.d * 2 : 0;
     L.q16 = take(in16);
     L.k16 = take(in16);
@@ -266,8 +271,12 @@ bsa_status bsa_attention(const bsa_params *p, const void *q, const void *k, cons
     }
     (void)blk_count;
     if (row_ptr == nullptr || col_idx == nullptr) FAIL(BSA_ERR_INVALID_ARG, "row_ptr / col_idx is NULL");
-    if (p->extra_tokens > 0)
-        FAIL(BSA_ERR_UNSUPPORTED, "extra_tokens > 0 is not available in this build yet");
+    if (p->extra_tokens > 0) {
+        if (p->dtype != BSA_DT_BF16) FAIL(BSA_ERR_UNSUPPORTED, "extra tokens need bf16 inputs");
+        if (extra_idx == nullptr || extra_count == nullptr) FAIL(BSA_ERR_INVALID_ARG, "extra_idx / extra_count is NULL");
+        TRY(check_tensor(kbar, "kbar"));
+        TRY(check_tensor(vbar, "vbar"));
+    }
     TRY(check_ws(p, ws, ws_bytes));
     const Dims D = dims_of(*p);
     const WsLayout L = ws_layout(*p);

@@ -30,8 +30,10 @@ struct WsLayout {
     size_t bitmask;        // [rows, nW] u32 kept-block bitmask (select)
     size_t counts;         // [rows] i32 kept counts (select)
     size_t kc16, vc16;     // [B*H, nKB, d] bf16 centroids (attention)
-    size_t cbias;          // [rows, nKB_pad] f32 per-row centroid bias overrides (extra tokens)
-    size_t xk16, xv16;     // [rows, E, d] bf16 modified centroids (extra tokens)
+    size_t xk16, xv16;     // [rows, min(E, nKB), d] bf16 modified centroids (extra tokens)
+    size_t xbias;          // [rows, min(E, nKB)] f32 their log2 token counts
+    size_t xcnt;           // [rows] i32 modified centroids per row
+    size_t xaff;           // [rows, nW] u32 blocks that gave extra tokens
     size_t q16, k16, v16;  // [B, N, H, d] bf16 copies of f32 inputs (attention, f32 only)
     size_t ex_theta;       // [rows] f32 extra-token score bounds
     size_t ex_buf;         // [rows, 1024] u64 surviving (score, token) pairs

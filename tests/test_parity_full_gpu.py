@@ -31,7 +31,7 @@ def _sample_tokens(w):
     return np.array(toks, np.int64)
 
 
-@pytest.mark.parametrize("name", ["sol_mid", "sla_topk", "long"])
+@pytest.mark.parametrize("name", ["sol_mid", "sla_topk", "sol_sinks", "long"])
 def test_full_size_parity(name):
     w = CONFIGS[name]
     q, k, v = make_qkv(w, "cuda")
@@ -39,7 +39,11 @@ def test_full_size_parity(name):
     assert status == 0
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     qr, kr, vr = oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc)
-    res = oracle.routing(w, qr, kr, vr, with_extra=False)
+    toks = _sample_tokens(w)
+    extra_rows = None
+    if w.extra_tokens > 0:
+        extra_rows = sorted({(int(b) * w.H + int(h)) * w.nQB + int(n) // w.q_block for b, h, n in toks})
+    res = oracle.routing(w, qr, kr, vr, extra_rows=extra_rows)
     # pooled means: bit for bit
     assert np.array_equal(buf.qbar.cpu().numpy(), res.qbar)
     assert np.array_equal(buf.kbar.cpu().numpy(), res.kbar)
@@ -48,7 +52,6 @@ def test_full_size_parity(name):
     exempt = compare_masks(mask, res, w)
     print(f"{name}: kept fraction {mask.mean():.4f}, exempt blocks {exempt}")
     # outputs on the sampled rows
-    toks = _sample_tokens(w)
     ref, ref_lse = oracle.layer_rows(w, qr, kr, vr, res, toks)
     got = out[toks[:, 0], toks[:, 2], toks[:, 1]].float().cpu().numpy()
     mx, mean = compare_outputs(got, ref, name)

@@ -36,6 +36,11 @@ SMALL = {
     "dense_split": Workload("dense_split", B=1, H=1, N=20032, d=128, dtype="bf16", method="sol", q_block=64,
                             k_block=64, tau=1.5, prefix_len=256, dense_rows=(100, 300), grid=(4, 24, 206),
                             seed=20),
+    "sol_extra64": Workload("sol_extra64", B=1, H=2, N=2120, d=128, dtype="bf16", method="sol", q_block=64,
+                            k_block=64, tau=1.3, prefix_len=200, dense_rows=(72, 200), extra_tokens=64,
+                            grid=(3, 16, 40), seed=21),
+    "sol_extra256": Workload("sol_extra256", B=1, H=2, N=3000, d=128, dtype="bf16", method="sol", q_block=64,
+                             k_block=64, tau=1.0, extra_tokens=256, grid=(3, 20, 50), seed=22),
     "no_diag_no_sink": Workload("no_diag_no_sink", B=1, H=2, N=1300, d=128, dtype="bf16", method="sol",
                                 q_block=64, k_block=64, tau=1.0, sink_blocks=0, keep_diag=0,
                                 grid=(2, 13, 50), seed=18),
