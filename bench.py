@@ -33,7 +33,7 @@ if ROOT not in sys.path:
 
 from workloads import CONFIGS, make_qkv  # noqa: E402
 
-DEFAULT_CONFIG = "long"
+DEFAULT_CONFIG = "sol_sinks"
 METRIC = "sparse-attn ms/layer & dense-equiv TFLOP/s at N tokens; % roofline (kept FLOPs)"
 UNIT = "TFLOP/s (dense-equivalent)"
 
@@ -68,9 +68,12 @@ def dense_equiv_flops(w) -> float:
     return 4.0 * w.B * w.H * float(w.N) * w.N * w.d
 
 
-def kept_flops(w, row_ptr: torch.Tensor, col: torch.Tensor) -> float:
+def kept_flops(w, row_ptr: torch.Tensor, col: torch.Tensor, extra_count=None) -> float:
     """FLOPs of the fine pass actually required: 4*d per (query row, key) pair over
-    the exact keys and centroids of every sparse row, plus 4*d*N per dense row."""
+    the exact keys (kept blocks and extra tokens) and centroids of every sparse
+    row, plus 4*d*N per dense row.  A block that gave extra tokens still counts
+    one (modified) centroid; the rare block whose every token became an extra
+    token is counted too (an overcount below 1 %)."""
     rp = row_ptr.to(torch.int64)
     cnt = (rp[1:] - rp[:-1]).view(w.B, w.H, w.nQB)
     nnz = int(rp[-1])
@@ -81,6 +84,8 @@ def kept_flops(w, row_ptr: torch.Tensor, col: torch.Tensor) -> float:
     short = torch.zeros(cnt.numel(), dtype=torch.int64, device=c.device)
     short.index_add_(0, row_of, (c == w.nKB - 1).to(torch.int64))
     exact_keys = cnt.reshape(-1) * w.k_block - short * (w.k_block - last_n)
+    if extra_count is not None:
+        exact_keys = exact_keys + extra_count.to(torch.int64).reshape(-1)
     cent = (w.nKB - cnt.reshape(-1)) if w.centroid else torch.zeros_like(exact_keys)
     per_row_keys = (exact_keys + cent).view(w.B, w.H, w.nQB).double()
     # query rows per query block (the last one may be short)
@@ -325,7 +330,7 @@ def main():
     status = bsa.bsa_device_status(buf.ws, stream)
     if status != 0:
         raise SystemExit(f"device status {status} after warm-up")
-    flops_kept = kept_flops(w, buf.row_ptr, buf.col_idx)
+    flops_kept = kept_flops(w, buf.row_ptr, buf.col_idx, buf.extra_count)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -392,7 +397,8 @@ def main():
     # the dense-row merge when dense rows are split, bf16 centroids (2), bf16 inputs (3)
     dense_split = w.dense_rows[1] > w.dense_rows[0] and w.N > 256 * 64
     launches_per_step = (1 + 4 + 1 + (1 if dense_split else 0) + (2 if w.centroid else 0)
-                         + (3 if w.dtype == "f32" else 0))
+                         + (3 if w.dtype == "f32" else 0)
+                         + (5 if w.extra_tokens > 0 else 0))   # theta, filter, finalize, fallback, modcent
     line = {
         "metric": METRIC,
         "value": world * dense_equiv_flops(w) / (ms_step * 1e-3) / 1e12,
@@ -417,6 +423,7 @@ def main():
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
                      "traffic": attn_traffic(w),
                      "traffic_unit": "bytes per launch (ncu dram read+write, scaled from a 4-head capture)"},
+        "extra_tokens_per_row": (float(buf.extra_count.float().mean()) if buf.extra_count is not None else 0.0),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
         "e2e": e2e,

@@ -907,29 +907,52 @@ __global__ void __launch_bounds__(128) combine_kernel(AttnArgs a, int d)
         a.lse[(int64_t)bh * a.N + n] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
 }
 
+template <int CPL>
+__device__ __forceinline__ void load_bf16_vec(const __nv_bfloat16 *p, float (&f)[CPL])
+{
+    if constexpr (CPL == 4) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(p));
+        f[0] = __uint_as_float(w.x << 16);
+        f[1] = __uint_as_float(w.x & 0xffff0000u);
+        f[2] = __uint_as_float(w.y << 16);
+        f[3] = __uint_as_float(w.y & 0xffff0000u);
+    } else {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(p));
+        f[0] = __uint_as_float(w << 16);
+        f[1] = __uint_as_float(w & 0xffff0000u);
+    }
+}
+
 // Per query block with extra tokens: the blocks they came from, and for each
 // such block that keeps tokens a centroid over its remaining tokens, (n k - sum
 // of the extra keys) / (n - e) in fp64 from the f32 block mean, stored in bf16
 // with bias log2(n - e).  One warp per row.
+// CPL = d / 32 channels per lane; each lane reads its channels of a token with
+// one vector load, four tokens in flight.
+template <int CPL>
 __global__ void __launch_bounds__(256) modcent_kernel(const int32_t *__restrict__ extra_idx,
                                                       const int32_t *__restrict__ extra_count,
                                                       const float *__restrict__ kbar, const float *__restrict__ vbar,
                                                       const __nv_bfloat16 *__restrict__ k,
                                                       const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
                                                       int64_t sh, int64_t rows, int H, int N, int nQB, int nKB, int nW,
-                                                      int d, int E, int Ecap, __nv_bfloat16 *__restrict__ xk,
+                                                      int E, int Ecap, __nv_bfloat16 *__restrict__ xk,
                                                       __nv_bfloat16 *__restrict__ xv, float *__restrict__ xbias,
                                                       int32_t *__restrict__ xcnt, uint32_t *__restrict__ xaff)
 {
+    constexpr int d = 32 * CPL;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * 8 + warp;
     if (r >= rows) return;
     const int bh = (int)(r / nQB);
     const int b = bh / H, h = bh % H;
+    const int c0 = lane * CPL;
     for (int w = lane; w < nW; w += 32) xaff[r * nW + w] = 0u;
     __syncwarp();
     const int n = extra_count[r];
     const int32_t *ex = extra_idx + r * E;
+    const __nv_bfloat16 *kh = k + (int64_t)b * sb + (int64_t)h * sh + c0;
+    const __nv_bfloat16 *vh = v + (int64_t)b * sb + (int64_t)h * sh + c0;
     int nent = 0;
     for (int i = 0; i < n;) {
         const int blk = ex[i] >> 6;
@@ -939,17 +962,52 @@ __global__ void __launch_bounds__(256) modcent_kernel(const int32_t *__restrict_
         const int nb = min(64, N - blk * 64);
         const int rem = nb - (jend - i);
         if (rem > 0) {
-            const float *kb = kbar + ((int64_t)bh * nKB + blk) * d;
-            const float *vb = vbar + ((int64_t)bh * nKB + blk) * d;
-            for (int c = lane; c < d; c += 32) {
-                double sk = (double)nb * (double)kb[c], sv = (double)nb * (double)vb[c];
-                for (int t = i; t < jend; ++t) {
-                    const int64_t off = (int64_t)b * sb + (int64_t)ex[t] * sn + (int64_t)h * sh + c;
-                    sk -= (double)__bfloat162float(k[off]);
-                    sv -= (double)__bfloat162float(v[off]);
+            const float *kb = kbar + ((int64_t)bh * nKB + blk) * d + c0;
+            const float *vb = vbar + ((int64_t)bh * nKB + blk) * d + c0;
+            double sk[CPL], sv[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                sk[j] = (double)nb * (double)kb[j];
+                sv[j] = (double)nb * (double)vb[j];
+            }
+            // block sum minus the extra tokens, in token order
+            int t = i;
+            for (; t + 4 <= jend; t += 4) {
+                float fk[4][CPL], fv[4][CPL];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    load_bf16_vec<CPL>(kh + (int64_t)ex[t + u] * sn, fk[u]);
+                    load_bf16_vec<CPL>(vh + (int64_t)ex[t + u] * sn, fv[u]);
                 }
-                xk[(r * Ecap + nent) * d + c] = __float2bfloat16_rn((float)(sk / rem));
-                xv[(r * Ecap + nent) * d + c] = __float2bfloat16_rn((float)(sv / rem));
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int j = 0; j < CPL; ++j) {
+                        sk[j] -= (double)fk[u][j];
+                        sv[j] -= (double)fv[u][j];
+                    }
+            }
+            for (; t < jend; ++t) {
+                float fk[CPL], fv[CPL];
+                load_bf16_vec<CPL>(kh + (int64_t)ex[t] * sn, fk);
+                load_bf16_vec<CPL>(vh + (int64_t)ex[t] * sn, fv);
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    sk[j] -= (double)fk[j];
+                    sv[j] -= (double)fv[j];
+                }
+            }
+            __nv_bfloat16 ok[CPL], ov[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                ok[j] = __float2bfloat16_rn((float)(sk[j] / rem));
+                ov[j] = __float2bfloat16_rn((float)(sv[j] / rem));
+            }
+            __nv_bfloat16 *dk = xk + (r * Ecap + nent) * d + c0, *dv = xv + (r * Ecap + nent) * d + c0;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                dk[j] = ok[j];
+                dv[j] = ov[j];
             }
             if (lane == 0) xbias[r * Ecap + nent] = log2f((float)rem);
             ++nent;
@@ -1162,9 +1220,10 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
             set_error("extra tokens need bf16 inputs");
             return cudaErrorInvalidValue;
         }
-        modcent_kernel<<<(unsigned)ceil_div(D.rows, 8), 256, 0, st>>>(
+        auto mc = D.d == 128 ? modcent_kernel<4> : modcent_kernel<2>;
+        mc<<<(unsigned)ceil_div(D.rows, 8), 256, 0, st>>>(
             extra_idx, extra_count, kbar, vbar, static_cast<const __nv_bfloat16 *>(k),
-            static_cast<const __nv_bfloat16 *>(v), sb, sn, sh, D.rows, D.H, D.N, D.nQB, D.nKB, D.nW, D.d, D.E,
+            static_cast<const __nv_bfloat16 *>(v), sb, sn, sh, D.rows, D.H, D.N, D.nQB, D.nKB, D.nW, D.E,
             a.Ecap, reinterpret_cast<__nv_bfloat16 *>(ws + L.xk16), reinterpret_cast<__nv_bfloat16 *>(ws + L.xv16),
             reinterpret_cast<float *>(ws + L.xbias), reinterpret_cast<int32_t *>(ws + L.xcnt),
             reinterpret_cast<uint32_t *>(ws + L.xaff));

@@ -15,12 +15,22 @@
 //                    largest, lowered by a safety margin, is a lower bound of
 //                    the row's true E-th score (they are real candidates).
 //   filter_kernel    tcgen05: S = Qt K^T for 128 query blocks x 128 tokens per
-//                    tile, streamed over all tokens; each row's thread keeps
-//                    the candidate tokens scoring >= its bound, in token order.
+//                    tile, streamed over all tokens, twice.  Pass A counts the
+//                    row's unselected tokens into 88 linear buckets from its
+//                    bound up and keeps the highest bucket with at least E
+//                    tokens at or above it; it counts only from a floor, the
+//                    highest bucket already holding E counted tokens, which
+//                    rises as the pass goes.  Pass B keeps the tokens in or
+//                    above the kept bucket, in token order.  Both passes compute
+//                    the same scores and the bucket map is monotone, so the
+//                    survivors include the true top E.  Two warps share each
+//                    row, one per 64-token block of a tile; in pass B they
+//                    swap per-tile counts so the row's list stays in order.
 //   finalize_kernel  one warp per row: exact E-th largest of the survivors by
 //                    radix select, ties resolved by token order, compaction.
 //   fallback_kernel  rows whose survivors overflowed the buffer: all candidate
 //                    scores into a scratch row, radix select over the row.
+#include <float.h>
 #include <math.h>
 
 #include <algorithm>
@@ -33,8 +43,12 @@ namespace {
 
 constexpr int kRowsPerCta = 128;   // query blocks per filter CTA (UMMA M)
 constexpr int kTok = 128;          // tokens per filter tile (UMMA N)
-constexpr int kFS = 4;             // K ring depth of the filter kernel
-constexpr int kSampleBlocks = 4;   // best unselected blocks beyond ceil(E/64) sampled for theta
+constexpr int kSampleBlocks = 0;   // best unselected blocks beyond ceil(E/64) sampled for theta
+constexpr int kBuckets = 88;       // pass-A histogram buckets per row
+constexpr int kHistPitch = kBuckets + 1;   // words per row: a row's buckets fall in distinct banks
+constexpr int kStagePitch = 33;            // words per staged row
+constexpr int kLaneMax = 3;                // most set bits per row a warp walks row by row
+constexpr float kSpan = 2.f;       // buckets cover [theta, theta + kSpan * (sampled max - theta)]
 
 // Order-preserving map of a float to uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t ord_key(float f)
@@ -60,6 +74,8 @@ struct ExArgs {
     const uint32_t *bitmask;           // [rows, nW] kept blocks
     int dense_begin, dense_end;
     float *theta;                      // [rows] raw-dot lower bounds (+inf: no extras)
+    float *smax;                       // [rows] largest sampled score
+    int32_t *bucket;                   // [rows] lowest bucket kept by pass B (-1: every unselected token)
     unsigned long long *buf;           // [rows, cap] (ord key << 32 | token)
     int32_t *cnt;                      // [rows] survivors (may exceed cap)
     int32_t *ovf;                      // [0]: count, [1..]: overflowed rows
@@ -130,7 +146,10 @@ __global__ void __launch_bounds__(256) theta_kernel(ExArgs a)
     const int64_t r = (int64_t)blockIdx.x * 8 + warp;
     if (r >= a.rows) return;
     if (row_all_dense(a, r)) {
-        if (lane == 0) a.theta[r] = INFINITY;
+        if (lane == 0) {
+            a.theta[r] = INFINITY;
+            a.smax[r] = INFINITY;
+        }
         return;
     }
     const int bh = (int)(r / a.nQB);
@@ -138,10 +157,11 @@ __global__ void __launch_bounds__(256) theta_kernel(ExArgs a)
     const uint32_t *bm = a.bitmask + r * a.nW;
     const float *srow = a.S + r * a.nKB;
     for (int c = lane; c < a.d; c += 32) qs[warp][c] = __bfloat162float(__float2bfloat16_rn(a.qbar[r * a.d + c]));
-    // best unselected blocks by pooled score (m rounds of warp argmax)
-    const int m = min(8, (a.E + 63) / 64 + kSampleBlocks);   // at most 512 sampled tokens
-    int got = 0;
-    for (int t = 0; t < m; ++t) {
+    // best unselected blocks by pooled score (rounds of warp argmax) until the
+    // sample holds E tokens (a partial last block holds fewer than 64), at most
+    // 8 blocks = 512 tokens
+    int got = 0, ntok = 0;
+    for (int t = 0; t < 8 && ntok < a.E + 64 * kSampleBlocks; ++t) {
         float best = -INFINITY;
         int bi = -1;
         for (int j = lane; j < a.nKB; j += 32) {
@@ -168,6 +188,7 @@ __global__ void __launch_bounds__(256) theta_kernel(ExArgs a)
         if (lane == 0) blks[warp][got] = bi;
         __syncwarp();
         ++got;
+        ntok += min(64, a.N - bi * 64);
     }
     // token scores of the sampled blocks (raw dot products)
     int n = 0;
@@ -192,6 +213,10 @@ __global__ void __launch_bounds__(256) theta_kernel(ExArgs a)
     }
     __syncwarp();
     float th = -INFINITY;
+    uint32_t mx = 0;
+    for (int j = lane; j < n; j += 32) mx = max(mx, keys[warp][j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     if (n >= a.E) {
         int need;
         const uint32_t *kk = keys[warp];
@@ -199,24 +224,62 @@ __global__ void __launch_bounds__(256) theta_kernel(ExArgs a)
         const float v = key_to_float(vk);
         th = v - (1e-3f * fabsf(v) + 1e-3f);   // covers fp32 accumulation-order differences
     }
-    if (lane == 0) a.theta[r] = th;
+    if (lane == 0) {
+        a.theta[r] = th;
+        a.smax[r] = n > 0 ? key_to_float(mx) : -INFINITY;
+    }
 }
 
 // ------------------------------------------------------------------ filter
 
+__device__ __forceinline__ void red_shared_add1(uint32_t addr)
+{
+    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
+}
+
 template <int D>
 struct FLay {
+    static constexpr int kFS = D == 128 ? 3 : 4;            // K ring depth
     static constexpr int kQBytes = kRowsPerCta * D * 2;
     static constexpr int kKBytes = kTok * D * 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kQBytes;
     static constexpr int kOffBar = kOffK + kFS * kKBytes;   // k_full[FS], k_empty[FS], s_full[2], s_free[2], done
     static constexpr int kOffMisc = kOffBar + (2 * kFS + 5) * 8;
-    static constexpr size_t bytes = (size_t)kOffMisc + 16 + 1024;
+    static constexpr int kOffHist = kOffMisc + 16;                              // [128 rows][kHistPitch] u32
+    static constexpr int kOffPair = kOffHist + kRowsPerCta * kHistPitch * 4;    // [2][2 groups][128 rows] i32
+    static constexpr int kOffStage = kOffPair + 4 * kRowsPerCta * 4;            // [8 warps][32 rows][33] u32
+    static constexpr int kOffBase = kOffStage + 8 * 32 * kStagePitch * 4;       // [8 warps][32] i32
+    static constexpr int kOffList = kOffBase + 8 * 32 * 4;                      // [8 warps][1024] u16
+    static constexpr size_t bytes = (size_t)kOffList + 8 * 1024 * 2 + 1024;
+    static_assert(bytes <= 232448, "filter tile exceeds the per-block shared memory limit");
 };
 
-template <int D>
-__global__ void __launch_bounds__(192, 1) filter_kernel(const __grid_constant__ CUtensorMap tm_k, ExArgs a)
+// v[e] for a runtime e in [0, 32) without local memory: a 5-level select tree.
+__device__ __forceinline__ uint32_t select32(const uint32_t *v, int e)
+{
+    uint32_t a16[16], a8[8], a4[4], a2[2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a16[i] = (e & 1) ? v[2 * i + 1] : v[2 * i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a8[i] = (e & 2) ? a16[2 * i + 1] : a16[2 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a4[i] = (e & 4) ? a8[2 * i + 1] : a8[2 * i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) a2[i] = (e & 8) ? a4[2 * i + 1] : a4[2 * i];
+    return (e & 16) ? a2[1] : a2[0];
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Warps 0-7 read the scores: warp w takes the rows of TMEM lane quarter w & 3
+// and, of each 128-token tile, key block 2t + (w >> 2).  Warp 8 loads K tiles,
+// warp 9 issues the MMAs and owns TMEM.
+template <int D, bool kCount>
+__global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ CUtensorMap tm_k, ExArgs a)
 {
     using L = FLay<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -227,33 +290,50 @@ __global__ void __launch_bounds__(192, 1) filter_kernel(const __grid_constant__ 
     const int i0 = blockIdx.x * kRowsPerCta;
     const int ntiles = (a.N + kTok - 1) / kTok;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kOffBar);
-    uint64_t *k_full = bars, *k_empty = bars + kFS, *s_full = bars + 2 * kFS, *s_free = s_full + 2,
+    uint64_t *k_full = bars, *k_empty = bars + L::kFS, *s_full = bars + 2 * L::kFS, *s_free = s_full + 2,
              *bar_done = s_full + 4;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kOffMisc);
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(sm + L::kOffMisc + 4);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sm + L::kOffHist);   // [row][kHistPitch]
+
+    // Per-row bucket map.  y = fma_rz(x, w, 2^23 + 1 - th w) clamped to 2^23 +
+    // kBuckets - 1, so that for x >= th the bits of y are 0x4B000000 + 1 +
+    // trunc((x - th) w) up to rounding (bucket 0 takes the rounding slack just
+    // below th).  w spreads the buckets over [th, th + kSpan (smax - th)]: the
+    // sampled maximum need not bound the row, so the range reaches well past
+    // it, and the last bucket is open-ended.  y is monotone in x, and both
+    // passes compute it identically, which is all exactness needs.  th = +inf
+    // marks rows without extra tokens; -FLT_MAX stands in for "no bound".
+    const int r = threadIdx.x & (kRowsPerCta - 1);
+    const int64_t row = (int64_t)bh * a.nQB + min(i0 + r, a.nQB - 1);
+    const bool live = i0 + r < a.nQB;
+    const float th0 = live ? a.theta[row] : INFINITY;
+    const float th = fmaxf(th0, -FLT_MAX);
+    const float hi = live ? a.smax[row] : 0.f;
+    const float inv_w = (hi > th && hi < INFINITY) ? (float)kBuckets / (kSpan * (hi - th)) : 0.f;
+    const float cw = 8388609.f - th * inv_w;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kFS; ++s) {
+        for (int s = 0; s < L::kFS; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);
+            mbar_init(&s_free[i], 8);
         }
         mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
     if (warp < 4) {
         // rounded pooled queries of the 128 rows -> the A operand (128-byte swizzle)
-        const int r = threadIdx.x;
         const int i = i0 + r;
-        const float *q = a.qbar + ((int64_t)bh * a.nQB + min(i, a.nQB - 1)) * D;
+        const float *q = a.qbar + row * D;
         const uint32_t base = smem_u32(sm + L::kOffQ) + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll 1
         for (int ch = 0; ch < D / 8; ++ch) {
@@ -264,18 +344,20 @@ __global__ void __launch_bounds__(192, 1) filter_kernel(const __grid_constant__ 
             st_shared_v4(base + dc * (kRowsPerCta * 128) + ((c16 ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
         }
         fence_async_smem();
+        if (kCount)
+            for (int k = 0; k < kBuckets; ++k) hist[r * kHistPitch + k] = 0;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == 8) {
         if (lane == 0) {
             prefetch_tmap(&tm_k);
             for (int t = 0; t < ntiles; ++t) {
-                const int s = t % kFS;
-                if (t >= kFS && !mbar_wait(&k_empty[s], ((t / kFS) - 1) & 1, abort_flag, a.status, 40)) break;
+                const int s = t % L::kFS;
+                if (t >= L::kFS && !mbar_wait(&k_empty[s], ((t / L::kFS) - 1) & 1, abort_flag, a.status, 40)) break;
                 mbar_expect_tx(&k_full[s], L::kKBytes);
                 uint8_t *dst = sm + L::kOffK + s * L::kKBytes;
                 for (int half = 0; half < 2; ++half)
@@ -284,18 +366,18 @@ __global__ void __launch_bounds__(192, 1) filter_kernel(const __grid_constant__ 
                                     t * kTok + half * 64, b);
             }
             volatile int32_t no_abort = 0;
-            for (int s = 0; s < kFS; ++s) {
-                const int n = (ntiles - s + kFS - 1) / kFS;
+            for (int s = 0; s < L::kFS; ++s) {
+                const int n = (ntiles - s + L::kFS - 1) / L::kFS;
                 if (n > 0) mbar_wait(&k_full[s], (n - 1) & 1, &no_abort, a.status, 41);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(kRowsPerCta, kTok, 0, 0);
             const uint32_t q_addr = smem_u32(sm + L::kOffQ), k_addr = smem_u32(sm + L::kOffK);
             for (int t = 0; t < ntiles; ++t) {
-                const int s = t % kFS, sb = t & 1;
-                if (!mbar_wait(&k_full[s], (t / kFS) & 1, abort_flag, a.status, 42)) break;
+                const int s = t % L::kFS, sb = t & 1;
+                if (!mbar_wait(&k_full[s], (t / L::kFS) & 1, abort_flag, a.status, 42)) break;
                 if (t >= 2 && !mbar_wait(&s_free[sb], ((t >> 1) - 1) & 1, abort_flag, a.status, 43)) break;
                 tc_fence_after();
 #pragma unroll
@@ -313,52 +395,192 @@ __global__ void __launch_bounds__(192, 1) filter_kernel(const __grid_constant__ 
             mbar_wait(bar_done, 0, &no_abort, a.status, 44);
         }
     } else {
-        const int r = threadIdx.x;
-        const int i = i0 + r;
-        const int64_t row = (int64_t)bh * a.nQB + min(i, a.nQB - 1);
-        const bool live = i < a.nQB;
-        const float th = live ? a.theta[row] : INFINITY;
-        const uint32_t *bm = a.bitmask + row * a.nW;
+        const int g = warp >> 2, sub = warp & 3;
+        const bool active = th0 < INFINITY;
+        const float ytop = 8388608.f + (float)(kBuckets - 1);
+        // pass B keeps y >= yk; keep_from < 0 (fewer than E candidates) keeps all
+        const int kf = (kCount || !live) ? 0 : a.bucket[row];
+        const float yk = kf < 0 ? -INFINITY : 8388608.f + (float)kf;
+        int32_t *pair = reinterpret_cast<int32_t *>(sm + L::kOffPair);
+        uint32_t *stage = reinterpret_cast<uint32_t *>(sm + L::kOffStage) + warp * 32 * kStagePitch;
+        int32_t *base = reinterpret_cast<int32_t *>(sm + L::kOffBase) + warp * 32;
+        uint16_t *list = reinterpret_cast<uint16_t *>(sm + L::kOffList) + warp * 1024;
         unsigned long long *out = a.buf + row * a.cap;
-        int cnt = 0;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        uint32_t word = 0;
-        int word_idx = -1;
-        for (int t = 0; t < ntiles; ++t) {
-            const int sb = t & 1;
-            bool ok = mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag, a.status, 45);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int c0 = 0; c0 < kTok; c0 += 32) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_base + 128 * sb + c0, v);
-                tmem_ld_wait();
-                if (th == INFINITY) continue;
+        // hist + 4 (kHistPitch r + bucket) = hbase0 + 4 kHistPitch r + 4 bits(y), wrapping mod 2^32
+        const uint32_t hbase0 = smem_u32(hist) - 4u * 0x4B000000u;
+        const uint32_t hrow = hbase0 + 4u * (uint32_t)(kHistPitch * r);
+        // Pass A counts only buckets >= floor.  The floor is the highest bucket
+        // already holding E counted tokens at or above it; it only rises, so the
+        // final cut is never below it and the counts from the cut up stay exact.
+        int floor_k = 0;
+        auto raise_floor = [&]() {
+            uint32_t acc = 0;
+            for (int k0 = kBuckets - 8; k0 + 7 > floor_k; k0 -= 8) {   // eight loads in flight
+                uint32_t h8[8];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int tok = t * kTok + c0 + e;
-                    const float sc = __uint_as_float(v[e]);
-                    if (tok >= a.N || !(sc >= th)) continue;
-                    const int blk = tok >> 6;
-                    if ((blk >> 5) != word_idx) {
-                        word_idx = blk >> 5;
-                        word = bm[word_idx];
+                for (int j = 0; j < 8; ++j) h8[j] = hist[r * kHistPitch + k0 + j];
+#pragma unroll
+                for (int j = 7; j >= 0; --j) {
+                    acc += h8[j];
+                    if (acc >= (uint32_t)a.E && k0 + j > floor_k) {
+                        floor_k = k0 + j;
+                        return;
                     }
-                    if ((word >> (blk & 31)) & 1u) continue;
-                    if (cnt < a.cap) out[cnt] = ((unsigned long long)ord_key(sc) << 32) | (uint32_t)tok;
-                    ++cnt;
                 }
             }
+        };
+        const uint32_t *bm = a.bitmask + row * a.nW;
+        int cnt = 0;   // pass B: survivors of this row so far (both warps of the row agree)
+        const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
+        uint32_t word = bm[g >> 5];
+        for (int t = 0; t < ntiles; ++t) {
+            const int sb = t & 1;
+            const int blk = 2 * t + g;
+            // bitmask word of the next tile's block, fetched a tile early
+            const uint32_t word_next = bm[min((blk + 2) >> 5, a.nW - 1)];
+            // After an abort every wait fails at once: the loop still runs to the
+            // end with no work, so both warps of a row meet at every pair barrier.
+            const bool go = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag, a.status, 45));
+            tc_fence_after();
+            uint32_t v[64];
+            if (go) {
+                tmem_ld32(tmem + lane_base + 128 * sb + 64 * g, *reinterpret_cast<uint32_t(*)[32]>(v));
+                tmem_ld32(tmem + lane_base + 128 * sb + 64 * g + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 64; ++e) v[e] = 0u;
+            }
+            const int tok0 = blk * 64;
+            const bool use = go && active && blk < a.nKB && !((word >> (blk & 31)) & 1u);
+            const int nvalid = max(0, min(64, a.N - tok0));
+            // threshold in bucket space: pass A counts from the floor up, pass B
+            // keeps from the cut up
+            const float ythr = kCount ? 8388608.f + (float)floor_k : yk;
+            uint32_t m0 = 0, m1 = 0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const float y0 = __fmaf_rz(__uint_as_float(v[e]), inv_w, cw);
+                const float y1 = __fmaf_rz(__uint_as_float(v[32 + e]), inv_w, cw);
+                m0 |= (y0 >= ythr) ? (1u << e) : 0u;
+                m1 |= (y1 >= ythr) ? (1u << e) : 0u;
+            }
+            if (!use) m0 = m1 = 0;
+            if (nvalid < 64) {   // tokens past the end
+                m0 &= nvalid >= 32 ? 0xffffffffu : (1u << nvalid) - 1u;
+                m1 &= nvalid <= 32 ? 0u : (1u << (nvalid - 32)) - 1u;
+            }
+            const int cmine = __popc(m0) + __popc(m1);
+            int out_at = cnt;   // pass B: this row's first output slot for this block
+            if (!kCount) {
+                // the row's other warp holds the tile's other block: swap counts so
+                // that block 2t's survivors precede block 2t + 1's
+                pair[((t & 1) * 2 + g) * kRowsPerCta + r] = cmine;
+                named_bar_sync(2 + sub, 64);
+                const int cother = pair[((t & 1) * 2 + (g ^ 1)) * kRowsPerCta + r];
+                if (g == 1) out_at += cother;
+                cnt += cmine + cother;
+            }
+            // Set bits, 32 values of a row at a time.  With few bits per row each
+            // row's thread walks its own, taking the value of bit e out of the
+            // registers through a select tree on e.  With more, the whole warp
+            // takes them 32 at a time: each row with bits stages its values and
+            // lists (lane, bit) entries at its exclusive offset, then every lane
+            // handles one entry per round.
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t *vh = v + 32 * hf;
+                const uint32_t m = hf ? m1 : m0;
+                const int c = __popc(m);
+                const int cmax = __reduce_max_sync(0xffffffffu, c);
+                if (cmax == 0) continue;
+                if (cmax <= kLaneMax) {
+                    for (uint32_t mm = m; mm != 0u; mm &= mm - 1u) {
+                        const int e = __ffs(mm) - 1;
+                        const uint32_t x = select32(vh, e);
+                        if (kCount) {
+                            const float y = fminf(__fmaf_rz(__uint_as_float(x), inv_w, cw), ytop);
+                            red_shared_add1(hrow + 4u * (uint32_t)__float_as_int(y));
+                        } else {
+                            if (out_at + (int)__popc(m & ((1u << e) - 1u)) < a.cap)
+                                out[out_at + __popc(m & ((1u << e) - 1u))] =
+                                    ((unsigned long long)ord_key(__uint_as_float(x)) << 32) |
+                                    (uint32_t)(tok0 + 32 * hf + e);
+                        }
+                    }
+                } else {
+                    int incl = c;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += y;
+                    }
+                    const int total = __shfl_sync(0xffffffffu, incl, 31);
+                    if (m != 0u) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            stage[lane * kStagePitch + e] =
+                                kCount ? 4u * (uint32_t)__float_as_int(
+                                                  fminf(__fmaf_rz(__uint_as_float(vh[e]), inv_w, cw), ytop))
+                                       : vh[e];
+                        int j = incl - c;
+                        base[lane] = out_at - j;   // output slot = base + list index
+                        for (uint32_t mm = m; mm != 0u; mm &= mm - 1u)
+                            list[j++] = (uint16_t)((lane << 5) | (__ffs(mm) - 1));
+                    }
+                    __syncwarp();
+                    for (int i0l = 0; i0l < total; i0l += 32) {
+                        const int idx = i0l + lane;
+                        if (idx < total) {
+                            const uint32_t ent = list[idx];
+                            const int e = (int)(ent & 31u), o = (int)(ent >> 5);
+                            const int rr = sub * 32 + o;
+                            const uint32_t x = stage[o * kStagePitch + e];
+                            if (kCount) {
+                                red_shared_add1(hbase0 + 4u * (uint32_t)(kHistPitch * rr) + x);
+                            } else {
+                                const int pos = base[o] + idx;
+                                if (pos < a.cap) {
+                                    const int64_t row_o = (int64_t)bh * a.nQB + min(i0 + rr, a.nQB - 1);
+                                    a.buf[row_o * a.cap + pos] =
+                                        ((unsigned long long)ord_key(__uint_as_float(x)) << 32) |
+                                        (uint32_t)(tok0 + 32 * hf + e);
+                                }
+                            }
+                        }
+                    }
+                    __syncwarp();
+                }
+                out_at += c;
+            }
+            word = word_next;
+            if (kCount && (t < 32 || (t & 7) == 7)) raise_floor();   // every tile while it climbs
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[sb]);
         }
-        if (live) a.cnt[row] = cnt;
+        named_bar_sync(1, 256);   // every count of the CTA is in
+        if (g == 0 && live) {
+            if (kCount) {
+                // highest bucket with at least E candidates at or above it
+                uint32_t acc = 0;
+                int keep_from = -1;
+                for (int k = kBuckets - 1; k >= 0; --k) {
+                    acc += hist[r * kHistPitch + k];
+                    if (acc >= (uint32_t)a.E) {
+                        keep_from = k;
+                        break;
+                    }
+                }
+                a.bucket[row] = keep_from;
+            } else {
+                a.cnt[row] = cnt;
+            }
+        }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
@@ -549,6 +771,19 @@ bool make_k_map(CUtensorMap *m, const void *base, const Dims &D, int64_t sb, int
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int D>
+cudaError_t launch_filter(dim3 grid, const CUtensorMap &tm, const ExArgs &a, cudaStream_t st)
+{
+    const int bytes = (int)FLay<D>::bytes;
+    cudaError_t e = cudaFuncSetAttribute(filter_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(filter_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    filter_kernel<D, true><<<grid, 320, bytes, st>>>(tm, a);
+    filter_kernel<D, false><<<grid, 320, bytes, st>>>(tm, a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 int64_t extra_buffer_capacity() { return 1024; }
@@ -578,6 +813,8 @@ cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, 
     a.dense_begin = p.dense_row_begin;
     a.dense_end = p.dense_row_end;
     a.theta = reinterpret_cast<float *>(ws + L.ex_theta);
+    a.smax = reinterpret_cast<float *>(ws + L.ex_smax);
+    a.bucket = reinterpret_cast<int32_t *>(ws + L.ex_bucket);
     a.buf = reinterpret_cast<unsigned long long *>(ws + L.ex_buf);
     a.cnt = reinterpret_cast<int32_t *>(ws + L.ex_cnt);
     a.ovf = reinterpret_cast<int32_t *>(ws + L.ex_ovf);
@@ -597,14 +834,11 @@ cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, 
     }
     dim3 grid((unsigned)ceil_div(D.nQB, kRowsPerCta), (unsigned)(D.B * D.H));
     if (D.d == 64) {
-        e = cudaFuncSetAttribute(filter_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FLay<64>::bytes);
-        if (e != cudaSuccess) return e;
-        filter_kernel<64><<<grid, 192, FLay<64>::bytes, st>>>(tm, a);
+        e = launch_filter<64>(grid, tm, a, st);
     } else {
-        e = cudaFuncSetAttribute(filter_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FLay<128>::bytes);
-        if (e != cudaSuccess) return e;
-        filter_kernel<128><<<grid, 192, FLay<128>::bytes, st>>>(tm, a);
+        e = launch_filter<128>(grid, tm, a, st);
     }
+    if (e != cudaSuccess) return e;
     finalize_kernel<<<g8, 256, 0, st>>>(a);
     fallback_kernel<<<148, 256, 0, st>>>(a);
     return cudaGetLastError();
