@@ -49,19 +49,25 @@ def _peaks():
 
 
 def attn_traffic(w):
-    """DRAM bytes per fine-pass launch from the committed ncu capture, or None
-    when the kernel source changed since the capture or the workload differs."""
+    """DRAM bytes per fine-pass launch from the committed ncu capture of this
+    workload (a few heads, scaled to all heads), or None when the kernel source
+    changed since the capture or no capture covers the workload."""
     import hashlib
     try:
-        rec = json.load(open(os.path.join(ROOT, "profiles", "attn_traffic.json")))
-        src = open(os.path.join(ROOT, rec["source"]), "rb").read()
-    except (OSError, ValueError, KeyError):
+        recs = json.load(open(os.path.join(ROOT, "profiles", "attn_traffic.json")))
+    except (OSError, ValueError):
         return None
-    if hashlib.sha256(src).hexdigest() != rec.get("source_sha256"):
-        return None
-    if w.name != "long" or w.H != 40:
-        return None
-    return float(rec["dram_bytes_per_launch"])
+    for rec in recs.get("captures", []):
+        if rec.get("workload") != w.name or int(rec.get("heads_full", -1)) != w.H:
+            continue
+        try:
+            src = open(os.path.join(ROOT, rec["source"]), "rb").read()
+        except (OSError, KeyError):
+            return None
+        if hashlib.sha256(src).hexdigest() != rec.get("source_sha256"):
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    return None
 
 
 def dense_equiv_flops(w) -> float:
@@ -398,7 +404,7 @@ def main():
     dense_split = w.dense_rows[1] > w.dense_rows[0] and w.N > 256 * 64
     launches_per_step = (1 + 4 + 1 + (1 if dense_split else 0) + (2 if w.centroid else 0)
                          + (3 if w.dtype == "f32" else 0)
-                         + (5 if w.extra_tokens > 0 else 0))   # theta, filter, finalize, fallback, modcent
+                         + (6 if w.extra_tokens > 0 else 0))   # theta, filter x2, finalize, fallback, modcent
     line = {
         "metric": METRIC,
         "value": world * dense_equiv_flops(w) / (ms_step * 1e-3) / 1e12,

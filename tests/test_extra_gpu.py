@@ -89,3 +89,44 @@ def test_extra_tokens_full_size_sampled():
     exempt = _check_rows(w, res, kc, buf.extra_idx.cpu().numpy(), buf.extra_count.cpu().numpy(), rows)
     print(f"sol_sinks: {len(rows)} sampled rows, exempted tokens {exempt}")
     assert exempt <= len(rows) * 2
+
+
+def test_extra_tokens_all_scores_tied():
+    """Every key token identical: every candidate ties, the survivors of the
+    bucketed filter overflow the per-row buffer, and the per-row fallback must
+    return the E lowest candidate indices (ties to the lower index)."""
+    w = Workload("extra_tied", B=1, H=2, N=4200, d=128, dtype="bf16", method="sol", q_block=64,
+                 k_block=64, tau=1.3, extra_tokens=64, grid=(3, 20, 70), seed=53)
+    qc, kc, vc = make_qkv(w, "cpu")
+    kc = kc[:, :1].expand_as(kc).contiguous()
+    p, buf = _gpu_select(w, qc.cuda(), kc.cuda(), vc.cuda())
+    res = oracle.routing(w, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc), with_extra=False)
+    ex, ec, _ = oracle.extra_tokens(res.qbar, oracle.as_raw(kc), res.keep, w.q_block, w.k_block,
+                                    w.extra_tokens, list(range(w.rows)))
+    gi, gc = buf.extra_idx.cpu().numpy(), buf.extra_count.cpu().numpy()
+    keep = res.keep.reshape(w.rows, w.nKB)
+    for r in range(w.rows):
+        cand = [t for t in range(w.N) if not keep[r, t // w.k_block]]
+        assert gc[r] == ec[r] == min(w.extra_tokens, len(cand)), r
+        assert gi[r, :gc[r]].tolist() == cand[:gc[r]] == ex[r, :ec[r]].tolist(), r
+
+
+def test_extra_tokens_fewer_candidates_than_E():
+    """A low tau keeps most blocks, leaving some rows fewer unselected tokens
+    than E: those rows take every candidate, in ascending order."""
+    w = Workload("extra_short", B=1, H=2, N=1000, d=128, dtype="bf16", method="sol", q_block=64,
+                 k_block=64, tau=-0.8, extra_tokens=256, grid=(2, 10, 50), seed=54)
+    qc, kc, vc = make_qkv(w, "cpu")
+    p, buf = _gpu_select(w, qc.cuda(), kc.cuda(), vc.cuda())
+    res = oracle.routing(w, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc), with_extra=False)
+    keep = res.keep.reshape(w.rows, w.nKB)
+    gi, gc = buf.extra_idx.cpu().numpy(), buf.extra_count.cpu().numpy()
+    short = 0
+    for r in range(w.rows):
+        cand = [t for t in range(w.N) if not keep[r, t // w.k_block]]
+        if len(cand) <= w.extra_tokens:
+            short += 1
+            assert gc[r] == len(cand) and gi[r, :gc[r]].tolist() == cand, r
+    assert short > 0, "no row with fewer candidates than E: the case is not exercised"
+    exempt = _check_rows(w, res, kc, gi, gc, list(range(w.rows)))
+    assert exempt <= w.rows * w.extra_tokens // 1000 + 2, exempt
