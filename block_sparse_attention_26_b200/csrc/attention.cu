@@ -71,7 +71,10 @@ constexpr int kMaxE = 256;     // extra tokens per query block (the node's range
 #ifdef BSA_TRACE
 // Per-tile clock64() stamps of a few CTAs (development builds only), kept in
 // shared memory while the CTA runs and copied out at its end.
-constexpr int kTraceCtas = 8, kTraceTiles = 64, kTraceEvents = 16;
+#ifndef BSA_TRACE_TILES
+#define BSA_TRACE_TILES 64
+#endif
+constexpr int kTraceCtas = 8, kTraceTiles = BSA_TRACE_TILES, kTraceEvents = 16;
 constexpr int kTraceBytes = kTraceTiles * kTraceEvents * 8;
 #define TRACE(ev, j)                                                                       \
     do {                                                                                   \
@@ -125,6 +128,12 @@ struct AttnArgs {
     const float *xbias;                        // [rows, Ecap] log2 of their token counts
     const int32_t *xcnt;                       // [rows] modified centroids per row
     const uint32_t *xaff;                      // [rows, nW] blocks that gave extra tokens
+    // gathers by TMA (tile::gather4) when K and V are one uniform 2-D array of token
+    // rows: row of (b, n, h) = b grow_b + n grow_n + h grow_h; else by cp.async
+    int gather_tma;
+    int64_t grow_b, grow_n, grow_h;
+    const uint32_t *glist;                     // [sparse tiles, kGlistCap] extra-token union per tile
+    const int32_t *glcnt;                      // [sparse tiles] its length (a multiple of 4)
 };
 
 template <int D>
@@ -144,10 +153,13 @@ struct Lay {
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
     static constexpr int kOffML = kOffMisc + 16;                 // [2][128] (m, l) per half
     static constexpr int kOffBias = kOffML + 2 * kM * 8;         // [VS][128] per-column bias (gathers)
-    static constexpr int kOffCodes = kOffBias + kVS * kTK * 4;   // [2 producers][128] gathered rows
-    static constexpr int kOffSBias = kOffCodes + 2 * kTK * 4;    // [128] staged bias of the next gather
-    static constexpr int kOffExt = kOffSBias + kTK * 4;          // [2][kMaxE] extra tokens + [4] counts
-    static constexpr int kOffTrace = kOffExt + 2 * kMaxE * 4 + 16;
+    // gathered columns of the CTA: the union of its query blocks' extra tokens, then
+    // each query block's modified centroids (code, query-block bits, bias source)
+    static constexpr int kOffGlCode = kOffBias + kVS * kTK * 4;   // [4 kMaxE] u32
+    static constexpr int kOffGlBias = kOffGlCode + 4 * kMaxE * 4; // [2][kMaxE] modified-centroid biases
+    static constexpr int kOffGlWho = kOffGlBias + 2 * kMaxE * 4;  // [4 kMaxE] u8
+    static constexpr int kOffExt = kOffGlWho + 4 * kMaxE;         // [8] list lengths
+    static constexpr int kOffTrace = kOffExt + 32;
     static constexpr int kOffMask = kOffTrace + kTraceBytes;     // kept [2][nW], then affected [2][nW]
     // at least 116 KB so that a single CTA owns an SM (it allocates all 512 TMEM columns)
     static size_t bytes(int nW)
@@ -197,7 +209,9 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
-                const __grid_constant__ CUtensorMap tm_vc, const AttnArgs a)
+                const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_gk,
+                const __grid_constant__ CUtensorMap tm_gv, const __grid_constant__ CUtensorMap tm_gxk,
+                const __grid_constant__ CUtensorMap tm_gxv, const AttnArgs a)
 {
     using L = Lay<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -210,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t nd_items = (int64_t)a.B * a.H * a.n_dense * a.dense_split;
     const bool dense = item < nd_items;
     int bh, row0, nvalid, kb0 = 0, kb1 = 0;
-    int64_t pidx = 0;
+    int64_t pidx = 0, sidx = 0;   // dense partial index; sparse tile index (b, h, tile)
     if (dense) {
         const int split = (int)(item % a.dense_split);
         const int64_t tt = item / a.dense_split;          // (bh, tile)
@@ -223,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         pidx = tt * a.dense_split + split;
     } else {
         item -= nd_items;
+        sidx = item;
         const int tile = (int)(item % a.n_sparse);
         bh = (int)(item / a.n_sparse);
         row0 = tile * kM;
@@ -249,8 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *kept = reinterpret_cast<uint32_t *>(sm + L::kOffMask);
     uint32_t *aff = kept + 2 * a.nW;                            // blocks that gave extra tokens
     float *bias_sm = reinterpret_cast<float *>(sm + L::kOffBias);
-    int32_t *ext = reinterpret_cast<int32_t *>(sm + L::kOffExt); // [2][kMaxE]
-    int32_t *ext_n = ext + 2 * kMaxE;                            // [2] extra tokens, [2..3] modified centroids
+    // [0..1] extra tokens, [2..3] modified centroids per query block; [4] union size
+    // (padded), [5] gathered columns in all
+    int32_t *ext_n = reinterpret_cast<int32_t *>(sm + L::kOffExt);
+    uint32_t *gl_code = reinterpret_cast<uint32_t *>(sm + L::kOffGlCode);
+    float *gl_bias = reinterpret_cast<float *>(sm + L::kOffGlBias);
+    uint8_t *gl_who = sm + L::kOffGlWho;
 #ifdef BSA_TRACE
     long long *trace_sm = reinterpret_cast<long long *>(sm + L::kOffTrace);
     for (int i = threadIdx.x; i < kTraceTiles * kTraceEvents; i += blockDim.x) trace_sm[i] = 0;
@@ -284,18 +303,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         // kept-block bitmasks of the tile's query blocks, from the CSR lists; with
         // extra tokens also their lists and the blocks they came from
         for (int w = lane; w < 4 * a.nW; w += 32) kept[w] = 0u;
-        if (lane < 4) ext_n[lane] = 0;
+        if (lane < 8) ext_n[lane] = 0;
         __syncwarp();
         if (a.E > 0) {
+            // gathered columns: the union of the query blocks' extra tokens (merged
+            // by glist_kernel, padded to a multiple of 4), then each query block's
+            // modified centroids
             for (int q = 0; q < nq; ++q) {
                 const int64_t rq = rbase + q;
-                const int n = min(a.extra_count[rq], a.E);
-                for (int e = lane; e < n; e += 32) ext[q * kMaxE + e] = a.extra_idx[rq * a.E + e];
+                const int nx = min(a.xcnt[rq], a.Ecap);
+                for (int e = lane; e < nx; e += 32) gl_bias[q * kMaxE + e] = a.xbias[rq * a.Ecap + e];
                 for (int w = lane; w < a.nW; w += 32) aff[q * a.nW + w] = a.xaff[rq * a.nW + w];
                 if (lane == 0) {
-                    ext_n[q] = n;
-                    ext_n[2 + q] = a.xcnt[rq];
+                    ext_n[q] = min(a.extra_count[rq], a.E);
+                    ext_n[2 + q] = nx;
                 }
+            }
+            __syncwarp();
+            const int64_t gi = sidx;
+            const int U = a.glcnt[gi], m0 = ext_n[2], m1 = ext_n[3];
+            for (int i = lane; i < U; i += 32) {
+                const uint32_t v = a.glist[gi * kGlistCap + i];
+                gl_code[i] = v & 0x3fffffffu;
+                gl_who[i] = (uint8_t)(v >> 30);
+            }
+            for (int e = lane; e < m0; e += 32) {
+                gl_code[U + e] = 0x80000000u | (uint32_t)e;
+                gl_who[U + e] = 1;
+            }
+            for (int e = lane; e < m1; e += 32) {
+                gl_code[U + m0 + e] = 0xC0000000u | (uint32_t)e;
+                gl_who[U + m0 + e] = 2;
+            }
+            if (lane == 0) {
+                ext_n[4] = U;
+                ext_n[5] = U + m0 + m1;
             }
         }
         for (int q = 0; q < nq; ++q) {
@@ -335,12 +377,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const CUtensorMap *tm_x = is_k ? &tm_k : &tm_v;
         const CUtensorMap *tm_c = is_k ? &tm_kc : &tm_vc;
+        const CUtensorMap *tm_gx = is_k ? &tm_gk : &tm_gv;     // token rows, for gathers
+        const CUtensorMap *tm_gc = is_k ? &tm_gxk : &tm_gxv;   // modified-centroid rows
         const int depth = is_k ? kKS : kVS;
         uint64_t *full = is_k ? k_full : v_full;
         uint64_t *empty = is_k ? k_empty : v_empty;
         uint8_t *ring = sm + (is_k ? L::kOffK : L::kOffV);
-        uint32_t *codes = reinterpret_cast<uint32_t *>(sm + L::kOffCodes) + (is_k ? 0 : kTK);
-        float *stage_bias = reinterpret_cast<float *>(sm + L::kOffSBias);
+        int gl0 = 0, gln = 0, glU = 0, glm0 = 0;   // the gathered tile: list entries [gl0, gl0 + gln)
         const __nv_bfloat16 *src_x = is_k ? a.kx : a.vx;
         const __nv_bfloat16 *src_c = is_k ? a.xk16 : a.xv16;
         int j = 0;
@@ -391,21 +434,61 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             uint8_t *dst = ring + s * L::kTileBytes;
             if (kind == TILE_GATHER && !is_k)
-                for (int c = lane; c < kTK; c += 32) bias_sm[s * kTK + c] = stage_bias[c];
-            if (kind == TILE_GATHER) {
-                // 128 rows from arbitrary addresses, written in the 128-byte-swizzled
-                // layout the tensor core reads; completion through the barrier
-                const uint32_t base = smem_u32(dst);
-                for (int t = lane; t < kTK * (D / 8); t += 32) {
-                    const int c = t / (D / 8), k16 = t % (D / 8);
-                    const int dc = k16 >> 3, c16 = k16 & 7;
-                    const uint32_t sa = base + dc * (kTK * 128) + (c >> 3) * 1024 + (c & 7) * 128 +
-                                        ((c16 ^ (c & 7)) << 4);
-                    const __nv_bfloat16 *ga = row_src(codes[c]) + k16 * 8;
-                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(ga) : "memory");
+                for (int c = lane; c < kTK; c += 32) {
+                    // bias 0 for extra tokens, log2 of the remaining count for modified centroids
+                    const int g = gl0 + c;
+                    float bs = 0.f;
+                    if (c < gln && g >= glU) bs = g < glU + glm0 ? gl_bias[g - glU] : gl_bias[kMaxE + g - glU - glm0];
+                    bias_sm[s * kTK + c] = bs;
                 }
-                asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-                fence_async_smem();
+            if (kind == TILE_GATHER && a.gather_tma) {
+                // 128 rows by TMA, 4 rows per gather: lane l takes columns 4l..4l+3
+                // (unused columns repeat the last entry; the 4 rows of a gather come
+                // from one array because the column list is 4-aligned per array)
+                if (lane == 0) mbar_expect_tx(&full[s], L::kTileBytes);
+                __syncwarp();
+                const int c = 4 * lane;
+                int rw[4];
+                bool cent = false;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t code = gl_code[c + i < gln ? gl0 + c + i : gl0 + gln - 1];
+                    if (i == 0) cent = (code & 0x80000000u) != 0u;
+                    rw[i] = cent ? (int)((rbase + ((code >> 30) & 1u)) * a.Ecap + (code & 0x3fffffffu))
+                                 : (int)(b * a.grow_b + h * a.grow_h + (int64_t)code * a.grow_n);
+                }
+#pragma unroll
+                for (int dc = 0; dc < D / 64; ++dc)
+                    tma_gather4(dst + dc * (kTK * 128) + c * 128, cent ? tm_gc : tm_gx, &full[s], dc * 64, rw);
+            } else if (kind == TILE_GATHER) {
+                // 128 rows from arbitrary addresses, written in the 128-byte-swizzled
+                // layout the tensor core reads; completion through the barrier.  Unused
+                // columns repeat the first row (a valid address; no column active).
+                // lane l copies 16-byte chunk l % (D/8) of rows l / (D/8) + (32/(D/8)) i: the
+                // row codes and addresses of a batch are formed before its copies issue
+                const uint32_t base = smem_u32(dst);
+                constexpr int kCh = D / 8, kRowsPerPass = 32 / kCh, kBatch = 16;
+                const int k16 = lane % kCh, dc = k16 >> 3, c16 = k16 & 7;
+                const uint32_t sbase = base + dc * (kTK * 128);
+#pragma unroll 1
+                for (int c0 = lane / kCh; c0 < kTK; c0 += kRowsPerPass * kBatch) {
+                    const __nv_bfloat16 *ga[kBatch];
+#pragma unroll
+                    for (int i = 0; i < kBatch; ++i) {
+                        const int c = c0 + kRowsPerPass * i;
+                        ga[i] = row_src(gl_code[c < gln ? gl0 + c : gl0]) + k16 * 8;
+                    }
+#pragma unroll
+                    for (int i = 0; i < kBatch; ++i) {
+                        const int c = c0 + kRowsPerPass * i;
+                        const uint32_t sa = sbase + (c >> 3) * 1024 + (c & 7) * 128 + ((c16 ^ (c & 7)) << 4);
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(ga[i]));
+                    }
+                }
+                // each lane's copies complete the slot asynchronously (one pending
+                // arrival per lane, added now); lane 0 gives the barrier's own arrival.
+                // The MMA warp orders them before its tensor-core reads with a proxy fence.
+                asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[s])) : "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[s]);
             } else if (lane == 0) {
@@ -423,6 +506,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t zero2[2][2] = {{0, 0}, {0, 0}};
         const int none[2] = {-1, -1};
         bool ok = true;
+        // Gathered tiles (128 entries of the CTA's column list each) are spread
+        // evenly among the exact tiles, so that each has the tiles before it to
+        // arrive from DRAM.
+        int gat_est = 0, gdone = 0, G = -1, n_exact = 0, exact_pushed = 0;
+        if (!dense && a.E > 0) {
+            gat_est = (ext_n[5] + kTK - 1) / kTK;
+            int nb = 0;
+            for (int w = lane; w < a.nW; w += 32) nb += __popc(kept[w] | kept[a.nW + w]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) nb += __shfl_xor_sync(0xffffffffu, nb, o);
+            n_exact = (nb + 1) / 2;
+        }
+        auto push_gather = [&]() -> bool {
+            if (G < 0) {
+                G = ext_n[5];
+                glU = ext_n[4];
+                glm0 = ext_n[2];
+            }
+            const int g0 = gdone * kTK;
+            if (g0 >= G) {   // fewer than the bound
+                gdone = gat_est;
+                return true;
+            }
+            gl0 = g0;
+            gln = min(kTK, G - g0);
+            uint64_t cm[2][2];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int c = 32 * k + lane;
+                const uint32_t who = c < gln ? gl_who[g0 + c] : 0u;
+                const uint64_t w1 = __ballot_sync(0xffffffffu, who & 1u), w2 = __ballot_sync(0xffffffffu, who & 2u);
+                if (k & 1) {
+                    cm[0][k >> 1] |= w1 << 32;
+                    cm[1][k >> 1] |= w2 << 32;
+                } else {
+                    cm[0][k >> 1] = w1;
+                    cm[1][k >> 1] = w2;
+                }
+            }
+            const int none2[2] = {-1, -1};
+            const int nc0[2] = {0, 0};
+            const uint32_t wh0[2] = {0u, 0u};
+            ++gdone;
+            return push(TILE_GATHER, none2, wh0, nc0, none2, 0.f, cm);
+        };
+        auto after_exact = [&]() {
+            ++exact_pushed;
+            while (ok && gdone < gat_est && exact_pushed >= ((gdone + 1) * n_exact) / (gat_est + 1))
+                ok = push_gather();
+        };
         // exact tiles: pairs of key blocks; an odd last tile repeats its block
         // in the empty half (a valid load) with no active column
         int pend = -1;
@@ -438,6 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nc[2] = {min(kBK, a.N - pend * kBK), min(kBK, a.N - blk * kBK)};
             ok = push(TILE_EXACT, bl, wh, nc, none, 0.f, zero2);
             pend = -1;
+            if (ok) after_exact();
         };
         if (dense) {
             for (int blk = kb0; blk < kb1 && ok; ++blk) emit_block(blk, 3u);
@@ -458,62 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nc[2] = {min(kBK, a.N - pend * kBK), 0};
             ok = push(TILE_EXACT, bl, wh, nc, none, 0.f, zero2);
             pend = -1;
+            if (ok) after_exact();
         }
-        if (!dense && a.E > 0 && ok) {
-            // gathered tiles: the union of the two query blocks' extra tokens (in
-            // token order), then each query block's modified centroids
-            const int n0 = ext_n[0], n1 = ext_n[1], m0 = ext_n[2], m1 = ext_n[3];
-            int i0 = 0, i1 = 0, e0 = 0, e1 = 0;
-            const int none2[2] = {-1, -1};
-            const int nc0[2] = {0, 0};
-            const uint32_t wh0[2] = {0u, 0u};
-            while (ok && (i0 < n0 || i1 < n1 || e0 < m0 || e1 < m1)) {
-                uint64_t cm[2][2] = {{0, 0}, {0, 0}};
-                int c = 0;
-                if (lane == 0) {
-                    float *bias = stage_bias;
-                    for (; c < kTK && (i0 < n0 || i1 < n1 || e0 < m0 || e1 < m1); ++c) {
-                        uint32_t code, who;
-                        float bs = 0.f;
-                        if (i0 < n0 || i1 < n1) {
-                            const int t0 = i0 < n0 ? ext[i0] : INT_MAX, t1 = i1 < n1 ? ext[kMaxE + i1] : INT_MAX;
-                            const int t = min(t0, t1);
-                            who = (t0 == t ? 1u : 0u) | (t1 == t ? 2u : 0u);
-                            i0 += t0 == t;
-                            i1 += t1 == t;
-                            code = (uint32_t)t;
-                        } else if (e0 < m0) {
-                            code = 0x80000000u | (uint32_t)e0;
-                            bs = a.xbias[rbase * a.Ecap + e0];
-                            who = 1u;
-                            ++e0;
-                        } else {
-                            code = 0xC0000000u | (uint32_t)e1;
-                            bs = a.xbias[(rbase + 1) * a.Ecap + e1];
-                            who = 2u;
-                            ++e1;
-                        }
-                        codes[c] = code;
-                        if (!is_k) bias[c] = bs;
-                        if (who & 1u) cm[0][c >> 6] |= 1ull << (c & 63);
-                        if (who & 2u) cm[1][c >> 6] |= 1ull << (c & 63);
-                    }
-                    for (int p = c; p < kTK; ++p) {
-                        codes[p] = codes[0];            // a valid row; no column active
-                        if (!is_k) bias[p] = 0.f;
-                    }
-                }
-                // the list state lives in lane 0: broadcast it
-                i0 = __shfl_sync(0xffffffffu, i0, 0);
-                i1 = __shfl_sync(0xffffffffu, i1, 0);
-                e0 = __shfl_sync(0xffffffffu, e0, 0);
-                e1 = __shfl_sync(0xffffffffu, e1, 0);
-                for (int x = 0; x < 2; ++x)
-                    for (int y = 0; y < 2; ++y) cm[x][y] = __shfl_sync(0xffffffffu, cm[x][y], 0);
-                __syncwarp();
-                ok = push(TILE_GATHER, none2, wh0, nc0, none2, 0.f, cm);
-            }
-        }
+        while (ok && gdone < gat_est) ok = push_gather();   // the rest (none if no exact tile)
         if (!dense && a.centroid && ok) {
             const int last_n = a.N - (a.nKB - 1) * kBK;
             const int nchunk = (a.nKB + kBK - 1) / kBK;
@@ -560,6 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (is_k) mbar_wait(bar_q, 0, &no_abort, a.status, 14);
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");   // this lane's gathered rows have landed
     } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
@@ -581,6 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int ks = ns % kKS;
                     if (mbar_test(&k_full[ks], (ns / kKS) & 1) && (ns < 1 || mbar_test(s_free, (ns - 1) & 1))) {
                         tc_fence_after();
+                        if (kkind[ks] == TILE_GATHER && !a.gather_tma) fence_async_smem();   // rows by cp.async
                         if (kkind[ks] == TILE_END) {
                             T = ns;
                         } else {
@@ -607,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int pb = t & 1, vs = t % kVS;
                     if (mbar_test(&p_full[2 * hf + pb], (t >> 1) & 1) && mbar_test(&v_full[vs], (t / kVS) & 1)) {
                         tc_fence_after();
+                        if (info[vs].kind == TILE_GATHER && !a.gather_tma) fence_async_smem();   // rows by cp.async
 #pragma unroll
                         for (int ks = 0; ks < kBK / 16; ++ks) {
                             const uint64_t bd = sdesc_sw128(
@@ -1017,6 +1101,88 @@ __global__ void __launch_bounds__(256) modcent_kernel(const int32_t *__restrict_
     if (lane == 0) xcnt[r] = nent;
 }
 
+// Per sparse tile of the fine pass (query blocks qb0 and qb0 + 1 for 64-row
+// blocks, one 128-row block otherwise): the union of its query blocks' ascending
+// extra-token lists, an entry being the token with bit 30 set if the first query
+// block chose it and bit 31 if the second did; padded to a multiple of 4 with
+// repeats of its last token (no bit set) so that a gather of 4 rows never mixes
+// tokens with modified centroids.  One warp per tile.  Union rank of a token of
+// one list = its index + the other list's tokens below it - those of them that
+// both lists hold.
+__global__ void __launch_bounds__(128) glist_kernel(const int32_t *__restrict__ extra_idx,
+                                                    const int32_t *__restrict__ extra_count, int E, int nQB, int Bq,
+                                                    int n_sparse, int64_t ntiles, uint32_t *__restrict__ glist,
+                                                    int32_t *__restrict__ glcnt)
+{
+    __shared__ int32_t sA[4][kMaxE], sB[4][kMaxE], lbA[4][kMaxE], lbB[4][kMaxE], PA[4][kMaxE + 1],
+        PB[4][kMaxE + 1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 4 + warp;
+    if (t >= ntiles) return;
+    const int64_t bh = t / n_sparse;
+    const int qb0 = (int)((t % n_sparse) * kM / Bq);
+    const int nq = (Bq == 64 && qb0 + 1 < nQB) ? 2 : 1;
+    const int64_t r0 = bh * nQB + qb0;
+    const int n0 = min(extra_count[r0], E), n1 = nq > 1 ? min(extra_count[r0 + 1], E) : 0;
+    int32_t *A = sA[warp], *B = sB[warp];
+    for (int i = lane; i < n0; i += 32) A[i] = extra_idx[r0 * E + i];
+    for (int i = lane; i < n1; i += 32) B[i] = extra_idx[(r0 + 1) * E + i];
+    __syncwarp();
+    auto lower_bound = [](const int32_t *X, int n, int key) {
+        int lo = 0, hi = n;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (X[mid] < key)
+                lo = mid + 1;
+            else
+                hi = mid;
+        }
+        return lo;
+    };
+    for (int i = lane; i < n0; i += 32) {
+        const int lb = lower_bound(B, n1, A[i]);
+        lbA[warp][i] = lb | ((lb < n1 && B[lb] == A[i]) ? 0x40000000 : 0);
+    }
+    for (int i = lane; i < n1; i += 32) {
+        const int lb = lower_bound(A, n0, B[i]);
+        lbB[warp][i] = lb | ((lb < n0 && A[lb] == B[i]) ? 0x40000000 : 0);
+    }
+    __syncwarp();
+    // P[k] = entries of a list among its first k that the other list holds too
+    auto prefix = [&](const int32_t *lb, int n, int32_t *P) {
+        int carry = 0;
+        for (int k0 = 0; k0 <= n; k0 += 32) {
+            const int k = k0 + lane;
+            int x = (k > 0 && k <= n) ? ((lb[k - 1] >> 30) & 1) : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (k <= n) P[k] = carry + x;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+    };
+    prefix(lbA[warp], n0, PA[warp]);
+    prefix(lbB[warp], n1, PB[warp]);
+    __syncwarp();
+    uint32_t *out = glist + t * kGlistCap;
+    for (int i = lane; i < n0; i += 32) {
+        const int v = lbA[warp][i], lb = v & 0x3fffffff;
+        const bool both = (v >> 30) & 1;
+        out[i + lb - PB[warp][lb]] = (uint32_t)A[i] | (both ? 0xC0000000u : 0x40000000u);
+    }
+    for (int i = lane; i < n1; i += 32) {
+        const int v = lbB[warp][i], lb = v & 0x3fffffff;
+        if ((v >> 30) & 1) continue;   // listed with the first query block
+        out[i + lb - PA[warp][lb]] = (uint32_t)B[i] | 0x80000000u;
+    }
+    const int U0 = n0 + n1 - PA[warp][n0], U = (U0 + 3) & ~3;
+    __syncwarp();
+    if (lane < U - U0) out[U0 + lane] = out[U0 - 1] & 0x3fffffffu;
+    if (lane == 0) glcnt[t] = U;
+}
+
 // bf16 copies of f32 centroids: elementwise, grid-stride.
 __global__ void to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst, int64_t n)
 {
@@ -1091,15 +1257,30 @@ bool make_map_cent(CUtensorMap *m, const void *base, int BH, int nKB, int d)
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 rows of a 2-D array [rows, d] with a row pitch; box = 64 channels x 1 row
+// (the shape tile::gather4 takes).
+bool make_map_rows(CUtensorMap *m, const void *base, int64_t rows, int d, int64_t pitch)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)pitch * 2};
+    cuuint32_t box[2] = {64, 1};
+    cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch_attn_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                               const CUtensorMap &tkc, const CUtensorMap &tvc, const AttnArgs &a, int64_t items,
-                               cudaStream_t st)
+                               const CUtensorMap &tkc, const CUtensorMap &tvc, const CUtensorMap (&tg)[4],
+                               const AttnArgs &a, int64_t items, cudaStream_t st)
 {
     const size_t smem = Lay<D>::bytes(a.nW);
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<D><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, a);
+    attn_kernel<D><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, tg[0], tg[1], tg[2], tg[3], a);
     return cudaGetLastError();
 }
 
@@ -1227,7 +1408,13 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
             a.Ecap, reinterpret_cast<__nv_bfloat16 *>(ws + L.xk16), reinterpret_cast<__nv_bfloat16 *>(ws + L.xv16),
             reinterpret_cast<float *>(ws + L.xbias), reinterpret_cast<int32_t *>(ws + L.xcnt),
             reinterpret_cast<uint32_t *>(ws + L.xaff));
+        const int64_t ntiles = (int64_t)BH * ceil_div(D.N, kM);
+        glist_kernel<<<(unsigned)ceil_div(ntiles, 4), 128, 0, st>>>(
+            extra_idx, extra_count, D.E, D.nQB, D.Bq, (int)ceil_div(D.N, kM), ntiles,
+            reinterpret_cast<uint32_t *>(ws + L.glist), reinterpret_cast<int32_t *>(ws + L.glcnt));
     }
+    a.glist = reinterpret_cast<const uint32_t *>(ws + L.glist);
+    a.glcnt = reinterpret_cast<const int32_t *>(ws + L.glcnt);
     a.n_sparse = dense_only ? 0 : (int)ceil_div(D.N, kM);
     a.skip_begin = row_begin;
     a.skip_end = row_end;
@@ -1241,8 +1428,36 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     a.part_ml = reinterpret_cast<float *>(ws + L.part_ml);
     const int64_t items = (int64_t)BH * (a.n_dense * (int64_t)a.dense_split + a.n_sparse);
     if (items == 0) return cudaSuccess;
-    cudaError_t e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, a, items, st)
-                              : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, a, items, st);
+    // gather maps: token rows of K and V as one 2-D array when the strides allow it
+    // (the row pitch min(sn, sh) divides every stride and holds a whole row), and the
+    // modified centroids [rows x Ecap, d]
+    CUtensorMap tg[4] = {tk, tv, tk, tv};
+    a.gather_tma = 0;
+    a.grow_b = a.grow_n = a.grow_h = 0;
+    if (a.E > 0) {
+        const int64_t rs = std::min(sn, sh);
+        if (rs >= D.d && sb % rs == 0 && sn % rs == 0 && sh % rs == 0) {
+            const int64_t nrows_k = (int64_t)(D.B - 1) * (sb / rs) + (int64_t)(D.N - 1) * (sn / rs) +
+                                    (int64_t)(D.H - 1) * (sh / rs) + 1;
+            const int64_t nrows_x = D.rows * (int64_t)a.Ecap;
+            if (nrows_k < INT32_MAX && nrows_x < INT32_MAX && make_map_rows(&tg[0], k16, nrows_k, D.d, rs) &&
+                make_map_rows(&tg[1], v16, nrows_k, D.d, rs) &&
+                make_map_rows(&tg[2], ws + L.xk16, nrows_x, D.d, D.d) &&
+                make_map_rows(&tg[3], ws + L.xv16, nrows_x, D.d, D.d)) {
+                a.gather_tma = 1;
+                a.grow_b = sb / rs;
+                a.grow_n = sn / rs;
+                a.grow_h = sh / rs;
+            } else {
+                tg[0] = tk;
+                tg[1] = tv;
+                tg[2] = tk;
+                tg[3] = tv;
+            }
+        }
+    }
+    cudaError_t e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, tg, a, items, st)
+                              : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, tg, a, items, st);
     if (e != cudaSuccess) return e;
     if (a.n_dense > 0 && a.dense_split > 1) {
         combine_kernel<<<(unsigned)(BH * (int64_t)a.n_dense), kM, 0, st>>>(a, D.d);

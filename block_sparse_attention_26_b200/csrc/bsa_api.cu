@@ -62,6 +62,9 @@ WsLayout ws_layout(const bsa_params &p)
     L.xbias = take((size_t)D.rows * ecap * 4);
     L.xcnt = take(D.E > 0 ? (size_t)D.rows * 4 : 0);
     L.xaff = take(D.E > 0 ? (size_t)D.rows * D.nW * 4 : 0);
+    const size_t ftiles = (size_t)BH * (size_t)((D.N + 127) / 128);
+    L.glist = take(D.E > 0 ? ftiles * kGlistCap * 4 : 0);
+    L.glcnt = take(D.E > 0 ? ftiles * 4 : 0);
     const size_t in16 = p.dtype == BSA_DT_F32 ? (size_t)D.B * D.N * D.H * D.d * 2 : 0;
     L.q16 = take(in16);
     L.k16 = take(in16);

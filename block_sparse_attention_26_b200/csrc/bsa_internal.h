@@ -10,6 +10,10 @@
 namespace bsa {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// entries per fine-pass tile of the extra-token union: two lists of at most 256,
+// padded to a multiple of 4
+constexpr int kGlistCap = 2 * 256 + 4;
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Derived sizes of one problem.
@@ -34,6 +38,8 @@ struct WsLayout {
     size_t xbias;          // [rows, min(E, nKB)] f32 their log2 token counts
     size_t xcnt;           // [rows] i32 modified centroids per row
     size_t xaff;           // [rows, nW] u32 blocks that gave extra tokens
+    size_t glist;          // [sparse tiles, kGlistCap] u32 extra-token union per fine-pass tile
+    size_t glcnt;          // [sparse tiles] i32 its length
     size_t q16, k16, v16;  // [B, N, H, d] bf16 copies of f32 inputs (attention, f32 only)
     size_t ex_theta;       // [rows] f32 extra-token score bounds
     size_t ex_smax;        // [rows] f32 largest sampled token score
