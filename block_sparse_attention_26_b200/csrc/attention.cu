@@ -39,10 +39,13 @@
 //              soon as its S product is done, the V producer also publishes each
 //              tile's masks to the softmax warps.
 //   warp 9     MMA issuer (one thread, event loop): S = Q K^T (A and B from
-//              shared memory) runs ahead of the softmax; O_h += P_h V_h (A = P_h
-//              from TMEM) is issued as soon as half h of a tile's P is in.
-// TMEM (512 columns): S [0,128); P of half h, buffer b at 128 + 64 h + 32 b;
-// O_h at 256 + 128 h.
+//              shared memory) runs up to two tiles ahead of the softmax, into two
+//              TMEM buffers; O_h += P_h V_h (A = P_h from TMEM) is issued as soon
+//              as half h of a tile's P is in.  S(j) may overwrite buffer j & 1 once
+//              P(j - 2) there has been issued to both P V products: the tensor pipe
+//              runs one thread's MMAs in issue order.
+// TMEM (512 columns): S of tile j at 128 (j & 1), half h's P (bf16 pairs) written
+// over its own S columns 128 (j & 1) + 64 h once read; O_h at 256 + 128 h.
 #include <math.h>
 
 #include <algorithm>
@@ -61,8 +64,7 @@ constexpr int kVS = 3;         // V ring depth (tiles)
 constexpr int kThreads = 352;  // 2 softmax warpgroups + K producer + MMA + V producer
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;          // S, 128 columns
-constexpr uint32_t kColP = 128;        // P of half h, buffer b at kColP + 64 h + 32 b
+constexpr uint32_t kColS = 0;          // S of tile j at kColS + 128 (j & 1); P of half h over its own S
 constexpr uint32_t kColO = 256;        // O of half h at kColO + 128 h
 
 enum : int32_t { TILE_EXACT = 0, TILE_CENT = 1, TILE_END = 2, TILE_GATHER = 3 };
@@ -147,7 +149,7 @@ struct Lay {
     static constexpr int kOffKind = kOffV + kVS * kTileBytes;
     static constexpr int kOffInfo = kOffKind + 16;
     static constexpr int kOffBar = kOffInfo + kVS * (int)sizeof(TileInfo);
-    // q, done, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full, s_free,
+    // q, done, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2 buffers],
     // p_full[2 halves][2], p_free[2 halves][2]
     static constexpr int kNumBar = 2 + 2 * kKS + 2 * kVS + 2 + 8;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
@@ -253,8 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bar_q = bars, *bar_done = bars + 1;
     uint64_t *k_full = bars + 2, *k_empty = k_full + kKS;
     uint64_t *v_full = k_empty + kKS, *v_empty = v_full + kVS;
-    uint64_t *s_full = v_empty + kVS, *s_free = s_full + 1;
-    uint64_t *p_full = s_free + 1;            // [half * 2 + buffer]
+    uint64_t *s_full = v_empty + kVS;         // [buffer]
+    uint64_t *p_full = s_full + 2;            // [half * 2 + buffer]
     uint64_t *p_free = p_full + 4;            // [half * 2 + buffer]
     volatile int32_t *kkind = reinterpret_cast<volatile int32_t *>(sm + L::kOffKind);
     volatile TileInfo *info = reinterpret_cast<volatile TileInfo *>(sm + L::kOffInfo);
@@ -286,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(s_free, 8);
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
         for (int i = 0; i < 4; ++i) {
             mbar_init(&p_full[i], 4);
             mbar_init(&p_free[i], 1);
@@ -661,7 +663,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool progressed = false;
                 if (T < 0) {
                     const int ks = ns % kKS;
-                    if (mbar_test(&k_full[ks], (ns / kKS) & 1) && (ns < 1 || mbar_test(s_free, (ns - 1) & 1))) {
+                    // S(ns) goes to buffer ns & 1 once P(ns - 2), which sits there, has been
+                    // issued to both halves' P V products (the tensor pipe keeps issue order)
+                    if (mbar_test(&k_full[ks], (ns / kKS) & 1) && (ns < 2 || (np[0] >= ns - 1 && np[1] >= ns - 1))) {
                         tc_fence_after();
                         if (kkind[ks] == TILE_GATHER && !a.gather_tma) fence_async_smem();   // rows by cp.async
                         if (kkind[ks] == TILE_END) {
@@ -673,9 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
                                 const uint64_t bd = sdesc_sw128(
                                     k_addr + ks * L::kTileBytes + (kk >> 2) * (kTK * 128) + (kk & 3) * 32, 16, 1024);
-                                umma_bf16(tmem + kColS, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                                umma_bf16(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                             }
-                            umma_commit(s_full);
+                            umma_commit(&s_full[ns & 1]);
                             umma_commit(&k_empty[ks]);
                             TRACE(2, ns);
                             ++ns;
@@ -695,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int ks = 0; ks < kBK / 16; ++ks) {
                             const uint64_t bd = sdesc_sw128(
                                 v_addr + vs * L::kTileBytes + hf * L::kHalfBytes + ks * 2048, kTK * 128, 1024);
-                            umma_bf16_ts(tmem + kColO + 128 * hf, tmem + kColP + 64 * hf + 32 * pb + 8 * ks, bd,
+                            umma_bf16_ts(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd,
                                          idesc_o, (t > 0 || ks > 0) ? 1u : 0u);
                         }
                         umma_commit(&p_free[2 * hf + pb]);
@@ -716,9 +720,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                 }
             }
-            // end-of-list marker for the softmax warps, once S is free again
-            if (ok && T >= 1) ok = mbar_wait(s_free, (T - 1) & 1, abort_flag, a.status, 27);
-            if (ok) umma_commit(s_full);
+            // end-of-list marker for the softmax warps (both halves have taken every
+            // earlier S, so buffer T & 1 may complete its next phase)
+            if (ok) umma_commit(&s_full[T & 1]);
             umma_commit(bar_done);
             volatile int32_t no_abort = 0;
             mbar_wait(bar_done, 0, &no_abort, a.status, 25);
@@ -739,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int j = 0;
         for (;; ++j) {
             const int vs = j % kVS;
-            ok = mbar_wait(s_full, j & 1, abort_flag, a.status, 30) &&
+            ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, a.status, 30) &&
                  mbar_wait(&v_full[vs], (j / kVS) & 1, abort_flag, a.status, 31);
             if (!(ok = __all_sync(0xffffffffu, ok))) break;
             tc_fence_after();
@@ -747,12 +751,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (kind == TILE_END) break;
             if (r == 0) TRACE(4 + 3 * hf, j);
             float s[64];
-            tmem_ld32(tmem + lane_base + kColS + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-            tmem_ld32(tmem + lane_base + kColS + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+            const uint32_t col_s = kColS + 128 * (j & 1) + 64 * hf;   // this half's S, then its P
+            tmem_ld32(tmem + lane_base + col_s, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+            tmem_ld32(tmem + lane_base + col_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
             tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(s_free);
             if (r == 0) TRACE(5 + 3 * hf, j);
 
             // 0: skip (no active column), 1: all 64 columns active, 2: masked / biased
@@ -834,12 +836,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
             if (r == 0) TRACE(10 + 3 * hf, j);
-            if (j >= 2) {
-                ok = mbar_wait(&pe[j & 1], ((j >> 1) - 1) & 1, abort_flag, a.status, 32);
-                if (!(ok = __all_sync(0xffffffffu, ok))) break;
-            }
             if (r == 0) TRACE(11 + 3 * hf, j);
-            tmem_st32(tmem + lane_base + kColP + 64 * hf + 32 * (j & 1), pk);
+            tmem_st32(tmem + lane_base + col_s, pk);   // over this half's S, already read
             if (__any_sync(0xffffffffu, rescale)) {
                 // the accumulator must hold every earlier P V product before it is scaled
                 ok = mbar_wait(&pe[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status, 33);
