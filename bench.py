@@ -70,6 +70,26 @@ def attn_traffic(w):
     return None
 
 
+def rank_workload(w, rank: int, world: int):
+    """Weak scaling: every rank runs its own layer of the same shape on its own
+    inputs (heads are independent; no collective on the data path)."""
+    return w.replace(seed=w.seed + 17 * rank) if world > 1 else w
+
+
+def max_over_ranks(value: float, pg, device) -> float:
+    """The job's time is the slowest rank's (all_reduce MAX); identity on one rank."""
+    if pg is None:
+        return float(value)
+    t = torch.tensor([float(value)], device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t)
+
+
+def job_throughput(w, world: int, ms_per_step: float) -> float:
+    """Whole-job dense-equivalent TFLOP/s: all ranks' layers over the slowest rank's time."""
+    return world * dense_equiv_flops(w) / (ms_per_step * 1e-3) / 1e12
+
+
 def dense_equiv_flops(w) -> float:
     return 4.0 * w.B * w.H * float(w.N) * w.N * w.d
 
@@ -284,8 +304,7 @@ def main():
     w = CONFIGS[args.config]
     if args.heads > 0:
         w = w.replace(H=args.heads)
-    if world > 1:
-        w = w.replace(seed=w.seed + 17 * rank)
+    w = rank_workload(w, rank, world)
 
     if args.impl == "reference":
         run_reference(args, w, rank, world)
@@ -351,11 +370,7 @@ def main():
         torch.cuda.synchronize(dev)
     if pg:
         pg.barrier()
-    total_ms = start.elapsed_time(stop)
-    if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t)
+    total_ms = max_over_ranks(start.elapsed_time(stop), pg, dev)
     status = bsa.bsa_device_status(buf.ws, stream)
     if status != 0:
         raise SystemExit(f"device status {status} after the timed steps")
@@ -386,13 +401,9 @@ def main():
             hout.copy_(out, non_blocking=True)
         s1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = s0.elapsed_time(s1) / args.e2e_steps
-        if pg:
-            t = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t)
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps, pg, dev)
         nbytes = q.numel() * q.element_size()
-        e2e = {"value": world * dense_equiv_flops(w) / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_throughput(w, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms}
         del hq, hk, hv, hout, dq, dk, dv
 
@@ -407,7 +418,7 @@ def main():
                          + (7 if w.extra_tokens > 0 else 0))   # theta, filter x2, finalize, fallback, modcent, glist
     line = {
         "metric": METRIC,
-        "value": world * dense_equiv_flops(w) / (ms_step * 1e-3) / 1e12,
+        "value": job_throughput(w, world, ms_step),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
