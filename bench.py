@@ -415,7 +415,7 @@ def main():
     dense_split = w.dense_rows[1] > w.dense_rows[0] and w.N > 256 * 64
     launches_per_step = (1 + 4 + 1 + (1 if dense_split else 0) + (2 if w.centroid else 0)
                          + (3 if w.dtype == "f32" else 0)
-                         + (7 if w.extra_tokens > 0 else 0))   # theta, filter x2, finalize, fallback, modcent, glist
+                         + (6 if w.extra_tokens > 0 else 0))   # theta, filter, finalize, fallback, modcent, glist
     line = {
         "metric": METRIC,
         "value": job_throughput(w, world, ms_step),

@@ -15,19 +15,18 @@
 //                    largest, lowered by a safety margin, is a lower bound of
 //                    the row's true E-th score (they are real candidates).
 //   filter_kernel    tcgen05: S = Qt K^T for 128 query blocks x 128 tokens per
-//                    tile, streamed over all tokens, twice.  Pass A counts the
-//                    row's unselected tokens into 88 linear buckets from its
-//                    bound up and keeps the highest bucket with at least E
-//                    tokens at or above it; it counts only from a floor, the
-//                    highest bucket already holding E counted tokens, which
-//                    rises as the pass goes.  Pass B keeps the tokens in or
-//                    above the kept bucket, in token order.  Both passes compute
-//                    the same scores and the bucket map is monotone, so the
-//                    survivors include the true top E.  Two warps share each
-//                    row, one per 64-token block of a tile; in pass B they
-//                    swap per-tile counts so the row's list stays in order.
-//   finalize_kernel  one warp per row: exact E-th largest of the survivors by
-//                    radix select, ties resolved by token order, compaction.
+//                    tile, streamed over all tokens once.  Each row's
+//                    unselected tokens are counted into 88 linear buckets from
+//                    its bound up, and kept (score key, token) in token order,
+//                    only from a floor that rises as the pass goes: the highest
+//                    bucket already holding E counted tokens.  A token of the
+//                    true top E is never below a floor, so every one of them is
+//                    kept (the bucket map is monotone); about 1.5-3k tokens per
+//                    row are.  Two warps share each row, one per 64-token block
+//                    of a tile, and swap per-tile counts so the row's list stays
+//                    in order.
+//   finalize_kernel  one warp per row: exact E-th largest of the kept tokens
+//                    by radix select, ties resolved by token order, compaction.
 //   fallback_kernel  rows whose survivors overflowed the buffer: all candidate
 //                    scores into a scratch row, radix select over the row.
 #include <float.h>
@@ -75,7 +74,6 @@ struct ExArgs {
     int dense_begin, dense_end;
     float *theta;                      // [rows] raw-dot lower bounds (+inf: no extras)
     float *smax;                       // [rows] largest sampled score
-    int32_t *bucket;                   // [rows] lowest bucket kept by pass B (-1: every unselected token)
     unsigned long long *buf;           // [rows, cap] (ord key << 32 | token)
     int32_t *cnt;                      // [rows] survivors (may exceed cap)
     int32_t *ovf;                      // [0]: count, [1..]: overflowed rows
@@ -247,7 +245,8 @@ struct FLay {
     static constexpr int kOffBar = kOffK + kFS * kKBytes;   // k_full[FS], k_empty[FS], s_full[2], s_free[2], done
     static constexpr int kOffMisc = kOffBar + (2 * kFS + 5) * 8;
     static constexpr int kOffHist = kOffMisc + 16;                              // [128 rows][kHistPitch] u32
-    static constexpr int kOffPair = kOffHist + kRowsPerCta * kHistPitch * 4;    // [2][2 groups][128 rows] i32
+    static constexpr int kOffPar = kOffHist + kRowsPerCta * kHistPitch * 4;     // [128 rows] {w, c}
+    static constexpr int kOffPair = kOffPar + kRowsPerCta * 8;                   // [2][2 groups][128 rows] i32
     static constexpr int kOffStage = kOffPair + 4 * kRowsPerCta * 4;            // [8 warps][32 rows][33] u32
     static constexpr int kOffBase = kOffStage + 8 * 32 * kStagePitch * 4;       // [8 warps][32] i32
     static constexpr int kOffList = kOffBase + 8 * 32 * 4;                      // [8 warps][1024] u16
@@ -278,7 +277,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads)
 // Warps 0-7 read the scores: warp w takes the rows of TMEM lane quarter w & 3
 // and, of each 128-token tile, key block 2t + (w >> 2).  Warp 8 loads K tiles,
 // warp 9 issues the MMAs and owns TMEM.
-template <int D, bool kCount>
+template <int D>
 __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ CUtensorMap tm_k, ExArgs a)
 {
     using L = FLay<D>;
@@ -295,14 +294,15 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kOffMisc);
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(sm + L::kOffMisc + 4);
     uint32_t *hist = reinterpret_cast<uint32_t *>(sm + L::kOffHist);   // [row][kHistPitch]
+    float2 *par = reinterpret_cast<float2 *>(sm + L::kOffPar);         // [row] bucket map
 
     // Per-row bucket map.  y = fma_rz(x, w, 2^23 + 1 - th w) clamped to 2^23 +
     // kBuckets - 1, so that for x >= th the bits of y are 0x4B000000 + 1 +
     // trunc((x - th) w) up to rounding (bucket 0 takes the rounding slack just
     // below th).  w spreads the buckets over [th, th + kSpan (smax - th)]: the
     // sampled maximum need not bound the row, so the range reaches well past
-    // it, and the last bucket is open-ended.  y is monotone in x, and both
-    // passes compute it identically, which is all exactness needs.  th = +inf
+    // it, and the last bucket is open-ended.  y is monotone in x, which is all
+    // exactness needs.  th = +inf
     // marks rows without extra tokens; -FLT_MAX stands in for "no bound".
     const int r = threadIdx.x & (kRowsPerCta - 1);
     const int64_t row = (int64_t)bh * a.nQB + min(i0 + r, a.nQB - 1);
@@ -344,8 +344,8 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
             st_shared_v4(base + dc * (kRowsPerCta * 128) + ((c16 ^ (r & 7)) << 4), w[0], w[1], w[2], w[3]);
         }
         fence_async_smem();
-        if (kCount)
-            for (int k = 0; k < kBuckets; ++k) hist[r * kHistPitch + k] = 0;
+        for (int k = 0; k < kBuckets; ++k) hist[r * kHistPitch + k] = 0;
+        par[r] = make_float2(inv_w, cw);
     }
     tc_fence_before();
     __syncthreads();
@@ -398,9 +398,6 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
         const int g = warp >> 2, sub = warp & 3;
         const bool active = th0 < INFINITY;
         const float ytop = 8388608.f + (float)(kBuckets - 1);
-        // pass B keeps y >= yk; keep_from < 0 (fewer than E candidates) keeps all
-        const int kf = (kCount || !live) ? 0 : a.bucket[row];
-        const float yk = kf < 0 ? -INFINITY : 8388608.f + (float)kf;
         int32_t *pair = reinterpret_cast<int32_t *>(sm + L::kOffPair);
         uint32_t *stage = reinterpret_cast<uint32_t *>(sm + L::kOffStage) + warp * 32 * kStagePitch;
         int32_t *base = reinterpret_cast<int32_t *>(sm + L::kOffBase) + warp * 32;
@@ -409,9 +406,10 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
         // hist + 4 (kHistPitch r + bucket) = hbase0 + 4 kHistPitch r + 4 bits(y), wrapping mod 2^32
         const uint32_t hbase0 = smem_u32(hist) - 4u * 0x4B000000u;
         const uint32_t hrow = hbase0 + 4u * (uint32_t)(kHistPitch * r);
-        // Pass A counts only buckets >= floor.  The floor is the highest bucket
-        // already holding E counted tokens at or above it; it only rises, so the
-        // final cut is never below it and the counts from the cut up stay exact.
+        // Tokens are counted and kept only from the floor up.  The floor is the
+        // highest bucket already holding E counted tokens at or above it; it only
+        // rises, so the true top E are all at or above every floor taken, and
+        // every token kept scores at least the floor of its time.
         int floor_k = 0;
         auto raise_floor = [&]() {
             uint32_t acc = 0;
@@ -430,7 +428,7 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
             }
         };
         const uint32_t *bm = a.bitmask + row * a.nW;
-        int cnt = 0;   // pass B: survivors of this row so far (both warps of the row agree)
+        int cnt = 0;   // survivors of this row so far (both warps of the row agree)
         const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
         uint32_t word = bm[g >> 5];
         for (int t = 0; t < ntiles; ++t) {
@@ -454,9 +452,7 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
             const int tok0 = blk * 64;
             const bool use = go && active && blk < a.nKB && !((word >> (blk & 31)) & 1u);
             const int nvalid = max(0, min(64, a.N - tok0));
-            // threshold in bucket space: pass A counts from the floor up, pass B
-            // keeps from the cut up
-            const float ythr = kCount ? 8388608.f + (float)floor_k : yk;
+            const float ythr = 8388608.f + (float)floor_k;   // the floor in bucket space
             uint32_t m0 = 0, m1 = 0;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -471,8 +467,8 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
                 m1 &= nvalid <= 32 ? 0u : (1u << (nvalid - 32)) - 1u;
             }
             const int cmine = __popc(m0) + __popc(m1);
-            int out_at = cnt;   // pass B: this row's first output slot for this block
-            if (!kCount) {
+            int out_at = cnt;   // this row's first output slot for this block
+            {
                 // the row's other warp holds the tile's other block: swap counts so
                 // that block 2t's survivors precede block 2t + 1's
                 pair[((t & 1) * 2 + g) * kRowsPerCta + r] = cmine;
@@ -498,15 +494,12 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
                     for (uint32_t mm = m; mm != 0u; mm &= mm - 1u) {
                         const int e = __ffs(mm) - 1;
                         const uint32_t x = select32(vh, e);
-                        if (kCount) {
-                            const float y = fminf(__fmaf_rz(__uint_as_float(x), inv_w, cw), ytop);
-                            red_shared_add1(hrow + 4u * (uint32_t)__float_as_int(y));
-                        } else {
-                            if (out_at + (int)__popc(m & ((1u << e) - 1u)) < a.cap)
-                                out[out_at + __popc(m & ((1u << e) - 1u))] =
-                                    ((unsigned long long)ord_key(__uint_as_float(x)) << 32) |
-                                    (uint32_t)(tok0 + 32 * hf + e);
-                        }
+                        const float y = fminf(__fmaf_rz(__uint_as_float(x), inv_w, cw), ytop);
+                        red_shared_add1(hrow + 4u * (uint32_t)__float_as_int(y));
+                        const int pos = out_at + (int)__popc(m & ((1u << e) - 1u));
+                        if (pos < a.cap)
+                            out[pos] = ((unsigned long long)ord_key(__uint_as_float(x)) << 32) |
+                                       (uint32_t)(tok0 + 32 * hf + e);
                     }
                 } else {
                     int incl = c;
@@ -518,11 +511,7 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
                     const int total = __shfl_sync(0xffffffffu, incl, 31);
                     if (m != 0u) {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            stage[lane * kStagePitch + e] =
-                                kCount ? 4u * (uint32_t)__float_as_int(
-                                                  fminf(__fmaf_rz(__uint_as_float(vh[e]), inv_w, cw), ytop))
-                                       : vh[e];
+                        for (int e = 0; e < 32; ++e) stage[lane * kStagePitch + e] = vh[e];
                         int j = incl - c;
                         base[lane] = out_at - j;   // output slot = base + list index
                         for (uint32_t mm = m; mm != 0u; mm &= mm - 1u)
@@ -536,16 +525,14 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
                             const int e = (int)(ent & 31u), o = (int)(ent >> 5);
                             const int rr = sub * 32 + o;
                             const uint32_t x = stage[o * kStagePitch + e];
-                            if (kCount) {
-                                red_shared_add1(hbase0 + 4u * (uint32_t)(kHistPitch * rr) + x);
-                            } else {
-                                const int pos = base[o] + idx;
-                                if (pos < a.cap) {
-                                    const int64_t row_o = (int64_t)bh * a.nQB + min(i0 + rr, a.nQB - 1);
-                                    a.buf[row_o * a.cap + pos] =
-                                        ((unsigned long long)ord_key(__uint_as_float(x)) << 32) |
-                                        (uint32_t)(tok0 + 32 * hf + e);
-                                }
+                            const float2 wc = par[rr];
+                            const float y = fminf(__fmaf_rz(__uint_as_float(x), wc.x, wc.y), ytop);
+                            red_shared_add1(hbase0 + 4u * (uint32_t)(kHistPitch * rr) + 4u * (uint32_t)__float_as_int(y));
+                            const int pos = base[o] + idx;
+                            if (pos < a.cap) {
+                                const int64_t row_o = (int64_t)bh * a.nQB + min(i0 + rr, a.nQB - 1);
+                                a.buf[row_o * a.cap + pos] = ((unsigned long long)ord_key(__uint_as_float(x)) << 32) |
+                                                             (uint32_t)(tok0 + 32 * hf + e);
                             }
                         }
                     }
@@ -554,29 +541,12 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
                 out_at += c;
             }
             word = word_next;
-            if (kCount && (t < 32 || (t & 7) == 7)) raise_floor();   // every tile while it climbs
+            if (t < 32 || (t & 7) == 7) raise_floor();   // every tile while it climbs
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[sb]);
         }
-        named_bar_sync(1, 256);   // every count of the CTA is in
-        if (g == 0 && live) {
-            if (kCount) {
-                // highest bucket with at least E candidates at or above it
-                uint32_t acc = 0;
-                int keep_from = -1;
-                for (int k = kBuckets - 1; k >= 0; --k) {
-                    acc += hist[r * kHistPitch + k];
-                    if (acc >= (uint32_t)a.E) {
-                        keep_from = k;
-                        break;
-                    }
-                }
-                a.bucket[row] = keep_from;
-            } else {
-                a.cnt[row] = cnt;
-            }
-        }
+        if (g == 0 && live) a.cnt[row] = cnt;
     }
     tc_fence_before();
     __syncthreads();
@@ -775,18 +745,15 @@ template <int D>
 cudaError_t launch_filter(dim3 grid, const CUtensorMap &tm, const ExArgs &a, cudaStream_t st)
 {
     const int bytes = (int)FLay<D>::bytes;
-    cudaError_t e = cudaFuncSetAttribute(filter_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = cudaFuncSetAttribute(filter_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(filter_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    filter_kernel<D, true><<<grid, 320, bytes, st>>>(tm, a);
-    filter_kernel<D, false><<<grid, 320, bytes, st>>>(tm, a);
+    filter_kernel<D><<<grid, 320, bytes, st>>>(tm, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-int64_t extra_buffer_capacity() { return 1024; }
+int64_t extra_buffer_capacity() { return 4096; }
 
 cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, const void *k,
                          int32_t *extra_idx, int32_t *extra_count, char *ws, const WsLayout &L, cudaStream_t st)
@@ -814,7 +781,6 @@ cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, 
     a.dense_end = p.dense_row_end;
     a.theta = reinterpret_cast<float *>(ws + L.ex_theta);
     a.smax = reinterpret_cast<float *>(ws + L.ex_smax);
-    a.bucket = reinterpret_cast<int32_t *>(ws + L.ex_bucket);
     a.buf = reinterpret_cast<unsigned long long *>(ws + L.ex_buf);
     a.cnt = reinterpret_cast<int32_t *>(ws + L.ex_cnt);
     a.ovf = reinterpret_cast<int32_t *>(ws + L.ex_ovf);
