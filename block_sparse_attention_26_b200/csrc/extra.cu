@@ -155,34 +155,47 @@ __global__ void __launch_bounds__(256) theta_kernel(ExArgs a)
     const uint32_t *bm = a.bitmask + r * a.nW;
     const float *srow = a.S + r * a.nKB;
     for (int c = lane; c < a.d; c += 32) qs[warp][c] = __bfloat162float(__float2bfloat16_rn(a.qbar[r * a.d + c]));
-    // best unselected blocks by pooled score (rounds of warp argmax) until the
-    // sample holds E tokens (a partial last block holds fewer than 64), at most
-    // 8 blocks = 512 tokens
+    // Good unselected blocks by pooled score until the sample holds E tokens (a
+    // partial last block holds fewer than 64), at most 8 blocks = 512 tokens: one
+    // scan in which each lane keeps its two best blocks, then picks among the
+    // lanes' candidates.  Any sample of real candidates gives a valid bound; a
+    // better sample gives a tighter one.
+    float b1 = -INFINITY, b2 = -INFINITY;
+    int i1 = -1, i2 = -1;
+    for (int j = lane; j < a.nKB; j += 32) {
+        if (is_kept(bm, j)) continue;
+        const float v = srow[j];
+        if (i1 < 0 || v > b1) {
+            b2 = b1;
+            i2 = i1;
+            b1 = v;
+            i1 = j;
+        } else if (i2 < 0 || v > b2) {
+            b2 = v;
+            i2 = j;
+        }
+    }
     int got = 0, ntok = 0;
     for (int t = 0; t < 8 && ntok < a.E + 64 * kSampleBlocks; ++t) {
-        float best = -INFINITY;
-        int bi = -1;
-        for (int j = lane; j < a.nKB; j += 32) {
-            if (is_kept(bm, j)) continue;
-            bool taken = false;
-            for (int u = 0; u < got; ++u) taken |= blks[warp][u] == j;
-            if (taken) continue;
-            const float v = srow[j];
-            if (bi < 0 || v > best || (v == best && j < bi)) {
-                best = v;
-                bi = j;
-            }
-        }
+        float best = i1 >= 0 ? b1 : -INFINITY;
+        int bi = i1, bl = i1 >= 0 ? lane : 32;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const float ob = __shfl_xor_sync(0xffffffffu, best, o);
             const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (oi >= 0 && (bi < 0 || ob > best || (ob == best && oi < bi))) {
+            const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
+            if (oi >= 0 && (bi < 0 || ob > best || (ob == best && ol < bl))) {
                 best = ob;
                 bi = oi;
+                bl = ol;
             }
         }
         if (bi < 0) break;
+        if (lane == bl) {   // the winning lane moves to its second candidate
+            b1 = b2;
+            i1 = i2;
+            i2 = -1;
+        }
         if (lane == 0) blks[warp][got] = bi;
         __syncwarp();
         ++got;

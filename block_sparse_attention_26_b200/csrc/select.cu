@@ -29,7 +29,7 @@
 namespace bsa {
 namespace {
 
-constexpr int kRows = 32;     // query-block rows per CTA
+constexpr int kRows = 64;     // query-block rows per CTA (8 per warp)
 constexpr int kKeys = 128;    // key blocks per pass
 constexpr int kChan = 32;     // channels staged per step
 
@@ -51,9 +51,9 @@ __global__ void __launch_bounds__(256) scores_kernel(const float *__restrict__ q
     }
     const float *kb = kbar + (int64_t)bh * nKB * d;
     for (int j0 = 0; j0 < nKB; j0 += kKeys) {
-        double acc[4][4];
+        double acc[8][4];   // 8 rows x 4 keys per thread: 12 shared loads per 32 FMAs
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int a = 0; a < 8; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
         for (int c0 = 0; c0 < d; c0 += kChan) {
@@ -65,20 +65,20 @@ __global__ void __launch_bounds__(256) scores_kernel(const float *__restrict__ q
             __syncthreads();
 #pragma unroll 2
             for (int c = 0; c < kChan; ++c) {
-                double qv[4], kv[4];
+                double qv[8], kv[4];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) qv[a] = qs[4 * warp + a][c0 + c];
+                for (int a = 0; a < 8; ++a) qv[a] = qs[8 * warp + a][c0 + c];
 #pragma unroll
                 for (int b = 0; b < 4; ++b) kv[b] = ks[c][lane + 32 * b];
 #pragma unroll
-                for (int a = 0; a < 4; ++a)
+                for (int a = 0; a < 8; ++a)
 #pragma unroll
                     for (int b = 0; b < 4; ++b) acc[a][b] = __fma_rn(qv[a], kv[b], acc[a][b]);
             }
         }
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            const int r = r0 + 4 * warp + a;
+        for (int a = 0; a < 8; ++a) {
+            const int r = r0 + 8 * warp + a;
             if (r >= nQB) continue;
             float *row = S + ((int64_t)bh * nQB + r) * nKB;
 #pragma unroll
