@@ -190,16 +190,26 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+__device__ __forceinline__ float fmax3(float x, float y, float z)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(x), "f"(y), "f"(z));
+    return r;
+}
+
+// Maximum of 64 values with three-input max instructions (32 of them).
 __device__ __forceinline__ float max64(const float (&x)[64])
 {
-    float m[16];
+    float m[22];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m[i] = fmaxf(fmaxf(x[4 * i], x[4 * i + 1]), fmaxf(x[4 * i + 2], x[4 * i + 3]));
+    for (int i = 0; i < 21; ++i) m[i] = fmax3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+    m[21] = x[63];
+    float n[8];
 #pragma unroll
-    for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
-    return m[0];
+    for (int i = 0; i < 7; ++i) n[i] = fmax3(m[3 * i], m[3 * i + 1], m[3 * i + 2]);
+    n[7] = m[21];
+    const float a = fmax3(n[0], n[1], n[2]), b = fmax3(n[3], n[4], n[5]);
+    return fmax3(a, b, fmaxf(n[6], n[7]));
 }
 
 __device__ __forceinline__ void named_bar(int id, int count)
