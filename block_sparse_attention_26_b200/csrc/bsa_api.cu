@@ -72,6 +72,7 @@ WsLayout ws_layout(const bsa_params &p)
     const bool ex = D.E > 0;
     L.ex_theta = take(ex ? (size_t)D.rows * 4 : 0);
     L.ex_smax = take(ex ? (size_t)D.rows * 4 : 0);
+    L.ex_cut = take(ex ? (size_t)D.rows * 16 : 0);
     L.ex_buf = take(ex ? (size_t)D.rows * extra_buffer_capacity() * 8 : 0);
     L.ex_cnt = take(ex ? (size_t)D.rows * 4 : 0);
     L.ex_ovf = take(ex ? (size_t)(D.rows + 1) * 4 : 0);

@@ -43,6 +43,7 @@ struct WsLayout {
     size_t q16, k16, v16;  // [B, N, H, d] bf16 copies of f32 inputs (attention, f32 only)
     size_t ex_theta;       // [rows] f32 extra-token score bounds
     size_t ex_smax;        // [rows] f32 largest sampled token score
+    size_t ex_cut;         // [rows] f32x4 bucket map and final cut of the kept tokens
     size_t ex_buf;         // [rows, 1024] u64 surviving (score, token) pairs
     size_t ex_cnt;         // [rows] i32 survivors per row
     size_t ex_ovf;         // [1 + rows] i32 overflowed rows

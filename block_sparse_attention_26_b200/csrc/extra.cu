@@ -25,8 +25,10 @@
 //                    row are.  Two warps share each row, one per 64-token block
 //                    of a tile, and swap per-tile counts so the row's list stays
 //                    in order.
-//   finalize_kernel  one warp per row: exact E-th largest of the kept tokens
-//                    by radix select, ties resolved by token order, compaction.
+//   finalize_kernel  one warp per row: the kept tokens at or above the final cut
+//                    bucket (the highest holding E counted tokens), then their
+//                    exact E-th largest by radix select, ties resolved by token
+//                    order, compaction.
 //   fallback_kernel  rows whose survivors overflowed the buffer: all candidate
 //                    scores into a scratch row, radix select over the row.
 #include <float.h>
@@ -74,6 +76,7 @@ struct ExArgs {
     int dense_begin, dense_end;
     float *theta;                      // [rows] raw-dot lower bounds (+inf: no extras)
     float *smax;                       // [rows] largest sampled score
+    float4 *cut;                       // [rows] bucket map {w, c} and the final cut, as y of fma_rz(x, w, c)
     unsigned long long *buf;           // [rows, cap] (ord key << 32 | token)
     int32_t *cnt;                      // [rows] survivors (may exceed cap)
     int32_t *ovf;                      // [0]: count, [1..]: overflowed rows
@@ -559,7 +562,22 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[sb]);
         }
-        if (g == 0 && live) a.cnt[row] = cnt;
+        named_bar_sync(1, 256);   // every count of the CTA is in
+        if (g == 0 && live) {
+            a.cnt[row] = cnt;
+            // the final cut: the highest bucket with at least E counted tokens at or
+            // above it; no token below it can be in the top E
+            uint32_t acc = 0;
+            int kcut = -1;
+            for (int k = kBuckets - 1; k >= 0; --k) {
+                acc += hist[r * kHistPitch + k];
+                if (acc >= (uint32_t)a.E) {
+                    kcut = k;
+                    break;
+                }
+            }
+            a.cut[row] = make_float4(inv_w, cw, kcut < 0 ? -INFINITY : 8388608.f + (float)kcut, 0.f);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -586,20 +604,39 @@ __global__ void __launch_bounds__(256) finalize_kernel(ExArgs a)
         }
         return;
     }
-    const unsigned long long *buf = a.buf + r * a.cap;
+    unsigned long long *buf = a.buf + r * a.cap;
+    const uint32_t lt = (1u << lane) - 1u;
+    int n = cnt;
+    const float4 cu = a.cut[r];
+    if (cnt > a.E && cu.z > -INFINITY) {
+        // keep the entries at or above the final cut bucket (the filter's own bucket
+        // map, recomputed from the score), in place and in order
+        int wpos = 0;
+        for (int j0 = 0; j0 < cnt; j0 += 32) {
+            const int j = j0 + lane;
+            const unsigned long long e = j < cnt ? buf[j] : 0ull;
+            const float y = __fmaf_rz(key_to_float((uint32_t)(e >> 32)), cu.x, cu.y);
+            const bool keep = j < cnt && y >= cu.z;
+            const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+            __syncwarp();
+            if (keep) buf[wpos + __popc(bal & lt)] = e;
+            wpos += __popc(bal);
+        }
+        __syncwarp();
+        n = wpos;
+    }
     uint32_t vk = 0;
     int need = 0;
-    if (cnt > a.E) vk = warp_kth([&](int j) { return (uint32_t)(buf[j] >> 32); }, cnt, a.E, hist[warp], &need);
+    if (n > a.E) vk = warp_kth([&](int j) { return (uint32_t)(buf[j] >> 32); }, n, a.E, hist[warp], &need);
     // survivors are in ascending token order: keep key > v_k, and the first `need` equal ones
     int taken = 0, eq_taken = 0;
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int j0 = 0; j0 < cnt; j0 += 32) {
+    for (int j0 = 0; j0 < n; j0 += 32) {
         const int j = j0 + lane;
-        const bool valid = j < cnt;
+        const bool valid = j < n;
         const unsigned long long e = valid ? buf[j] : 0ull;
         const uint32_t key = (uint32_t)(e >> 32);
         bool keep;
-        if (cnt <= a.E) {
+        if (n <= a.E) {
             keep = valid;
         } else {
             const bool eq = valid && key == vk;
@@ -794,6 +831,7 @@ cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, 
     a.dense_end = p.dense_row_end;
     a.theta = reinterpret_cast<float *>(ws + L.ex_theta);
     a.smax = reinterpret_cast<float *>(ws + L.ex_smax);
+    a.cut = reinterpret_cast<float4 *>(ws + L.ex_cut);
     a.buf = reinterpret_cast<unsigned long long *>(ws + L.ex_buf);
     a.cnt = reinterpret_cast<int32_t *>(ws + L.ex_cnt);
     a.ovf = reinterpret_cast<int32_t *>(ws + L.ex_ovf);
