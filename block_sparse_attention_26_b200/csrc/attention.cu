@@ -664,71 +664,60 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t v_addr = smem_u32(sm + L::kOffV);
             bool ok = mbar_wait(bar_q, 0, abort_flag, a.status, 22);
             tc_fence_after();
-            // Event loop: S of the next tile is issued as soon as both halves have
-            // read the current S; O_h += P_h V_h as soon as half h's P is in.
-            int ns = 0, T = -1;
-            int np[2] = {0, 0};
-            long long idle_since = clock64();
-            while (ok && (T < 0 || np[0] < T || np[1] < T)) {
-                bool progressed = false;
-                if (T < 0) {
-                    const int ks = ns % kKS;
-                    // S(ns) goes to buffer ns & 1 once P(ns - 2), which sits there, has been
-                    // issued to both halves' P V products (the tensor pipe keeps issue order)
-                    if (mbar_test(&k_full[ks], (ns / kKS) & 1) && (ns < 2 || (np[0] >= ns - 1 && np[1] >= ns - 1))) {
-                        tc_fence_after();
-                        if (kkind[ks] == TILE_GATHER && !a.gather_tma) fence_async_smem();   // rows by cp.async
-                        if (kkind[ks] == TILE_END) {
-                            T = ns;
-                        } else {
-#pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk) {
-                                const uint64_t ad =
-                                    sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
-                                const uint64_t bd = sdesc_sw128(
-                                    k_addr + ks * L::kTileBytes + (kk >> 2) * (kTK * 128) + (kk & 3) * 32, 16, 1024);
-                                umma_bf16(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-                            }
-                            umma_commit(&s_full[ns & 1]);
-                            umma_commit(&k_empty[ks]);
-                            TRACE(2, ns);
-                            ++ns;
-                        }
-                        progressed = true;
-                    }
+            // Fixed order: S(0), S(1), then for each tile j the P V products of
+            // both halves and S(j + 2), which goes to the buffer P(j) held (the tensor
+            // pipe runs one thread's MMAs in issue order).  Every wait is a blocking
+            // try_wait: polling barriers from this thread between MMAs stalls the
+            // tensor pipe (each test costs tens of cycles while MMAs read shared
+            // memory).
+            int T = -1;   // tile count, once the end marker is seen
+            auto issue_s = [&](int ns) -> bool {
+                const int ks = ns % kKS;
+                ok = mbar_wait(&k_full[ks], (ns / kKS) & 1, abort_flag, a.status, 27);
+                if (!ok) return false;
+                tc_fence_after();
+                const int kind = kkind[ks];
+                if (kind == TILE_END) {
+                    T = ns;
+                    return false;
                 }
+                if (!a.gather_tma && kind == TILE_GATHER) fence_async_smem();   // rows by cp.async
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int t = np[hf];
-                    if (t >= ns) continue;
-                    const int pb = t & 1, vs = t % kVS;
-                    if (mbar_test(&p_full[2 * hf + pb], (t >> 1) & 1) && mbar_test(&v_full[vs], (t / kVS) & 1)) {
-                        tc_fence_after();
-                        if (info[vs].kind == TILE_GATHER && !a.gather_tma) fence_async_smem();   // rows by cp.async
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd =
+                        sdesc_sw128(k_addr + ks * L::kTileBytes + (kk >> 2) * (kTK * 128) + (kk & 3) * 32, 16, 1024);
+                    umma_bf16(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[ns & 1]);
+                umma_commit(&k_empty[ks]);
+                TRACE(2, ns);
+                return true;
+            };
+            // P_h(t) is in only after the softmax warps waited for V(t) (they read the
+            // tile's metadata there), so the V rows are in too
+            auto issue_pv = [&](int t, int hf) {
+                const int pb = t & 1, vs = t % kVS;
+                ok = mbar_wait(&p_full[2 * hf + pb], (t >> 1) & 1, abort_flag, a.status, 28);
+                if (!ok) return;
+                tc_fence_after();
+                if (!a.gather_tma && info[vs].kind == TILE_GATHER) fence_async_smem();   // rows by cp.async
 #pragma unroll
-                        for (int ks = 0; ks < kBK / 16; ++ks) {
-                            const uint64_t bd = sdesc_sw128(
-                                v_addr + vs * L::kTileBytes + hf * L::kHalfBytes + ks * 2048, kTK * 128, 1024);
-                            umma_bf16_ts(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd,
-                                         idesc_o, (t > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        umma_commit(&p_free[2 * hf + pb]);
-                        // the V slot is free once both halves used it; the later half releases it
-                        if (np[1 - hf] > t) umma_commit(&v_empty[vs]);
-                        if (hf == 0) TRACE(3, t);
-                        np[hf] = t + 1;
-                        progressed = true;
-                    }
+                for (int ks = 0; ks < kBK / 16; ++ks) {
+                    const uint64_t bd =
+                        sdesc_sw128(v_addr + vs * L::kTileBytes + hf * L::kHalfBytes + ks * 2048, kTK * 128, 1024);
+                    umma_bf16_ts(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd, idesc_o,
+                                 (t > 0 || ks > 0) ? 1u : 0u);
                 }
-                if (progressed) {
-                    idle_since = clock64();
-                } else if (*abort_flag) {
-                    ok = false;
-                } else if (clock64() - idle_since > kWaitCycles) {
-                    *abort_flag = 1;
-                    report(a.status, BSA_DEV_TIMEOUT, 26);
-                    ok = false;
-                }
+                umma_commit(&p_free[2 * hf + pb]);
+                if (hf == 1) umma_commit(&v_empty[vs]);   // both halves have used the V slot
+                if (hf == 0) TRACE(3, t);
+            };
+            if (ok && issue_s(0)) issue_s(1);
+            for (int j = 0; ok && (T < 0 || j < T); ++j) {
+                issue_pv(j, 0);
+                if (ok) issue_pv(j, 1);
+                if (ok && T < 0) issue_s(j + 2);
             }
             // end-of-list marker for the softmax warps (both halves have taken every
             // earlier S, so buffer T & 1 may complete its next phase)
