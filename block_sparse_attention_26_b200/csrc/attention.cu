@@ -38,12 +38,14 @@
 //              so K prefetch never waits for V slots; a K slot is released as
 //              soon as its S product is done, the V producer also publishes each
 //              tile's masks to the softmax warps.
-//   warp 9     MMA issuer (one thread, event loop): S = Q K^T (A and B from
-//              shared memory) runs up to two tiles ahead of the softmax, into two
-//              TMEM buffers; O_h += P_h V_h (A = P_h from TMEM) is issued as soon
-//              as half h of a tile's P is in.  S(j) may overwrite buffer j & 1 once
-//              P(j - 2) there has been issued to both P V products: the tensor pipe
-//              runs one thread's MMAs in issue order.
+//   warp 9     MMA issuer (one thread, fixed order): S = Q K^T (A and B from
+//              shared memory) runs one tile ahead of the softmax, into two TMEM
+//              buffers; per tile j it issues O_h += P_h V_h (A = P_h from TMEM)
+//              for h = 0, 1 as each half's P comes in, then S(j + 2) into the
+//              buffer P(j) held: the tensor pipe runs one thread's MMAs in issue
+//              order.  The completion of S(j) also frees K slot j % 2, and the
+//              completion of S(j + 1) tells a softmax warp that wants to rescale
+//              O at tile j that P V(j - 1) is done.
 // TMEM (512 columns): S of tile j at 128 (j & 1), half h's P (bf16 pairs) written
 // over its own S columns 128 (j & 1) + 64 h once read; O_h at 256 + 128 h.
 #include <math.h>
@@ -149,9 +151,8 @@ struct Lay {
     static constexpr int kOffKind = kOffV + kVS * kTileBytes;
     static constexpr int kOffInfo = kOffKind + 16;
     static constexpr int kOffBar = kOffInfo + kVS * (int)sizeof(TileInfo);
-    // q, done, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2 buffers],
-    // p_full[2 halves][2], p_free[2 halves][2]
-    static constexpr int kNumBar = 2 + 2 * kKS + 2 * kVS + 2 + 8;
+    // q, done, k_full[KS], v_full[VS], v_empty[VS], s_full[2 buffers], p_full[2 halves][2]
+    static constexpr int kNumBar = 2 + kKS + 2 * kVS + 2 + 4;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
     static constexpr int kOffML = kOffMisc + 16;                 // [2][128] (m, l) per half
     static constexpr int kOffBias = kOffML + 2 * kM * 8;         // [VS][128] per-column bias (gathers)
@@ -263,11 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kOffBar);
     uint64_t *bar_q = bars, *bar_done = bars + 1;
-    uint64_t *k_full = bars + 2, *k_empty = k_full + kKS;
-    uint64_t *v_full = k_empty + kKS, *v_empty = v_full + kVS;
+    uint64_t *k_full = bars + 2;
+    uint64_t *v_full = k_full + kKS, *v_empty = v_full + kVS;
     uint64_t *s_full = v_empty + kVS;         // [buffer]
     uint64_t *p_full = s_full + 2;            // [half * 2 + buffer]
-    uint64_t *p_free = p_full + 4;            // [half * 2 + buffer]
     volatile int32_t *kkind = reinterpret_cast<volatile int32_t *>(sm + L::kOffKind);
     volatile TileInfo *info = reinterpret_cast<volatile TileInfo *>(sm + L::kOffInfo);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kOffMisc);
@@ -290,20 +290,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
         mbar_init(bar_done, 1);
-        for (int s = 0; s < kKS; ++s) {
-            mbar_init(&k_full[s], 1);
-            mbar_init(&k_empty[s], 1);
-        }
+        for (int s = 0; s < kKS; ++s) mbar_init(&k_full[s], 1);
         for (int s = 0; s < kVS; ++s) {
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        for (int i = 0; i < 4; ++i) {
-            mbar_init(&p_full[i], 4);
-            mbar_init(&p_free[i], 1);
-        }
+        for (int i = 0; i < 4; ++i) mbar_init(&p_full[i], 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -393,7 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap *tm_gc = is_k ? &tm_gxk : &tm_gxv;   // modified-centroid rows
         const int depth = is_k ? kKS : kVS;
         uint64_t *full = is_k ? k_full : v_full;
-        uint64_t *empty = is_k ? k_empty : v_empty;
+        // a K slot is free once the S product that read it is done (S(j) sits in
+        // buffer j & 1 = slot j % 2)
+        static_assert(kKS == 2, "K slots and S buffers must pair up");
+        uint64_t *empty = is_k ? s_full : v_empty;
         uint8_t *ring = sm + (is_k ? L::kOffK : L::kOffV);
         int gl0 = 0, gln = 0, glU = 0, glm0 = 0;   // the gathered tile: list entries [gl0, gl0 + gln)
         const __nv_bfloat16 *src_x = is_k ? a.kx : a.vx;
@@ -678,6 +675,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const int kind = kkind[ks];
                 if (kind == TILE_END) {
+                    // end-of-list marker for the softmax warps, committed at once: it
+                    // completes after every MMA issued so far (P V of tiles < T - 1)
+                    umma_commit(&s_full[ns & 1]);
                     T = ns;
                     return false;
                 }
@@ -690,7 +690,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_bf16(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&s_full[ns & 1]);
-                umma_commit(&k_empty[ks]);
                 TRACE(2, ns);
                 return true;
             };
@@ -709,7 +708,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_bf16_ts(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd, idesc_o,
                                  (t > 0 || ks > 0) ? 1u : 0u);
                 }
-                umma_commit(&p_free[2 * hf + pb]);
                 if (hf == 1) umma_commit(&v_empty[vs]);   // both halves have used the V slot
                 if (hf == 0) TRACE(3, t);
             };
@@ -719,9 +717,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok) issue_pv(j, 1);
                 if (ok && T < 0) issue_s(j + 2);
             }
-            // end-of-list marker for the softmax warps (both halves have taken every
-            // earlier S, so buffer T & 1 may complete its next phase)
-            if (ok) umma_commit(&s_full[T & 1]);
             umma_commit(bar_done);
             volatile int32_t no_abort = 0;
             mbar_wait(bar_done, 0, &no_abort, a.status, 25);
@@ -736,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qsel = (a.Bq == 64 && !dense) ? (r >> 6) : 0;
         const float scale = a.scale_log2;
         const uint32_t col_o = kColO + 128 * hf;
-        uint64_t *pf = p_full + 2 * hf, *pe = p_free + 2 * hf;
+        uint64_t *pf = p_full + 2 * hf;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         int j = 0;
@@ -839,7 +834,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(tmem + lane_base + col_s, pk);   // over this half's S, already read
             if (__any_sync(0xffffffffu, rescale)) {
                 // the accumulator must hold every earlier P V product before it is scaled
-                ok = mbar_wait(&pe[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status, 33);
+                // (S(j + 1), or the end marker, is issued after P V(j - 1))
+                ok = mbar_wait(&s_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.status, 33);
                 if (!(ok = __all_sync(0xffffffffu, ok))) break;
                 tc_fence_after();
 #pragma unroll 1
@@ -860,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (r == 0) TRACE(6 + 3 * hf, j);
         }
         const int T = j;
-        if (ok && T >= 1) ok = mbar_wait(&pe[(T - 1) & 1], ((T - 1) >> 1) & 1, abort_flag, a.status, 34);
+        if (ok && T >= 1) ok = mbar_wait(bar_done, 0, abort_flag, a.status, 34);   // every MMA done
         ok = __all_sync(0xffffffffu, ok);
         // ------------------------------------------------------ epilogue
         // merge the halves: O = (wA O_A + wB O_B) / (wA lA + wB lB), w = 2^(m_half - m)
