@@ -38,7 +38,8 @@
 //              so K prefetch never waits for V slots; a K slot is released as
 //              soon as its S product is done, the V producer also publishes each
 //              tile's masks to the softmax warps.
-//   warp 9     MMA issuer (one thread, fixed order): S = Q K^T (A and B from
+//   warp 9     MMA issuer (fixed order; the whole warp runs it, one elected
+//              lane issues): S = Q K^T (A and B from
 //              shared memory) runs one tile ahead of the softmax, into two TMEM
 //              buffers; per tile j it issues O_h += P_h V_h (A = P_h from TMEM)
 //              for h = 0, 1 as each half's P comes in, then S(j + 2) into the
@@ -180,15 +181,40 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// O[tmem] (+)= A[tmem] * B[smem]: A (M x K, bf16 pairs per 32-bit column) from TMEM.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t accumulate)
+// UMMA issue in warp-wide form: every lane of the warp executes these with the
+// same operands and one elected lane issues (the operands stay warp-uniform).
+// D[tmem] (+)= A[smem] * B[smem]^T.
+__device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]: A (M x K, bf16 pairs per 32-bit column) from TMEM.
+__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive on `bar` once every tcgen05 operation the warp issued so far completes.
+__device__ __forceinline__ void umma_commit_w(uint64_t *bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
 }
 
 __device__ __forceinline__ float fmax3(float x, float y, float z)
@@ -653,13 +679,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("cp.async.wait_all;" ::: "memory");   // this lane's gathered rows have landed
     } else if (warp == 9) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // The whole warp runs it (warp-uniform operands); one elected lane issues.
+        {
             const uint32_t idesc_s = idesc_bf16_f32(kM, kTK, 0, 0);
             const uint32_t idesc_o = idesc_bf16_f32(kM, D, 0, 1);
             const uint32_t q_addr = smem_u32(sm + L::kOffQ);
             const uint32_t k_addr = smem_u32(sm + L::kOffK);
             const uint32_t v_addr = smem_u32(sm + L::kOffV);
-            bool ok = mbar_wait(bar_q, 0, abort_flag, a.status, 22);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag, a.status, 22));
             tc_fence_after();
             // Fixed order: S(0), S(1), then for each tile j the P V products of
             // both halves and S(j + 2), which goes to the buffer P(j) held (the tensor
@@ -670,14 +697,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             int T = -1;   // tile count, once the end marker is seen
             auto issue_s = [&](int ns) -> bool {
                 const int ks = ns % kKS;
-                ok = mbar_wait(&k_full[ks], (ns / kKS) & 1, abort_flag, a.status, 27);
+                ok = __all_sync(0xffffffffu, mbar_wait(&k_full[ks], (ns / kKS) & 1, abort_flag, a.status, 27));
                 if (!ok) return false;
                 tc_fence_after();
-                const int kind = kkind[ks];
+                const int kind = __shfl_sync(0xffffffffu, (int)kkind[ks], 0);
                 if (kind == TILE_END) {
                     // end-of-list marker for the softmax warps, committed at once: it
                     // completes after every MMA issued so far (P V of tiles < T - 1)
-                    umma_commit(&s_full[ns & 1]);
+                    umma_commit_w(&s_full[ns & 1]);
                     T = ns;
                     return false;
                 }
@@ -687,17 +714,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
                     const uint64_t bd =
                         sdesc_sw128(k_addr + ks * L::kTileBytes + (kk >> 2) * (kTK * 128) + (kk & 3) * 32, 16, 1024);
-                    umma_bf16(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    umma_ss_w(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_full[ns & 1]);
-                TRACE(2, ns);
+                umma_commit_w(&s_full[ns & 1]);
+                if (lane == 0) TRACE(2, ns);
                 return true;
             };
             // P_h(t) is in only after the softmax warps waited for V(t) (they read the
             // tile's metadata there), so the V rows are in too
             auto issue_pv = [&](int t, int hf) {
                 const int pb = t & 1, vs = t % kVS;
-                ok = mbar_wait(&p_full[2 * hf + pb], (t >> 1) & 1, abort_flag, a.status, 28);
+                ok = __all_sync(0xffffffffu, mbar_wait(&p_full[2 * hf + pb], (t >> 1) & 1, abort_flag, a.status, 28));
                 if (!ok) return;
                 tc_fence_after();
                 if (!a.gather_tma && info[vs].kind == TILE_GATHER) fence_async_smem();   // rows by cp.async
@@ -705,11 +732,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int ks = 0; ks < kBK / 16; ++ks) {
                     const uint64_t bd =
                         sdesc_sw128(v_addr + vs * L::kTileBytes + hf * L::kHalfBytes + ks * 2048, kTK * 128, 1024);
-                    umma_bf16_ts(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd, idesc_o,
+                    umma_ts_w(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd, idesc_o,
                                  (t > 0 || ks > 0) ? 1u : 0u);
                 }
-                if (hf == 1) umma_commit(&v_empty[vs]);   // both halves have used the V slot
-                if (hf == 0) TRACE(3, t);
+                if (hf == 1) umma_commit_w(&v_empty[vs]);   // both halves have used the V slot
+                if (hf == 0 && lane == 0) TRACE(3, t);
             };
             if (ok && issue_s(0)) issue_s(1);
             for (int j = 0; ok && (T < 0 || j < T); ++j) {
@@ -717,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok) issue_pv(j, 1);
                 if (ok && T < 0) issue_s(j + 2);
             }
-            umma_commit(bar_done);
+            umma_commit_w(bar_done);
             volatile int32_t no_abort = 0;
             mbar_wait(bar_done, 0, &no_abort, a.status, 25);
         }
