@@ -217,6 +217,40 @@ __device__ __forceinline__ void umma_commit_w(uint64_t *bar)
         : "memory");
 }
 
+// Packed pairs of f32 (one instruction for two values; round to nearest).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 __device__ __forceinline__ float fmax3(float x, float y, float z)
 {
     float r;
@@ -789,8 +823,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mode = 0;
                 } else {
                     mode = 2;
+                    const float2 sc2 = make_float2(scale, scale);
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) s[c] = c < nc ? s[c] * scale : -INFINITY;
+                    for (int c = 0; c < 32; ++c) {
+                        const float2 y = fmul2(make_float2(s[2 * c], s[2 * c + 1]), sc2);
+                        s[2 * c] = 2 * c < nc ? y.x : -INFINITY;
+                        s[2 * c + 1] = 2 * c + 1 < nc ? y.y : -INFINITY;
+                    }
                 }
             } else if (kind == TILE_CENT) {
                 const uint64_t msk = info[vs].cmask[qsel][hf];
@@ -798,10 +837,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float pbias = info[vs].last_bias;
                 mode = msk ? 2 : 0;
                 if (msk) {
+                    const float2 sc2 = make_float2(scale, scale);
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        const float bias = c == pc ? pbias : 6.0f;       // log2(64) for full blocks
-                        s[c] = ((msk >> c) & 1ull) ? fmaf(s[c], scale, bias) : -INFINITY;
+                    for (int c = 0; c < 32; ++c) {
+                        // log2(64) for full blocks
+                        const float2 b2 = make_float2(2 * c == pc ? pbias : 6.0f, 2 * c + 1 == pc ? pbias : 6.0f);
+                        const float2 y = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, b2);
+                        s[2 * c] = ((msk >> (2 * c)) & 1ull) ? y.x : -INFINITY;
+                        s[2 * c + 1] = ((msk >> (2 * c + 1)) & 1ull) ? y.y : -INFINITY;
                     }
                 }
             } else {
@@ -811,9 +854,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float *bias = bias_sm + vs * kTK + 64 * hf;
                 mode = msk ? 2 : 0;
                 if (msk) {
+                    const float2 sc2 = make_float2(scale, scale);
+                    const float2 *bias2 = reinterpret_cast<const float2 *>(bias);
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        s[c] = ((msk >> c) & 1ull) ? fmaf(s[c], scale, bias[c]) : -INFINITY;
+                    for (int c = 0; c < 32; ++c) {
+                        const float2 y = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, bias2[c]);
+                        s[2 * c] = ((msk >> (2 * c)) & 1ull) ? y.x : -INFINITY;
+                        s[2 * c + 1] = ((msk >> (2 * c + 1)) & 1ull) ? y.y : -INFINITY;
+                    }
                 }
             }
             uint32_t pk[32];
@@ -835,26 +883,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 const float mref = m_ref == -INFINITY ? 0.f : m_ref;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                const float2 nm2 = make_float2(-mref, -mref);
                 if (mode == 1) {
-                    const float nm = -mref;
+                    const float2 sc2 = make_float2(scale, scale);
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const float p0 = ex2(fmaf(s[2 * c], scale, nm));
-                        const float p1 = ex2(fmaf(s[2 * c + 1], scale, nm));
-                        acc[c & 3] += p0 + p1;
+                        const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+                        const float p0 = ex2(x.x), p1 = ex2(x.y);
+                        acc[c & 1] = fadd2(acc[c & 1], make_float2(p0, p1));
                         pk[c] = pack_bf16x2(p0, p1);
                     }
                 } else {
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const float p0 = ex2(s[2 * c] - mref);
-                        const float p1 = ex2(s[2 * c + 1] - mref);
-                        acc[c & 3] += p0 + p1;
+                        const float2 x = fadd2(make_float2(s[2 * c], s[2 * c + 1]), nm2);
+                        const float p0 = ex2(x.x), p1 = ex2(x.y);
+                        acc[c & 1] = fadd2(acc[c & 1], make_float2(p0, p1));
                         pk[c] = pack_bf16x2(p0, p1);
                     }
                 }
-                l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
             }
             if (r == 0) TRACE(10 + 3 * hf, j);
             if (r == 0) TRACE(11 + 3 * hf, j);
