@@ -92,14 +92,15 @@ constexpr int kTraceBytes = 0;
 
 // What one 128-key tile holds; half h is one key block (or 64 centroids).
 struct TileInfo {
-    int32_t kind;
+    // per half, read by its softmax warps with one 16-byte load: {kind, who (exact:
+    // bit q set = query block q of the tile keeps the half's block), ncols (exact:
+    // valid key columns, 0 = empty half), pcol (centroid: column of a partial block,
+    // or -1)}
+    int4 h[2];
     int32_t blk[2];       // key block of each half (exact) or centroid chunk (centroid)
-    uint32_t who[2];      // exact: bit q set = query block q of the tile keeps the half's block
-    int32_t ncols[2];     // exact: valid key columns of each half (0 = empty half)
-    int32_t pcol[2];      // centroid: column of a partial block in each half, or -1
     float last_bias;      // centroid: log2 of the partial block's size
     int32_t pad;
-    uint64_t cmask[2][2]; // centroid: [query block][half] active centroid columns
+    uint64_t cmask[2][2]; // centroid / gathered: [query block][half] active columns
 };
 
 struct AttnArgs {
@@ -489,12 +490,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     TRACE(0, j);
                 } else {
                     TRACE(1, j);
-                    info[s].kind = kind;
                     for (int x = 0; x < 2; ++x) {
                         info[s].blk[x] = blk[x];
-                        info[s].who[x] = who[x];
-                        info[s].ncols[x] = nc[x];
-                        info[s].pcol[x] = pcol[x];
+                        info[s].h[x].x = kind;
+                        info[s].h[x].y = (int32_t)who[x];
+                        info[s].h[x].z = nc[x];
+                        info[s].h[x].w = pcol[x];
                         info[s].cmask[x][0] = cm[x][0];
                         info[s].cmask[x][1] = cm[x][1];
                     }
@@ -761,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(&p_full[2 * hf + pb], (t >> 1) & 1, abort_flag, a.status, 28));
                 if (!ok) return;
                 tc_fence_after();
-                if (!a.gather_tma && info[vs].kind == TILE_GATHER) fence_async_smem();   // rows by cp.async
+                if (!a.gather_tma && info[vs].h[0].x == TILE_GATHER) fence_async_smem();   // rows by cp.async
 #pragma unroll
                 for (int ks = 0; ks < kBK / 16; ++ks) {
                     const uint64_t bd =
@@ -802,7 +803,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                  mbar_wait(&v_full[vs], (j / kVS) & 1, abort_flag, a.status, 31);
             if (!(ok = __all_sync(0xffffffffu, ok))) break;
             tc_fence_after();
-            const int kind = info[vs].kind;
+            // (plain loads: the barrier waits above order them)
+            const TileInfo *ti = const_cast<const TileInfo *>(info) + vs;
+            const int4 hq = ti->h[hf];
+            const int kind = hq.x;
             if (kind == TILE_END) break;
             if (r == 0) TRACE(4 + 3 * hf, j);
             float s[64];
@@ -815,8 +819,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // 0: skip (no active column), 1: all 64 columns active, 2: masked / biased
             int mode;
             if (kind == TILE_EXACT) {
-                const bool act = (info[vs].who[hf] >> qsel) & 1u;
-                const int nc = act ? info[vs].ncols[hf] : 0;
+                const bool act = ((uint32_t)hq.y >> qsel) & 1u;
+                const int nc = act ? hq.z : 0;
                 if (nc >= kBK) {
                     mode = 1;
                 } else if (nc <= 0) {
@@ -832,9 +836,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else if (kind == TILE_CENT) {
-                const uint64_t msk = info[vs].cmask[qsel][hf];
-                const int pc = info[vs].pcol[hf];
-                const float pbias = info[vs].last_bias;
+                const uint64_t msk = ti->cmask[qsel][hf];
+                const int pc = hq.w;
+                const float pbias = ti->last_bias;
                 mode = msk ? 2 : 0;
                 if (msk) {
                     const float2 sc2 = make_float2(scale, scale);
@@ -850,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 // gathered columns: extra tokens (bias 0) and modified centroids
                 // (bias log2 of their remaining token count)
-                const uint64_t msk = info[vs].cmask[qsel][hf];
+                const uint64_t msk = ti->cmask[qsel][hf];
                 const float *bias = bias_sm + vs * kTK + 64 * hf;
                 mode = msk ? 2 : 0;
                 if (msk) {
