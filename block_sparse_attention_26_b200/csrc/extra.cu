@@ -304,6 +304,10 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
     const int b = bh / a.H, h = bh % a.H;
     const int i0 = blockIdx.x * kRowsPerCta;
     const int ntiles = (a.N + kTok - 1) / kTok;
+    // key tiles in the order t_first, t_first + 1, ..., wrapping: t_first sits a few
+    // frames' worth of tiles before the CTA's query rows, where scores run highest
+    const int t_first = max(0, min(ntiles - 1, (int)(((int64_t)(i0 + kRowsPerCta / 2) * a.Bq) / kTok)) - 32);
+    auto tile_at = [&](int t) { const int u = t_first + t; return u >= ntiles ? u - ntiles : u; };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kOffBar);
     uint64_t *k_full = bars, *k_empty = bars + L::kFS, *s_full = bars + 2 * L::kFS, *s_free = s_full + 2,
              *bar_done = s_full + 4;
@@ -379,7 +383,7 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
                 for (int half = 0; half < 2; ++half)
                     for (int dc = 0; dc < D / 64; ++dc)
                         tma_load_4d(dst + dc * (kTok * 128) + half * (64 * 128), &tm_k, &k_full[s], dc * 64, h,
-                                    t * kTok + half * 64, b);
+                                    tile_at(t) * kTok + half * 64, b);
             }
             volatile int32_t no_abort = 0;
             for (int s = 0; s < L::kFS; ++s) {
@@ -446,12 +450,12 @@ __global__ void __launch_bounds__(320, 1) filter_kernel(const __grid_constant__ 
         const uint32_t *bm = a.bitmask + row * a.nW;
         int cnt = 0;   // survivors of this row so far (both warps of the row agree)
         const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
-        uint32_t word = bm[g >> 5];
+        uint32_t word = bm[min((2 * tile_at(0) + g) >> 5, a.nW - 1)];
         for (int t = 0; t < ntiles; ++t) {
             const int sb = t & 1;
-            const int blk = 2 * t + g;
+            const int blk = 2 * tile_at(t) + g;
             // bitmask word of the next tile's block, fetched a tile early
-            const uint32_t word_next = bm[min((blk + 2) >> 5, a.nW - 1)];
+            const uint32_t word_next = bm[min((2 * tile_at(t + 1 < ntiles ? t + 1 : t) + g) >> 5, a.nW - 1)];
             // After an abort every wait fails at once: the loop still runs to the
             // end with no work, so both warps of a row meet at every pair barrier.
             const bool go = __all_sync(0xffffffffu, mbar_wait(&s_full[sb], (t >> 1) & 1, abort_flag, a.status, 45));
@@ -628,11 +632,21 @@ __global__ void __launch_bounds__(256) finalize_kernel(ExArgs a)
     uint32_t vk = 0;
     int need = 0;
     if (n > a.E) vk = warp_kth([&](int j) { return (uint32_t)(buf[j] >> 32); }, n, a.E, hist[warp], &need);
-    // survivors are in ascending token order: keep key > v_k, and the first `need` equal ones
+    // the survivors are two ascending token runs (the filter wraps around the key
+    // tiles): the second run starts at the one place where the token decreases
+    int split = 0;
+    for (int j0 = 1; j0 < n && split == 0; j0 += 32) {
+        const int j = j0 + lane;
+        const bool down = j < n && (uint32_t)buf[j] < (uint32_t)buf[j - 1];
+        const uint32_t dm = __ballot_sync(0xffffffffu, down);
+        if (dm) split = j0 + __ffs(dm) - 1;
+    }
+    // in ascending token order: keep key > v_k, and the first `need` equal ones
     int taken = 0, eq_taken = 0;
     for (int j0 = 0; j0 < n; j0 += 32) {
-        const int j = j0 + lane;
-        const bool valid = j < n;
+        const int i = j0 + lane;
+        const bool valid = i < n;
+        const int j = i + split < n ? i + split : i + split - n;
         const unsigned long long e = valid ? buf[j] : 0ull;
         const uint32_t key = (uint32_t)(e >> 32);
         bool keep;
