@@ -361,6 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 4; ++i) mbar_init(&p_full[i], 4);
         *abort_flag = 0;
         fence_mbar_init();
+        // Q first: its load overlaps the rest of the set-up
+        prefetch_tmap(&tm_q);
+        mbar_expect_tx(bar_q, L::kQBytes);
+        for (int dc = 0; dc < D / 64; ++dc)
+            tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
     }
     if (warp == 9) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -376,24 +381,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             // gathered columns: the union of the query blocks' extra tokens (merged
             // by glist_kernel, padded to a multiple of 4), then each query block's
             // modified centroids
+            // list lengths in one round of loads, then the lists, eight loads in
+            // flight per lane
+            const int64_t gi = sidx;
+            int len = 0;
+            if (lane < nq) len = a.xcnt[rbase + lane];
+            else if (lane >= 2 && lane < 2 + nq) len = a.extra_count[rbase + lane - 2];
+            else if (lane == 4) len = a.glcnt[gi];
+            const int U = __shfl_sync(0xffffffffu, len, 4);
             for (int q = 0; q < nq; ++q) {
                 const int64_t rq = rbase + q;
-                const int nx = min(a.xcnt[rq], a.Ecap);
-                for (int e = lane; e < nx; e += 32) gl_bias[q * kMaxE + e] = a.xbias[rq * a.Ecap + e];
-                for (int w = lane; w < a.nW; w += 32) aff[q * a.nW + w] = a.xaff[rq * a.nW + w];
+                const int nx = min(__shfl_sync(0xffffffffu, len, q), a.Ecap);
+                const int ec = min(__shfl_sync(0xffffffffu, len, 2 + q), a.E);
+                for (int e0 = 0; e0 < nx; e0 += 256) {
+                    float xb[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int e = e0 + 32 * u + lane;
+                        xb[u] = e < nx ? a.xbias[rq * a.Ecap + e] : 0.f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int e = e0 + 32 * u + lane;
+                        if (e < nx) gl_bias[q * kMaxE + e] = xb[u];
+                    }
+                }
+                for (int w0 = 0; w0 < a.nW; w0 += 128) {
+                    uint32_t xw[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int w = w0 + 32 * u + lane;
+                        xw[u] = w < a.nW ? a.xaff[rq * a.nW + w] : 0u;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int w = w0 + 32 * u + lane;
+                        if (w < a.nW) aff[q * a.nW + w] = xw[u];
+                    }
+                }
                 if (lane == 0) {
-                    ext_n[q] = min(a.extra_count[rq], a.E);
+                    ext_n[q] = ec;
                     ext_n[2 + q] = nx;
                 }
             }
-            __syncwarp();
-            const int64_t gi = sidx;
-            const int U = a.glcnt[gi], m0 = ext_n[2], m1 = ext_n[3];
-            for (int i = lane; i < U; i += 32) {
-                const uint32_t v = a.glist[gi * kGlistCap + i];
-                gl_code[i] = v & 0x3fffffffu;
-                gl_who[i] = (uint8_t)(v >> 30);
+            for (int i0 = 0; i0 < U; i0 += 256) {
+                uint32_t gv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + 32 * u + lane;
+                    gv[u] = i < U ? a.glist[gi * kGlistCap + i] : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + 32 * u + lane;
+                    if (i < U) {
+                        gl_code[i] = gv[u] & 0x3fffffffu;
+                        gl_who[i] = (uint8_t)(gv[u] >> 30);
+                    }
+                }
             }
+            __syncwarp();
+            const int m0 = ext_n[2], m1 = ext_n[3];
             for (int e = lane; e < m0; e += 32) {
                 gl_code[U + e] = 0x80000000u | (uint32_t)e;
                 gl_who[U + e] = 1;
@@ -407,14 +455,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ext_n[5] = U + m0 + m1;
             }
         }
+        // the query blocks' CSR ranges in one round of loads, then their column
+        // lists, eight loads in flight per lane
+        const int64_t pr = lane <= nq ? a.row_ptr[rbase + lane] : 0;
         for (int q = 0; q < nq; ++q) {
-            const int64_t p0 = a.row_ptr[rbase + q], p1 = a.row_ptr[rbase + q + 1];
-            for (int64_t p = p0 + lane; p < p1; p += 32) {
-                const int c = a.col_idx[p];
-                if (c >= 0 && c < a.nKB)
-                    atomicOr(&kept[q * a.nW + (c >> 5)], 1u << (c & 31));
-                else
-                    report(a.status, BSA_DEV_INTERNAL, 1);
+            const int64_t p0 = __shfl_sync(0xffffffffu, pr, q), p1 = __shfl_sync(0xffffffffu, pr, q + 1);
+            for (int64_t pb = p0; pb < p1; pb += 256) {
+                int cv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int64_t p = pb + 32 * u + lane;
+                    cv[u] = p < p1 ? a.col_idx[p] : -2;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int c = cv[u];
+                    if (c == -2) continue;   // past the list
+                    if (c >= 0 && c < a.nKB)
+                        atomicOr(&kept[q * a.nW + (c >> 5)], 1u << (c & 31));
+                    else
+                        report(a.status, BSA_DEV_INTERNAL, 1);
+                }
             }
         }
         __syncwarp();
@@ -431,12 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool is_k = warp == 8;
         if (lane == 0) {
             if (is_k) {
-                prefetch_tmap(&tm_q);
                 prefetch_tmap(&tm_k);
                 if (!dense && a.centroid) prefetch_tmap(&tm_kc);
-                mbar_expect_tx(bar_q, L::kQBytes);
-                for (int dc = 0; dc < D / 64; ++dc)
-                    tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
             } else {
                 prefetch_tmap(&tm_v);
                 if (!dense && a.centroid) prefetch_tmap(&tm_vc);
