@@ -373,75 +373,94 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 8 && !dense) {
         // kept-block bitmasks of the tile's query blocks, from the CSR lists; with
-        // extra tokens also their lists and the blocks they came from
+        // extra tokens also their lists and the blocks they came from.  Two rounds
+        // of loads: the CSR ranges and list lengths, then every list at once.
         for (int w = lane; w < 4 * a.nW; w += 32) kept[w] = 0u;
         if (lane < 8) ext_n[lane] = 0;
-        __syncwarp();
+        int64_t pr = 0;
+        int len = 0;
+        if (lane <= nq) pr = a.row_ptr[rbase + lane];
         if (a.E > 0) {
-            // gathered columns: the union of the query blocks' extra tokens (merged
-            // by glist_kernel, padded to a multiple of 4), then each query block's
-            // modified centroids
-            // list lengths in one round of loads, then the lists, eight loads in
-            // flight per lane
-            const int64_t gi = sidx;
-            int len = 0;
-            if (lane < nq) len = a.xcnt[rbase + lane];
-            else if (lane >= 2 && lane < 2 + nq) len = a.extra_count[rbase + lane - 2];
-            else if (lane == 4) len = a.glcnt[gi];
-            const int U = __shfl_sync(0xffffffffu, len, 4);
-            for (int q = 0; q < nq; ++q) {
-                const int64_t rq = rbase + q;
-                const int nx = min(__shfl_sync(0xffffffffu, len, q), a.Ecap);
-                const int ec = min(__shfl_sync(0xffffffffu, len, 2 + q), a.E);
-                for (int e0 = 0; e0 < nx; e0 += 256) {
-                    float xb[8];
+            if (lane >= 8 && lane < 8 + nq) len = a.xcnt[rbase + lane - 8];
+            else if (lane >= 10 && lane < 10 + nq) len = a.extra_count[rbase + lane - 10];
+            else if (lane == 12) len = a.glcnt[sidx];
+        }
+        const int64_t p0 = __shfl_sync(0xffffffffu, pr, 0), p2 = __shfl_sync(0xffffffffu, pr, nq);
+        const int64_t p1 = nq > 1 ? __shfl_sync(0xffffffffu, pr, 1) : p2;   // query block 1's list starts there
+        const int nx0 = min(__shfl_sync(0xffffffffu, len, 8), a.Ecap);
+        const int nx1 = nq > 1 ? min(__shfl_sync(0xffffffffu, len, 9), a.Ecap) : 0;
+        const int ec0 = min(__shfl_sync(0xffffffffu, len, 10), a.E);
+        const int ec1 = nq > 1 ? min(__shfl_sync(0xffffffffu, len, 11), a.E) : 0;
+        const int U = __shfl_sync(0xffffffffu, len, 12);
+        __syncwarp();
+        // the column lists of both query blocks (contiguous in the CSR), 16 in flight per lane
+        for (int64_t pb = p0; pb < p2; pb += 512) {
+            int cv[16];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int e = e0 + 32 * u + lane;
-                        xb[u] = e < nx ? a.xbias[rq * a.Ecap + e] : 0.f;
-                    }
+            for (int u = 0; u < 16; ++u) {
+                const int64_t p = pb + 32 * u + lane;
+                cv[u] = p < p2 ? a.col_idx[p] : -2;
+            }
+            // the extra-token lists ride along with the first batch
+            float xb[16];
+            uint32_t gv[17];
+            if (a.E > 0 && pb == p0) {
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int e = e0 + 32 * u + lane;
-                        if (e < nx) gl_bias[q * kMaxE + e] = xb[u];
-                    }
+                for (int u = 0; u < 16; ++u) {
+                    const int e = 32 * (u & 7) + lane;
+                    const int q = u >> 3;
+                    xb[u] = e < (q ? nx1 : nx0) ? a.xbias[(rbase + q) * a.Ecap + e] : 0.f;
                 }
-                for (int w0 = 0; w0 < a.nW; w0 += 128) {
-                    uint32_t xw[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int w = w0 + 32 * u + lane;
-                        xw[u] = w < a.nW ? a.xaff[rq * a.nW + w] : 0u;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int w = w0 + 32 * u + lane;
-                        if (w < a.nW) aff[q * a.nW + w] = xw[u];
-                    }
-                }
-                if (lane == 0) {
-                    ext_n[q] = ec;
-                    ext_n[2 + q] = nx;
+                for (int u = 0; u < 17; ++u) {
+                    const int i = 32 * u + lane;
+                    gv[u] = i < U ? a.glist[sidx * kGlistCap + i] : 0u;
                 }
             }
-            for (int i0 = 0; i0 < U; i0 += 256) {
-                uint32_t gv[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + 32 * u + lane;
-                    gv[u] = i < U ? a.glist[gi * kGlistCap + i] : 0u;
+            for (int u = 0; u < 16; ++u) {
+                const int c = cv[u];
+                if (c == -2) continue;   // past the lists
+                const int q = pb + 32 * u + lane < p1 ? 0 : 1;
+                if (c >= 0 && c < a.nKB)
+                    atomicOr(&kept[q * a.nW + (c >> 5)], 1u << (c & 31));
+                else
+                    report(a.status, BSA_DEV_INTERNAL, 1);
+            }
+            if (a.E > 0 && pb == p0) {
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int e = 32 * (u & 7) + lane;
+                    const int q = u >> 3;
+                    if (e < (q ? nx1 : nx0)) gl_bias[q * kMaxE + e] = xb[u];
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int i = i0 + 32 * u + lane;
+                for (int u = 0; u < 17; ++u) {
+                    const int i = 32 * u + lane;
                     if (i < U) {
                         gl_code[i] = gv[u] & 0x3fffffffu;
                         gl_who[i] = (uint8_t)(gv[u] >> 30);
                     }
                 }
             }
-            __syncwarp();
-            const int m0 = ext_n[2], m1 = ext_n[3];
+        }
+        if (a.E > 0) {
+            if (p0 >= p2) {   // no kept block at all: the lists did not ride along
+                for (int q = 0; q < nq; ++q)
+                    for (int e = lane; e < (q ? nx1 : nx0); e += 32)
+                        gl_bias[q * kMaxE + e] = a.xbias[(rbase + q) * a.Ecap + e];
+                for (int i = lane; i < U; i += 32) {
+                    const uint32_t v = a.glist[sidx * kGlistCap + i];
+                    gl_code[i] = v & 0x3fffffffu;
+                    gl_who[i] = (uint8_t)(v >> 30);
+                }
+            }
+            for (int q = 0; q < nq; ++q)
+                for (int w = lane; w < a.nW; w += 32) aff[q * a.nW + w] = a.xaff[(rbase + q) * a.nW + w];
+            // gathered columns: the union of the query blocks' extra tokens (merged
+            // by glist_kernel, padded to a multiple of 4), then each query block's
+            // modified centroids
+            const int m0 = nx0, m1 = nx1;
             for (int e = lane; e < m0; e += 32) {
                 gl_code[U + e] = 0x80000000u | (uint32_t)e;
                 gl_who[U + e] = 1;
@@ -451,31 +470,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 gl_who[U + m0 + e] = 2;
             }
             if (lane == 0) {
+                ext_n[0] = ec0;
+                ext_n[1] = ec1;
+                ext_n[2] = nx0;
+                ext_n[3] = nx1;
                 ext_n[4] = U;
                 ext_n[5] = U + m0 + m1;
-            }
-        }
-        // the query blocks' CSR ranges in one round of loads, then their column
-        // lists, eight loads in flight per lane
-        const int64_t pr = lane <= nq ? a.row_ptr[rbase + lane] : 0;
-        for (int q = 0; q < nq; ++q) {
-            const int64_t p0 = __shfl_sync(0xffffffffu, pr, q), p1 = __shfl_sync(0xffffffffu, pr, q + 1);
-            for (int64_t pb = p0; pb < p1; pb += 256) {
-                int cv[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int64_t p = pb + 32 * u + lane;
-                    cv[u] = p < p1 ? a.col_idx[p] : -2;
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int c = cv[u];
-                    if (c == -2) continue;   // past the list
-                    if (c >= 0 && c < a.nKB)
-                        atomicOr(&kept[q * a.nW + (c >> 5)], 1u << (c & 31));
-                    else
-                        report(a.status, BSA_DEV_INTERNAL, 1);
-                }
             }
         }
         __syncwarp();
