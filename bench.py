@@ -1,17 +1,23 @@
 """Benchmark: one layer of block-sparse "sol-attn" attention per step.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--split heads|replicas] [--impl reference]
 
 A step is the whole hot path on one batch of synthetic inputs already resident
 in HBM: bsa_pool -> bsa_select -> bsa_attention (sparse + centroid + dense
-rows).  Rank 0 prints one JSON line.  Metric: sparse-attention ms per layer
-and dense-equivalent TFLOP/s (4*B*H*N^2*d / layer time); the roofline block
-reports the fine pass (bsa_attention) against the measured bf16 tensor peak on
-the FLOPs it really has to do (kept FLOPs, counted from the CSR of the run).
+rows), the last as bsa_attention_prepare + bsa_attention_run so that the fine
+pass kernel is timed alone.  Rank 0 prints one JSON line.  Metric:
+sparse-attention ms per layer and dense-equivalent TFLOP/s (4*B*H*N^2*d /
+layer time).  The roofline block reports the fine pass (bsa_attention_run)
+against the measured bf16 tensor peak on the FLOPs it really has to do (kept
+FLOPs, counted from the CSR of the run); roofline_select reports pooling and
+selection against the measured HBM copy bandwidth.
 
-Multi-GPU (torchrun): attention is independent per (batch, head), so every
-rank runs its own layer on its own inputs (weak scaling, no collective on the
-data path); the step time is the max over ranks.
+Multi-GPU (torchrun): attention is independent per (batch, head).  The default
+split gives each of the N ranks a contiguous range of the same layer's heads
+(strong scaling: the job is one layer, no collective on the data path; the
+step time is the max over ranks).  --split replicas runs one whole layer per
+rank on its own inputs instead (weak scaling).
 """
 from __future__ import annotations
 
@@ -33,7 +39,7 @@ if ROOT not in sys.path:
 
 from workloads import CONFIGS, make_qkv  # noqa: E402
 
-DEFAULT_CONFIG = "sol_sinks"
+DEFAULT_CONFIG = "long"
 METRIC = "sparse-attn ms/layer & dense-equiv TFLOP/s at N tokens; % roofline (kept FLOPs)"
 UNIT = "TFLOP/s (dense-equivalent)"
 
@@ -71,9 +77,19 @@ def attn_traffic(w):
 
 
 def rank_workload(w, rank: int, world: int):
-    """Weak scaling: every rank runs its own layer of the same shape on its own
-    inputs (heads are independent; no collective on the data path)."""
+    """--split replicas: every rank runs its own layer of the same shape on its
+    own inputs (heads are independent; no collective on the data path)."""
     return w.replace(seed=w.seed + 17 * rank) if world > 1 else w
+
+
+def head_range(H: int, rank: int, world: int):
+    """--split heads: rank's contiguous share [h0, h1) of the layer's H heads
+    (the first H % world ranks take one head more)."""
+    if world > H:
+        raise ValueError(f"{world} ranks for {H} heads: every rank needs at least one head")
+    base, extra = divmod(H, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
 
 
 def max_over_ranks(value: float, pg, device) -> float:
@@ -85,9 +101,25 @@ def max_over_ranks(value: float, pg, device) -> float:
     return float(t)
 
 
-def job_throughput(w, world: int, ms_per_step: float) -> float:
-    """Whole-job dense-equivalent TFLOP/s: all ranks' layers over the slowest rank's time."""
-    return world * dense_equiv_flops(w) / (ms_per_step * 1e-3) / 1e12
+def job_throughput(w, world: int, ms_per_step: float, split: str = "replicas") -> float:
+    """Whole-job dense-equivalent TFLOP/s over the slowest rank's time: all
+    ranks' layers (replicas), or the one layer whose heads the ranks share."""
+    layers = world if split == "replicas" else 1
+    return layers * dense_equiv_flops(w) / (ms_per_step * 1e-3) / 1e12
+
+
+def pool_bytes(w) -> float:
+    """Algorithmic HBM bytes of bsa_pool: Q, K and V read once, the f32 means
+    and the block sizes written once."""
+    s_in = 2 if w.dtype == "bf16" else 4
+    read = 3.0 * w.B * w.N * w.H * w.d * s_in
+    write = (w.nQB + 2 * w.nKB) * w.B * w.H * w.d * 4 + 4 * w.nKB
+    return read + write
+
+
+def select_flops(w) -> float:
+    """Block-score FLOPs of bsa_select: 2*d per (row, key block)."""
+    return 2.0 * w.rows * w.nKB * w.d
 
 
 def dense_equiv_flops(w) -> float:
@@ -267,23 +299,37 @@ def run_reference(args, w, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": _config_json(w, world),
+            "data": "synthetic", "config": _config_json(w, world, "heads" if world > 1 else "replicas", [0, w.H]),
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
                              "sample": cb["sample"]},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def _config_json(w, world):
+def _config_json(w, world, split="replicas", heads=None):
+    par = (f"heads split over {world} ranks (ranges {heads}; no collective)" if split == "heads" and world > 1
+           else f"replicas x{world} (heads independent, no collective)")
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "dtype": w.dtype,
             "method": w.method, "q_block": w.q_block, "k_block": w.k_block,
             "tau": w.tau if w.method == "sol" else None,
             "keep_percent": w.keep_percent if w.method == "sla" else None,
             "prefix_len": w.prefix_len, "dense_rows": list(w.dense_rows), "extra_tokens": w.extra_tokens,
             "centroid": w.centroid, "grid": list(w.grid) if w.grid else None,
-            "parallelism": f"replicas x{world} (heads independent, no collective)",
+            "parallelism": par,
             "l2": "inputs larger than L2 (126 MB); no flush" if 3 * w.B * w.N * w.H * w.d * 2 > 126e6
             else "L2 flushed between steps"}
+
+
+def launches_per_step(w) -> int:
+    """Kernels of ours one step launches: pool 1; select: scores, rows, scan,
+    expand (+ theta, filter, finalize, fallback with extra tokens); attention
+    preparation: bf16 centroids (2), bf16 copies of f32 inputs (3), modified
+    centroids and gather lists (2, extra tokens); fine pass 1 (+ the dense-row
+    merge when dense rows are split over keys)."""
+    dense_split = w.dense_rows[1] > w.dense_rows[0] and w.N > 256 * 64
+    return (1 + 4 + (4 if w.extra_tokens > 0 else 0)
+            + (2 if w.centroid else 0) + (3 if w.dtype == "f32" else 0) + (2 if w.extra_tokens > 0 else 0)
+            + 1 + (1 if dense_split else 0))
 
 
 def main():
@@ -293,6 +339,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--split", default="heads", choices=["heads", "replicas"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--heads", type=int, default=0, help="override H (profiling a smaller case)")
@@ -301,13 +348,19 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = CONFIGS[args.config]
+    w_job = CONFIGS[args.config]
     if args.heads > 0:
-        w = w.replace(H=args.heads)
-    w = rank_workload(w, rank, world)
+        w_job = w_job.replace(H=args.heads)
+    split = args.split if world > 1 else "replicas"
+    if split == "replicas":
+        w_job = rank_workload(w_job, rank, world)
+        h0, h1 = 0, w_job.H
+    else:
+        h0, h1 = head_range(w_job.H, rank, world)
+    w = w_job.replace(H=h1 - h0)              # this rank's share of the work
 
     if args.impl == "reference":
-        run_reference(args, w, rank, world)
+        run_reference(args, w_job, rank, world)
         return
 
     import block_sparse_attention_26_b200 as bsa
@@ -323,7 +376,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
         pg = dist
 
-    q, k, v = make_qkv(w, dev)
+    qf, kf, vf = make_qkv(w_job, dev)
+    # this rank's heads: a strided view of the layer's tensors (same strides)
+    q, k, v = (t[:, :, h0:h1] for t in (qf, kf, vf))
     p = params_for(w, q)
     buf = bsa.Buffers(p, dev)
     out = torch.empty_like(q)
@@ -344,10 +399,14 @@ def main():
                        buf.extra_count, buf.ws, stream)
         if ev:
             ev[2].record(stream)
-        bsa.bsa_attention(p, q, k, v, buf.kbar, buf.vbar, buf.blk_count, buf.row_ptr, buf.col_idx,
-                          buf.extra_idx, buf.extra_count, out, buf.lse, buf.ws, stream)
+        att = (p, q, k, v, buf.kbar, buf.vbar, buf.blk_count, buf.row_ptr, buf.col_idx, buf.extra_idx,
+               buf.extra_count, out, buf.lse, buf.ws, stream)
+        bsa.bsa_attention_prepare(*att)
         if ev:
             ev[3].record(stream)
+        bsa.bsa_attention_run(*att)
+        if ev:
+            ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -357,7 +416,7 @@ def main():
         raise SystemExit(f"device status {status} after warm-up")
     flops_kept = kept_flops(w, buf.row_ptr, buf.col_idx, buf.extra_count)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if pg:
         pg.barrier()
@@ -374,22 +433,22 @@ def main():
     status = bsa.bsa_device_status(buf.ws, stream)
     if status != 0:
         raise SystemExit(f"device status {status} after the timed steps")
-    ph = {"pool": [], "select": [], "attention": []}
-    for e in evs:
-        ph["pool"].append(e[0].elapsed_time(e[1]))
-        ph["select"].append(e[1].elapsed_time(e[2]))
-        ph["attention"].append(e[2].elapsed_time(e[3]))
+    names = ["pool", "select", "attention_prepare", "attention_fine_pass"]
+    ph = {n: [e[i].elapsed_time(e[i + 1]) for e in evs] for i, n in enumerate(names)}
+    ph_ms = {n: statistics.mean(x) for n, x in ph.items()}
+    ph_ms["attention"] = ph_ms["attention_prepare"] + ph_ms["attention_fine_pass"]
     ms_step = total_ms / args.steps
-    attn_ms = statistics.mean(ph["attention"])
 
-    # end to end through the public API with host buffers: H2D of Q/K/V, the
-    # layer, D2H of the output, every step
+    # end to end through the public API with host buffers: H2D of this rank's
+    # Q/K/V heads, the layer, D2H of the output, every step
     e2e = None
     if args.e2e_steps > 0:
-        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hq, hk, hv = (t.contiguous().cpu().pin_memory() for t in (q, k, v))
         hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dq, dk, dv = torch.empty_like(hq, device=dev), torch.empty_like(hk, device=dev), torch.empty_like(hv, device=dev)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if pg:
+            pg.barrier()
         for i in range(args.e2e_steps + 1):
             if i == 1:
                 torch.cuda.synchronize(dev)
@@ -403,45 +462,50 @@ def main():
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps, pg, dev)
         nbytes = q.numel() * q.element_size()
-        e2e = {"value": job_throughput(w, world, e2e_ms), "unit": UNIT,
+        e2e = {"value": job_throughput(w_job, world, e2e_ms, split), "unit": UNIT,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms}
         del hq, hk, hv, hout, dq, dk, dv
 
     peaks, peak_src = _peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    achieved = flops_kept / (attn_ms * 1e-3) / 1e12
-    # pool 1; select: scores, rows, scan, expand; attention: fine-pass kernel, plus
-    # the dense-row merge when dense rows are split, bf16 centroids (2), bf16 inputs (3)
-    dense_split = w.dense_rows[1] > w.dense_rows[0] and w.N > 256 * 64
-    launches_per_step = (1 + 4 + 1 + (1 if dense_split else 0) + (2 if w.centroid else 0)
-                         + (3 if w.dtype == "f32" else 0)
-                         + (6 if w.extra_tokens > 0 else 0))   # theta, filter, finalize, fallback, modcent, glist
+    peak = float(peaks.get("bf16_tflops"))
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+    hbm = float(peaks.get("hbm_gbs"))
+    fine_ms = ph_ms["attention_fine_pass"]
+    achieved = flops_kept / (fine_ms * 1e-3) / 1e12
+    pool_gbs = pool_bytes(w) / (ph_ms["pool"] * 1e-3) / 1e9
+    ps_gbs = pool_bytes(w) / ((ph_ms["pool"] + ph_ms["select"]) * 1e-3) / 1e9
     line = {
         "metric": METRIC,
-        "value": job_throughput(w, world, ms_step),
+        "value": job_throughput(w_job, world, ms_step, split),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if split == "heads" and world > 1 else "weak",
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic (smooth Gaussian-filtered fields + noise, seeded)",
-        "config": _config_json(w, world),
+        "config": _config_json(w_job, world, split, [h0, h1]),
         "ms_per_layer": ms_step,
-        "phases_ms": {k2: statistics.mean(v2) for k2, v2 in ph.items()},
+        "phases_ms": ph_ms,
         "kept_tflop": flops_kept / 1e12,
         "dense_equiv_tflop": dense_equiv_flops(w) / 1e12,
         "kept_fraction_of_dense": flops_kept / dense_equiv_flops(w),
-        "roofline": {"bound": "tensor", "kernel": "bsa_attention (fine pass: sparse + centroid + dense rows)",
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel (bsa_attention_run: sparse + centroid + dense rows)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "peak_source": f"{peak_src} bf16_tflops (burst: the kernel runs inside a sub-second step)",
+                     "frac_of_sustained": achieved / peak_sus,
                      "traffic": attn_traffic(w),
                      "traffic_unit": "bytes per launch (ncu dram read+write, scaled from a 4-head capture)"},
+        "roofline_select": {"bound": "hbm", "peak": hbm, "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs",
+                            "pool_bytes": pool_bytes(w), "pool_achieved": pool_gbs, "pool_frac": pool_gbs / hbm,
+                            "pool_plus_select_achieved": ps_gbs, "pool_plus_select_frac": ps_gbs / hbm,
+                            "select_flop": select_flops(w),
+                            "select_tflops": select_flops(w) / (ph_ms["select"] * 1e-3) / 1e12},
         "extra_tokens_per_row": (float(buf.extra_count.float().mean()) if buf.extra_count is not None else 0.0),
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step(w) * args.steps,
         "clocks": clocks.summary(),
         "e2e": e2e,
     }

@@ -62,6 +62,9 @@ def _load() -> ctypes.CDLL:
     lib.bsa_select.argtypes = [PP, P, P, P, P, P, I64, P, P, P, P, SZ, P]
     lib.bsa_select_static.argtypes = [PP, P, P, P, P, I64, P, P]
     lib.bsa_attention.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+    lib.bsa_attention_prepare.argtypes = lib.bsa_attention.argtypes
+    lib.bsa_attention_run.argtypes = lib.bsa_attention.argtypes
+    lib.bsa_selftest_bounded_wait.argtypes = [P, I64, P]
     lib.bsa_dense_ref_rows.argtypes = [PP, P, P, P, I32, I32, P, P, P, SZ, P]
     lib.bsa_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
     lib.bsa_status_string.argtypes = [I32]
@@ -69,7 +72,8 @@ def _load() -> ctypes.CDLL:
     lib.bsa_last_error.argtypes = []
     lib.bsa_last_error.restype = ctypes.c_char_p
     for f in ("bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_select_static", "bsa_attention",
-              "bsa_dense_ref_rows", "bsa_device_status"):
+              "bsa_attention_prepare", "bsa_attention_run", "bsa_dense_ref_rows", "bsa_device_status",
+              "bsa_selftest_bounded_wait"):
         getattr(lib, f).restype = I32
     return lib
 
@@ -77,7 +81,8 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 
 EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_select_static",
-            "bsa_attention", "bsa_dense_ref_rows", "bsa_device_status", "bsa_status_string", "bsa_last_error")
+            "bsa_attention", "bsa_attention_prepare", "bsa_attention_run", "bsa_dense_ref_rows",
+            "bsa_device_status", "bsa_selftest_bounded_wait", "bsa_status_string", "bsa_last_error")
 
 
 def _check(status: int, where: str):
@@ -171,6 +176,26 @@ def bsa_attention(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra_idx
                              _ptr(blk_count), _ptr(row_ptr), _ptr(col_idx), _ptr(extra_idx),
                              _ptr(extra_count), _ptr(out), _ptr(lse), _ptr(ws),
                              ws.numel() * ws.element_size(), _stream(stream)), "bsa_attention")
+
+
+def bsa_attention_prepare(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra_idx, extra_count, out,
+                          lse, ws, stream=None):
+    _check(lib.bsa_attention_prepare(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vbar),
+                                     _ptr(blk_count), _ptr(row_ptr), _ptr(col_idx), _ptr(extra_idx),
+                                     _ptr(extra_count), _ptr(out), _ptr(lse), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "bsa_attention_prepare")
+
+
+def bsa_attention_run(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra_idx, extra_count, out,
+                      lse, ws, stream=None):
+    _check(lib.bsa_attention_run(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(kbar), _ptr(vbar),
+                                 _ptr(blk_count), _ptr(row_ptr), _ptr(col_idx), _ptr(extra_idx),
+                                 _ptr(extra_count), _ptr(out), _ptr(lse), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "bsa_attention_run")
+
+
+def bsa_selftest_bounded_wait(ws, cycles: int, stream=None):
+    _check(lib.bsa_selftest_bounded_wait(_ptr(ws), int(cycles), _stream(stream)), "bsa_selftest_bounded_wait")
 
 
 def bsa_dense_ref_rows(p, q, k, v, row_begin, row_end, out, lse, ws, stream=None):

@@ -1432,8 +1432,9 @@ int dense_split_for(const Dims &D, int nrows, int64_t max_partials)
 {
     if (nrows <= 0) return 1;
     const int64_t tiles = (int64_t)D.B * D.H * ceil_div(nrows, kM);
-    if (tiles >= 2 * 148) return 1;
-    int split = (int)std::min<int64_t>(ceil_div(D.nKB, 256), ceil_div(2 * 148, tiles));
+    const int64_t fill = 2 * (int64_t)sm_count();
+    if (tiles >= fill) return 1;
+    int split = (int)std::min<int64_t>(ceil_div(D.nKB, 256), ceil_div(fill, tiles));
     split = std::max(1, split);
     while (split > 1 && tiles * split > max_partials) --split;
     return split;
@@ -1449,21 +1450,28 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
                              const void *v, const float *kbar, const float *vbar,
                              const int64_t *row_ptr, const int32_t *col_idx, const int32_t *extra_idx,
                              const int32_t *extra_count, void *out, float *lse, int dense_only,
-                             int row_begin, int row_end, char *ws, const WsLayout &L, cudaStream_t st)
+                             int row_begin, int row_end, char *ws, const WsLayout &L, cudaStream_t st,
+                             int phase)
 {
+    // phase: 0 = everything, 1 = only the preparation kernels (bf16 copies,
+    // centroids, modified centroids, gather lists), 2 = only the fine pass
+    // (and the dense-row merge), which reads what phase 1 wrote.
+    const bool prep = phase != 2, run = phase != 1;
     const int BH = D.B * D.H;
     int64_t sb = p.stride_b, sn = p.stride_n, sh = p.stride_h;
     const void *q16 = q, *k16 = k, *v16 = v;
     if (p.dtype == BSA_DT_F32) {
         // the tensor cores take bf16 operands: round the f32 inputs once
         const int64_t n = (int64_t)D.B * D.N * D.H * D.d;
-        const unsigned g = (unsigned)std::min<int64_t>(ceil_div(n, 256), 148 * 16);
+        const unsigned g = (unsigned)std::min<int64_t>(ceil_div(n, 256), (int64_t)sm_count() * 16);
         __nv_bfloat16 *dq = reinterpret_cast<__nv_bfloat16 *>(ws + L.q16);
         __nv_bfloat16 *dk = reinterpret_cast<__nv_bfloat16 *>(ws + L.k16);
         __nv_bfloat16 *dv = reinterpret_cast<__nv_bfloat16 *>(ws + L.v16);
-        inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(q), dq, D.B, D.N, D.H, D.d, sb, sn, sh);
-        inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(k), dk, D.B, D.N, D.H, D.d, sb, sn, sh);
-        inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(v), dv, D.B, D.N, D.H, D.d, sb, sn, sh);
+        if (prep) {
+            inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(q), dq, D.B, D.N, D.H, D.d, sb, sn, sh);
+            inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(k), dk, D.B, D.N, D.H, D.d, sb, sn, sh);
+            inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(v), dv, D.B, D.N, D.H, D.d, sb, sn, sh);
+        }
         q16 = dq;
         k16 = dk;
         v16 = dv;
@@ -1474,9 +1482,9 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     __nv_bfloat16 *kc = reinterpret_cast<__nv_bfloat16 *>(ws + L.kc16);
     __nv_bfloat16 *vc = reinterpret_cast<__nv_bfloat16 *>(ws + L.vc16);
     const bool use_cent = !dense_only && p.centroid;
-    if (use_cent) {
+    if (use_cent && prep) {
         const int64_t n = (int64_t)BH * D.nKB * D.d;
-        const unsigned g = (unsigned)std::min<int64_t>(ceil_div(n, 256), 148 * 8);
+        const unsigned g = (unsigned)std::min<int64_t>(ceil_div(n, 256), (int64_t)sm_count() * 8);
         to_bf16_kernel<<<g, 256, 0, st>>>(kbar, kc, n);
         to_bf16_kernel<<<g, 256, 0, st>>>(vbar, vc, n);
     }
@@ -1525,12 +1533,12 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     a.xbias = reinterpret_cast<const float *>(ws + L.xbias);
     a.xcnt = reinterpret_cast<const int32_t *>(ws + L.xcnt);
     a.xaff = reinterpret_cast<const uint32_t *>(ws + L.xaff);
-    if (a.E > 0) {
+    if (a.E > 0 && p.dtype != BSA_DT_BF16) {
         // the gathers read rows through the input strides
-        if (p.dtype != BSA_DT_BF16) {
-            set_error("extra tokens need bf16 inputs");
-            return cudaErrorInvalidValue;
-        }
+        set_error("extra tokens need bf16 inputs");
+        return cudaErrorInvalidValue;
+    }
+    if (a.E > 0 && prep) {
         auto mc = D.d == 128 ? modcent_kernel<4> : modcent_kernel<2>;
         mc<<<(unsigned)ceil_div(D.rows, 8), 256, 0, st>>>(
             extra_idx, extra_count, kbar, vbar, static_cast<const __nv_bfloat16 *>(k),
@@ -1557,7 +1565,7 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     a.part_o = reinterpret_cast<float *>(ws + L.part_o);
     a.part_ml = reinterpret_cast<float *>(ws + L.part_ml);
     const int64_t items = (int64_t)BH * (a.n_dense * (int64_t)a.dense_split + a.n_sparse);
-    if (items == 0) return cudaSuccess;
+    if (items == 0 || !run) return cudaGetLastError();
     // gather maps: token rows of K and V as one 2-D array when the strides allow it
     // (the row pitch min(sn, sh) divides every stride and holds a whole row), and the
     // modified centroids [rows x Ecap, d]

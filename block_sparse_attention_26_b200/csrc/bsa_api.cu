@@ -7,7 +7,9 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 
+#include "bsa_device.cuh"
 #include "bsa_internal.h"
 
 namespace bsa {
@@ -20,6 +22,21 @@ void set_error(const char *fmt, ...)
     va_start(ap, fmt);
     vsnprintf(g_err, sizeof g_err, fmt, ap);
     va_end(ap);
+}
+
+int sm_count()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
 }
 
 Dims dims_of(const bsa_params &p)
@@ -76,7 +93,7 @@ WsLayout ws_layout(const bsa_params &p)
     L.ex_buf = take(ex ? (size_t)D.rows * extra_buffer_capacity() * 8 : 0);
     L.ex_cnt = take(ex ? (size_t)D.rows * 4 : 0);
     L.ex_ovf = take(ex ? (size_t)(D.rows + 1) * 4 : 0);
-    L.ex_scratch = take(ex ? (size_t)148 * D.N * 4 : 0);
+    L.ex_scratch = take(ex ? (size_t)fallback_ctas() * D.N * 4 : 0);
     L.part_tiles = dense_partial_tiles(D, p.dense_row_end - p.dense_row_begin);
     L.part_o = take((size_t)L.part_tiles * 128 * D.d * sizeof(float));
     L.part_ml = take((size_t)L.part_tiles * 128 * 2 * sizeof(float));
@@ -259,10 +276,14 @@ bsa_status bsa_select_static(const bsa_params *p, const float *qbar, const float
                      "bsa_select_static");
 }
 
-bsa_status bsa_attention(const bsa_params *p, const void *q, const void *k, const void *v, const float *kbar,
-                         const float *vbar, const int32_t *blk_count, const int64_t *row_ptr,
-                         const int32_t *col_idx, const int32_t *extra_idx, const int32_t *extra_count,
-                         void *out, float *lse, void *ws, size_t ws_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+bsa_status attention_call(const bsa_params *p, const void *q, const void *k, const void *v, const float *kbar,
+                          const float *vbar, const int32_t *blk_count, const int64_t *row_ptr,
+                          const int32_t *col_idx, const int32_t *extra_idx, const int32_t *extra_count,
+                          void *out, float *lse, void *ws, size_t ws_bytes, void *stream, int phase)
 {
     g_err[0] = 0;
     TRY(check_params(p));
@@ -287,8 +308,65 @@ bsa_status bsa_attention(const bsa_params *p, const void *q, const void *k, cons
     const WsLayout L = ws_layout(*p);
     return from_cuda(launch_attention(*p, D, q, k, v, kbar, vbar, row_ptr, col_idx, extra_idx, extra_count,
                                       out, lse, 0, p->dense_row_begin, p->dense_row_end,
-                                      static_cast<char *>(ws), L, (cudaStream_t)stream),
-                     "bsa_attention");
+                                      static_cast<char *>(ws), L, (cudaStream_t)stream, phase),
+                     phase == 1 ? "bsa_attention_prepare" : phase == 2 ? "bsa_attention_run" : "bsa_attention");
+}
+
+// One warp waits, with a limit of `cycles`, on an mbarrier nothing arrives on;
+// the bounded wait gives up, records BSA_DEV_TIMEOUT and the kernel returns.
+__global__ void bounded_wait_kernel(int32_t *status, long long cycles)
+{
+    __shared__ uint64_t bar;
+    __shared__ int32_t abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    mbar_wait_for(&bar, 0, &abort_flag, status, 0x5e1f, cycles);
+}
+
+}  // namespace
+
+extern "C" {
+
+bsa_status bsa_attention(const bsa_params *p, const void *q, const void *k, const void *v, const float *kbar,
+                         const float *vbar, const int32_t *blk_count, const int64_t *row_ptr,
+                         const int32_t *col_idx, const int32_t *extra_idx, const int32_t *extra_count,
+                         void *out, float *lse, void *ws, size_t ws_bytes, void *stream)
+{
+    return attention_call(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra_idx, extra_count, out, lse,
+                          ws, ws_bytes, stream, 0);
+}
+
+bsa_status bsa_attention_prepare(const bsa_params *p, const void *q, const void *k, const void *v,
+                                 const float *kbar, const float *vbar, const int32_t *blk_count,
+                                 const int64_t *row_ptr, const int32_t *col_idx, const int32_t *extra_idx,
+                                 const int32_t *extra_count, void *out, float *lse, void *ws, size_t ws_bytes,
+                                 void *stream)
+{
+    return attention_call(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra_idx, extra_count, out, lse,
+                          ws, ws_bytes, stream, 1);
+}
+
+bsa_status bsa_attention_run(const bsa_params *p, const void *q, const void *k, const void *v, const float *kbar,
+                             const float *vbar, const int32_t *blk_count, const int64_t *row_ptr,
+                             const int32_t *col_idx, const int32_t *extra_idx, const int32_t *extra_count,
+                             void *out, float *lse, void *ws, size_t ws_bytes, void *stream)
+{
+    return attention_call(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra_idx, extra_count, out, lse,
+                          ws, ws_bytes, stream, 2);
+}
+
+bsa_status bsa_selftest_bounded_wait(void *ws, int64_t cycles, void *stream)
+{
+    g_err[0] = 0;
+    if (ws == nullptr) FAIL(BSA_ERR_INVALID_ARG, "ws is NULL");
+    if (!aligned16(ws)) FAIL(BSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    if (cycles < 1 || cycles > 2000000000LL) FAIL(BSA_ERR_INVALID_ARG, "cycles outside [1, 2e9]");
+    bounded_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(static_cast<int32_t *>(ws), (long long)cycles);
+    return from_cuda(cudaGetLastError(), "bsa_selftest_bounded_wait");
 }
 
 bsa_status bsa_dense_ref_rows(const bsa_params *p, const void *q, const void *k, const void *v,

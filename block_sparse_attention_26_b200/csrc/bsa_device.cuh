@@ -95,20 +95,26 @@ constexpr long long kWaitCycles = 2000000000LL;
 // Wait for completion of the phase with the given parity.  Returns false
 // (after recording a timeout) if it does not complete within kWaitCycles or if
 // another warp of the CTA already gave up (*abort != 0).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int32_t *abort,
-                                          int32_t *status, int32_t where)
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int32_t *abort,
+                                              int32_t *status, int32_t where, long long limit)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             *abort = 1;
             report(status, BSA_DEV_TIMEOUT, where);
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int32_t *abort,
+                                          int32_t *status, int32_t where)
+{
+    return mbar_wait_for(bar, parity, abort, status, where, kWaitCycles);
 }
 
 // ------------------------------------------------------------------ TMA

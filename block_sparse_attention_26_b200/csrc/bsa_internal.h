@@ -11,6 +11,12 @@ namespace bsa {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Streaming multiprocessors of the current device (looked up once per device;
+// 148 on a B200).  Grids that should cover the whole GPU are sized from it.
+int sm_count();
+// CTAs of the extra-token fallback pass (one scratch row of N keys each).
+inline int fallback_ctas() { return sm_count(); }
+
 // entries per fine-pass tile of the extra-token union: two lists of at most 256,
 // padded to a multiple of 4
 constexpr int kGlistCap = 2 * 256 + 4;
@@ -47,7 +53,7 @@ struct WsLayout {
     size_t ex_buf;         // [rows, 1024] u64 surviving (score, token) pairs
     size_t ex_cnt;         // [rows] i32 survivors per row
     size_t ex_ovf;         // [1 + rows] i32 overflowed rows
-    size_t ex_scratch;     // [148, N] u32 fallback keys
+    size_t ex_scratch;     // [fallback_ctas(), N] u32 fallback keys
     size_t part_o;         // [part_tiles, 128, d] f32 dense-row partial outputs
     size_t part_ml;        // [part_tiles, 128, 2] f32 dense-row partial (max, sum)
     int64_t part_tiles;    // capacity of the partial buffers, in 128-row tiles
@@ -74,7 +80,7 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
                              const int64_t *row_ptr, const int32_t *col_idx, const int32_t *extra_idx,
                              const int32_t *extra_count, void *out, float *lse, int dense_only,
                              int row_begin, int row_end, char *ws, const WsLayout &L,
-                             cudaStream_t st);
+                             cudaStream_t st, int phase = 0);
 
 // Selection with the library's static scratch array instead of a workspace.
 bool static_select_layout(const bsa_params &p, WsLayout *L, size_t *need);

@@ -871,7 +871,7 @@ cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, 
     }
     if (e != cudaSuccess) return e;
     finalize_kernel<<<g8, 256, 0, st>>>(a);
-    fallback_kernel<<<148, 256, 0, st>>>(a);
+    fallback_kernel<<<(unsigned)fallback_ctas(), 256, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -353,24 +353,61 @@ static __device__ __align__(256) unsigned char g_select_scratch[kStaticScratchBy
 namespace {
 
 constexpr int kMaxDevices = 64;
-std::atomic<char *> g_static_base[kMaxDevices];
+
+// The array's device address belongs to the module as loaded into one CUDA
+// context; after a device reset the module is loaded again, possibly at
+// another address.  Each device's entry therefore remembers the context it was
+// looked up in and is looked up again when the current context differs.
+struct StaticBase {
+    std::atomic<void *> ctx{nullptr};
+    std::atomic<char *> base{nullptr};
+};
+StaticBase g_static_base[kMaxDevices];
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current_fn()
+{
+    static std::atomic<CtxGetCurrentFn> fn{nullptr};
+    CtxGetCurrentFn f = fn.load(std::memory_order_acquire);
+    if (f == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            f = reinterpret_cast<CtxGetCurrentFn>(p);
+            fn.store(f, std::memory_order_release);
+        }
+    }
+    return f;
+}
 
 // Device address of g_select_scratch on the current device (looked up once per
-// device; the host-side symbol is only a stand-in and must never be passed to
-// a kernel).
+// device and context; the host-side symbol is only a stand-in and must never
+// be passed to a kernel).
 cudaError_t static_scratch(char **out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    char *p = g_static_base[dev].load(std::memory_order_acquire);
-    if (p == nullptr) {
+    CtxGetCurrentFn get = ctx_get_current_fn();
+    if (get == nullptr) return cudaErrorDeviceUninitialized;
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    StaticBase &slot = g_static_base[dev];
+    char *p = slot.base.load(std::memory_order_acquire);
+    if (ctx == nullptr || p == nullptr || slot.ctx.load(std::memory_order_acquire) != (void *)ctx) {
+        // (the lookup also makes the device's primary context current when
+        // this thread has none yet)
         void *addr = nullptr;
         e = cudaGetSymbolAddress(&addr, g_select_scratch);
         if (e != cudaSuccess) return e;
+        if (ctx == nullptr && (get(&ctx) != CUDA_SUCCESS || ctx == nullptr)) return cudaErrorDeviceUninitialized;
         p = static_cast<char *>(addr);
-        g_static_base[dev].store(p, std::memory_order_release);
+        slot.base.store(nullptr, std::memory_order_release);
+        slot.ctx.store((void *)ctx, std::memory_order_release);
+        slot.base.store(p, std::memory_order_release);
     }
     *out = p;
     return cudaSuccess;

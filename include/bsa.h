@@ -124,6 +124,9 @@ BSA_API bsa_status bsa_pool(const bsa_params *p, const void *q, const void *k, c
  *   extra_idx   : out [rows, E] int32 extra tokens, ascending, -1 padded (NULL if E == 0).
  *   extra_count : out [rows] int32 (NULL if E == 0).
  *   ws, ws_bytes: workspace of at least bsa_workspace_size() bytes.
+ * A query block whose every row lies in [dense_row_begin, dense_row_end) gets
+ * no extra tokens (extra_count 0): those rows are computed densely by
+ * bsa_attention and never read the list.
  * Scores are computed in fp64 and rounded to f32 (S = fl32(qbar.kbar / sqrt d));
  * row mean and population std are taken in fp64 over all nKB scores;
  * thr = fl32(mean + tau * std); block b is kept iff S_b > thr.  If the total
@@ -146,6 +149,10 @@ BSA_API bsa_status bsa_select(const bsa_params *p, const float *qbar, const floa
  *   BSA_ERR_CAPACITY before anything is launched.
  *   The first call on a device looks the array's device address up (one
  *   cudaGetSymbolAddress); make that first call before any stream capture.
+ *   The address is remembered per device together with the CUDA context it
+ *   belongs to, and looked up again when a call finds another context current
+ *   (after a device reset the module, and the array, may sit elsewhere); the
+ *   contents do not survive such a reset.
  *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   All calls share the one array: calls whose work overlaps on the GPU (on
  *   different streams) race; serialise them.  The array keeps the last call's
@@ -174,6 +181,24 @@ BSA_API bsa_status bsa_attention(const bsa_params *p, const void *q, const void 
                          const int32_t *extra_idx, const int32_t *extra_count,
                          void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
 
+/* bsa_attention in two calls on the same stream, with the same arguments:
+ * bsa_attention_prepare launches the preparation kernels (bf16 copies of f32
+ * inputs, bf16 centroids, the modified centroids of blocks that gave extra
+ * tokens and the per-tile extra-token lists, all written to the workspace);
+ * bsa_attention_run then launches the fine pass itself (and the dense-row
+ * merge), reading them.  prepare followed by run is exactly bsa_attention;
+ * the split lets a caller overlap or time the two parts. */
+BSA_API bsa_status bsa_attention_prepare(const bsa_params *p, const void *q, const void *k, const void *v,
+                                 const float *kbar, const float *vbar, const int32_t *blk_count,
+                                 const int64_t *row_ptr, const int32_t *col_idx,
+                                 const int32_t *extra_idx, const int32_t *extra_count,
+                                 void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+BSA_API bsa_status bsa_attention_run(const bsa_params *p, const void *q, const void *k, const void *v,
+                             const float *kbar, const float *vbar, const int32_t *blk_count,
+                             const int64_t *row_ptr, const int32_t *col_idx,
+                             const int32_t *extra_idx, const int32_t *extra_count,
+                             void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
 /* Step 4, dense rows ([DOC] sink_conditioning = exact_kv_and_rows: designated
  * query rows attend densely): rows [row_begin, row_end) of every (b, h) attend
  * to all N keys; writes those rows of out (and lse, if not NULL). */
@@ -185,6 +210,14 @@ BSA_API bsa_status bsa_dense_ref_rows(const bsa_params *p, const void *q, const 
  * last call (BSA_OK if none) in *device_status, and clear it.  The return value
  * is BSA_ERR_CUDA if the synchronisation itself failed. */
 BSA_API bsa_status bsa_device_status(void *ws, void *stream, int32_t *device_status);
+
+/* Self-test of the kernels' bounded waits (not a step of the method): one warp
+ * waits on an mbarrier that nothing ever arrives on, with a limit of `cycles`
+ * SM clock cycles (1 .. 2e9; the pipelines use about one second).  The wait
+ * gives up, writes BSA_ERR_DEVICE's timeout code 7 into the status word of
+ * `ws` (read it with bsa_device_status) and the kernel returns; nothing traps
+ * and the context stays usable. */
+BSA_API bsa_status bsa_selftest_bounded_wait(void *ws, int64_t cycles, void *stream);
 
 /* Static description of a status code. */
 BSA_API const char *bsa_status_string(bsa_status s);

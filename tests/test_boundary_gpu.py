@@ -1,0 +1,66 @@
+"""Boundary behaviour on the GPU: the split form of the fine-pass entry point,
+and the kernels' bounded waits.
+
+bsa_attention_prepare followed by bsa_attention_run must give, bit for bit,
+what bsa_attention gives.  The bounded-wait self-test makes one wait run out
+(an mbarrier nothing arrives on, a short limit): the kernel must return on its
+own, report code 7 (timeout) through the workspace status word, and leave the
+context usable for the next launch.
+"""
+import pytest
+import torch
+
+import block_sparse_attention_26_b200 as bsa
+from workloads import Workload, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    Workload("split_sinks_extra", B=1, H=2, N=2120, d=128, dtype="bf16", method="sol", q_block=64, k_block=64,
+             tau=1.3, prefix_len=200, dense_rows=(72, 200), extra_tokens=64, grid=(3, 16, 40), seed=61),
+    Workload("split_f32", B=1, H=2, N=1024, d=64, dtype="f32", method="sol", q_block=64, k_block=64, tau=1.0,
+             seed=62),
+    Workload("split_sla", B=1, H=2, N=2880, d=128, dtype="bf16", method="sla", q_block=128, k_block=64,
+             keep_percent=15.0, centroid=0, grid=(4, 24, 30), seed=63),
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_prepare_then_run_equals_attention(w):
+    q, k, v = (t.cuda() for t in make_qkv(w, "cpu"))
+    p = bsa.params_for(w, q)
+    buf = bsa.Buffers(p, q.device)
+    bsa.bsa_pool(p, q, k, v, buf.qbar, buf.kbar, buf.vbar, buf.blk_count)
+    bsa.bsa_select(p, buf.qbar, buf.kbar, k, buf.row_ptr, buf.col_idx, buf.kept_count, buf.extra_idx,
+                   buf.extra_count, buf.ws)
+    args = (buf.kbar, buf.vbar, buf.blk_count, buf.row_ptr, buf.col_idx, buf.extra_idx, buf.extra_count)
+    out_a, out_b = torch.empty_like(q), torch.empty_like(q)
+    lse_a, lse_b = torch.empty_like(buf.lse), torch.empty_like(buf.lse)
+    bsa.bsa_attention(p, q, k, v, *args, out_a, lse_a, buf.ws)
+    bsa.bsa_attention_prepare(p, q, k, v, *args, out_b, lse_b, buf.ws)
+    bsa.bsa_attention_run(p, q, k, v, *args, out_b, lse_b, buf.ws)
+    assert bsa.bsa_device_status(buf.ws) == 0
+    assert torch.equal(out_a, out_b)
+    assert torch.equal(lse_a, lse_b)
+
+
+def test_bounded_wait_times_out_and_reports():
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    bsa.bsa_selftest_bounded_wait(ws, 2_000_000)          # about 1 ms at the B200's clock
+    stop.record()
+    assert bsa.bsa_device_status(ws) == 7                 # BSA_DEV_TIMEOUT
+    assert start.elapsed_time(stop) < 1000.0
+    assert bsa.bsa_device_status(ws) == 0                 # read-and-clear
+    # the context is still usable
+    x = torch.arange(1000, device="cuda", dtype=torch.float32)
+    assert float(x.sum()) == 499500.0
+
+
+def test_bounded_wait_rejects_bad_limits():
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    with pytest.raises(bsa.BsaError):
+        bsa.bsa_selftest_bounded_wait(ws, 0)
+    with pytest.raises(bsa.BsaError):
+        bsa.bsa_selftest_bounded_wait(ws, 3_000_000_000)

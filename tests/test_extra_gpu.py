@@ -2,10 +2,27 @@
 Built-in Node Documentation", general inputs, extra_tokens) against the CPU
 oracle.
 
-The GPU ranks tokens by tensor-core dot products (fp32 accumulation), the
-oracle by fp64 dot products: the selected sets must agree except for tokens
-whose oracle score lies within a relative 1e-4 of the row's E-th score
-(near-ties at the cut), which are counted.
+Both sides score token j of query block i as qt_i . k_j / sqrt(d) with qt_i the
+pooled query rounded to bf16, so every product qt_c * k_jc is exact in fp32.
+The GPU sums the 128 products on the tensor cores in fp32 (order and rounding
+of the hardware's accumulation unspecified), the oracle in fp64 and rounds the
+scaled sum to fp32.  With A_j = sum_c |qt_c k_jc|, the two scores of a token
+differ by at most
+
+    delta_j = gamma_128 * A_j / sqrt(d) + 2^-24 * |t_j|,
+    gamma_n = n u / (1 - n u),  u = 2^-23
+
+(u = 2^-23 rather than 2^-24 allows the accumulation to truncate instead of
+rounding to nearest; the second term is the oracle's rounding to fp32).  Two
+tokens can therefore trade places only if their oracle scores lie within the
+sum of their deltas: a token in one set and not the other is exempt iff its
+oracle score is within delta_j + delta_max of the row's E-th oracle score t_E,
+delta_max being the largest delta of the row's differing and E-th tokens.
+Exempted tokens are counted and reported.
+
+Query blocks whose rows all run dense get no extra tokens (the design's
+reading R14): bsa_attention replaces those rows by dense attention, which
+never reads the list.
 """
 import math
 
@@ -19,7 +36,11 @@ from workloads import CONFIGS, Workload, make_qkv, sample_heads, sample_query_bl
 
 pytestmark = pytest.mark.gpu
 
-BAND = 1e-4
+U_ACC = 2.0 ** -23
+
+
+def gamma(n: int) -> float:
+    return n * U_ACC / (1.0 - n * U_ACC)
 
 
 def _gpu_select(w, q, k, v):
@@ -43,6 +64,7 @@ def _check_rows(w, res, kc, gpu_idx, gpu_cnt, rows):
     ex, ec, _ = oracle.extra_tokens(res.qbar, oracle.as_raw(kc), res.keep, w.q_block, w.k_block,
                                     w.extra_tokens, rows)
     K = kc.double().numpy()
+    g_d = gamma(w.d)
     exempt = 0
     for n, r in enumerate(rows):
         if _row_all_dense(w, r):
@@ -58,10 +80,19 @@ def _check_rows(w, res, kc, gpu_idx, gpu_cnt, rows):
             continue
         b, h, i = r // (w.H * w.nQB), (r // w.nQB) % w.H, r % w.nQB
         qt = torch.from_numpy(res.qbar[b, h, i]).to(torch.bfloat16).double().numpy()
-        sc = lambda t: float(K[b, t, h] @ qt) / math.sqrt(w.d)
-        t_e = min(sc(t) for t in a)              # the oracle's E-th score
+        rs = math.sqrt(w.d)
+
+        def score(t):   # the oracle's score: fp64 sum, scaled, rounded to fp32
+            return float(np.float32(float(K[b, t, h] @ qt) / rs))
+
+        def delta(t):
+            return g_d * float(np.abs(K[b, t, h] * qt).sum()) / rs + 2.0 ** -24 * abs(score(t))
+
+        e_tok = min(a, key=lambda t: (score(t), -t))          # the oracle's E-th token
+        t_e = score(e_tok)
+        d_max = max(delta(t) for t in list(diff) + [e_tok])
         for t in diff:
-            assert abs(sc(t) - t_e) <= BAND * (1.0 + abs(t_e)), (r, t, sc(t), t_e)
+            assert abs(score(t) - t_e) <= delta(t) + d_max, (r, t, score(t), t_e, delta(t), d_max)
         exempt += len(diff)
     return exempt
 
@@ -85,7 +116,7 @@ def test_extra_tokens_full_size_sampled():
     p, buf = _gpu_select(w, q, k, v)
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     res = oracle.routing(w, oracle.as_raw(qc), oracle.as_raw(kc), oracle.as_raw(vc), with_extra=False)
-    rows = [(0 * w.H + h) * w.nQB + i for h in sample_heads(w)[:2] for i in sample_query_blocks(w, 16)]
+    rows = [(0 * w.H + h) * w.nQB + i for h in sample_heads(w) for i in sample_query_blocks(w, 64)]
     exempt = _check_rows(w, res, kc, buf.extra_idx.cpu().numpy(), buf.extra_count.cpu().numpy(), rows)
     print(f"sol_sinks: {len(rows)} sampled rows, exempted tokens {exempt}")
     assert exempt <= len(rows) * 2
