@@ -26,7 +26,7 @@ BSA_ERR_CUDA = 5
 BSA_ERR_DEVICE = 6
 
 BSA_DT_BF16, BSA_DT_F32 = 0, 1
-BSA_SOL, BSA_SLA = 0, 1
+BSA_SOL, BSA_SLA, BSA_VSA = 0, 1, 2
 
 
 class bsa_params(ctypes.Structure):
@@ -40,7 +40,21 @@ class bsa_params(ctypes.Structure):
         ("prefix_len", ctypes.c_int32),
         ("dense_row_begin", ctypes.c_int32), ("dense_row_end", ctypes.c_int32),
         ("extra_tokens", ctypes.c_int32), ("centroid", ctypes.c_int32),
+        ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+        ("cube_t", ctypes.c_int32), ("cube_h", ctypes.c_int32), ("cube_w", ctypes.c_int32),
     ]
+
+
+class bsa_policy(ctypes.Structure):
+    _fields_ = [
+        ("start_percent", ctypes.c_double), ("end_percent", ctypes.c_double),
+        ("min_tokens", ctypes.c_int32), ("hybrid", ctypes.c_int32),
+        ("hybrid_guard_steps", ctypes.c_int32), ("pad_", ctypes.c_int32),
+        ("dense_blocks", ctypes.c_char_p),
+    ]
+
+
+BSA_RUN_SPARSE, BSA_DENSE_SHORT, BSA_DENSE_BLOCK, BSA_DENSE_HYBRID, BSA_DENSE_WINDOW = 0, 1, 2, 3, 4
 
 
 class BsaError(RuntimeError):
@@ -67,6 +81,11 @@ def _load() -> ctypes.CDLL:
     lib.bsa_selftest_bounded_wait.argtypes = [P, I64, P]
     lib.bsa_dense_ref_rows.argtypes = [PP, P, P, P, I32, I32, P, P, P, SZ, P]
     lib.bsa_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
+    PolP = ctypes.POINTER(bsa_policy)
+    lib.bsa_default_policy.argtypes = [PolP]
+    lib.bsa_default_policy.restype = None
+    lib.bsa_policy_decide.argtypes = [PolP, I32, I32, ctypes.c_double, I32, I32, ctypes.POINTER(I32)]
+    lib.bsa_policy_decide.restype = I32
     lib.bsa_status_string.argtypes = [I32]
     lib.bsa_status_string.restype = ctypes.c_char_p
     lib.bsa_last_error.argtypes = []
@@ -82,7 +101,8 @@ lib = _load()
 
 EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_select_static",
             "bsa_attention", "bsa_attention_prepare", "bsa_attention_run", "bsa_dense_ref_rows",
-            "bsa_device_status", "bsa_selftest_bounded_wait", "bsa_status_string", "bsa_last_error")
+            "bsa_device_status", "bsa_selftest_bounded_wait", "bsa_default_policy", "bsa_policy_decide",
+            "bsa_status_string", "bsa_last_error")
 
 
 def _check(status: int, where: str):
@@ -106,9 +126,10 @@ def _stream(stream) -> ctypes.c_void_p:
 def make_params(q: torch.Tensor, method: str = "sol", *, q_block: Optional[int] = None,
                 tau: float = 1.3, keep_percent: float = 10.0, sink_blocks: int = 1,
                 keep_diag: int = 1, prefix_len: int = 0, dense_rows=(0, 0), extra_tokens: int = 0,
-                centroid: Optional[int] = None) -> bsa_params:
-    """Parameters for a [B, N, H, d] query tensor `q` (strides taken from q)."""
-    m = {"sol": BSA_SOL, "sla": BSA_SLA}[method]
+                centroid: Optional[int] = None, grid=None, cube=(4, 4, 4)) -> bsa_params:
+    """Parameters for a [B, N, H, d] query tensor `q` (strides taken from q).
+    method "vsa" needs `grid` = (T, Hs, Ws) of the tokens after the prefix."""
+    m = {"sol": BSA_SOL, "sla": BSA_SLA, "vsa": BSA_VSA}[method]
     p = bsa_params()
     lib.bsa_default_params(ctypes.byref(p), m)
     B, N, H, d = q.shape
@@ -124,6 +145,11 @@ def make_params(q: torch.Tensor, method: str = "sol", *, q_block: Optional[int] 
     p.extra_tokens = extra_tokens
     if centroid is not None:
         p.centroid = centroid
+    if m == BSA_VSA:
+        if grid is None:
+            raise ValueError("method vsa needs the latent grid (T, Hs, Ws)")
+        p.grid_t, p.grid_h, p.grid_w = grid
+        p.cube_t, p.cube_h, p.cube_w = cube
     return p
 
 
@@ -133,7 +159,8 @@ def params_for(w, q: torch.Tensor) -> bsa_params:
     extra_tokens, centroid) for query tensor `q`."""
     return make_params(q, w.method, q_block=w.q_block, tau=w.tau, keep_percent=w.keep_percent,
                        sink_blocks=w.sink_blocks, keep_diag=w.keep_diag, prefix_len=w.prefix_len,
-                       dense_rows=tuple(w.dense_rows), extra_tokens=w.extra_tokens, centroid=w.centroid)
+                       dense_rows=tuple(w.dense_rows), extra_tokens=w.extra_tokens, centroid=w.centroid,
+                       grid=getattr(w, "grid", None), cube=getattr(w, "cube", (4, 4, 4)))
 
 
 def dims(p: bsa_params):
@@ -211,6 +238,25 @@ def bsa_device_status(ws, stream=None) -> int:
     return code.value
 
 
+def make_policy(start_percent: float = 0.2, end_percent: float = 1.0, min_tokens: int = 12288,
+                hybrid: bool = False, hybrid_guard_steps: int = 1, dense_blocks: str = "") -> bsa_policy:
+    pol = bsa_policy()
+    lib.bsa_default_policy(ctypes.byref(pol))
+    pol.start_percent, pol.end_percent = float(start_percent), float(end_percent)
+    pol.min_tokens, pol.hybrid, pol.hybrid_guard_steps = int(min_tokens), int(bool(hybrid)), int(hybrid_guard_steps)
+    pol._dense_blocks_bytes = dense_blocks.encode()      # kept alive with the struct
+    pol.dense_blocks = pol._dense_blocks_bytes
+    return pol
+
+
+def bsa_policy_decide(pol: bsa_policy, n_tokens: int, block_index: int, progress: float, step: int = -1,
+                      n_steps: int = 0) -> int:
+    out = ctypes.c_int32()
+    _check(lib.bsa_policy_decide(ctypes.byref(pol), int(n_tokens), int(block_index), float(progress), int(step),
+                                 int(n_steps), ctypes.byref(out)), "bsa_policy_decide")
+    return out.value
+
+
 # ------------------------------------------------------------------ buffers
 
 class Buffers:
@@ -236,6 +282,18 @@ class Buffers:
         self.ws = torch.zeros((ws_bytes + 255) // 256 * 256, dtype=torch.uint8, device=device)
         self.lse = torch.empty((p.B, p.H, p.N), dtype=f32, device=device)
         del BH
+
+
+def run_step(p: bsa_params, pol: bsa_policy, q, k, v, out, buf: Buffers, block_index: int, progress: float,
+             step: int = -1, n_steps: int = 0, stream=None, lse: bool = True) -> int:
+    """One attention call under the per-step policy: the sparse hot path, or
+    dense attention over every row; returns the bsa_decision taken."""
+    decision = bsa_policy_decide(pol, p.N, block_index, progress, step, n_steps)
+    if decision == BSA_RUN_SPARSE:
+        run_layer(p, q, k, v, out, buf, stream, lse)
+    else:
+        bsa_dense_ref_rows(p, q, k, v, 0, p.N, out, buf.lse if lse else None, buf.ws, stream)
+    return decision
 
 
 def run_layer(p: bsa_params, q, k, v, out, buf: Buffers, stream=None, lse: bool = True):

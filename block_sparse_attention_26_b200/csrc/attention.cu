@@ -140,7 +140,37 @@ struct AttnArgs {
     int64_t grow_b, grow_n, grow_h;
     const uint32_t *glist;                     // [sparse tiles, kGlistCap] extra-token union per tile
     const int32_t *glcnt;                      // [sparse tiles] its length (a multiple of 4)
+    // cube tiling (vsa): positions are in block order (the prefix's 64-token
+    // blocks, then the grid's cubes); tiles of cubes come through 5-D maps
+    int cube, pre_blocks, P, gH, gW, cT, cH, cW, ncx, ncy;
 };
+
+// Token of block-order position p (identity without cube tiling).
+__device__ __forceinline__ int pos_token(const AttnArgs &a, int p)
+{
+    if (!a.cube) return p;
+    const int blk = p >> 6, t = p & 63;
+    if (blk < a.pre_blocks) return p;
+    const int c = blk - a.pre_blocks;
+    const int cx = c % a.ncx, cy = (c / a.ncx) % a.ncy, ct = c / (a.ncx * a.ncy);
+    const int dx = t % a.cW, dy = (t / a.cW) % a.cH, dt = t / (a.cW * a.cH);
+    return a.P + ((ct * a.cT + dt) * a.gH + cy * a.cH + dy) * a.gW + cx * a.cW + dx;
+}
+
+// 64 rows from block-order position pos through the 4-D map (64-row box) when
+// they are prefix tokens (any pos) or past the end (zeros), else the cube that
+// starts at pos (a multiple of 64) through the 5-D map.
+__device__ __forceinline__ void load_rows64(uint8_t *dst, const AttnArgs &a, const CUtensorMap *m4,
+                                            const CUtensorMap *m5, uint64_t *bar, int dc, int h, int b, int pos)
+{
+    if (pos < a.P || pos >= a.N) {
+        tma_load_4d(dst, m4, bar, dc * 64, h, pos, b);
+    } else {
+        const int c = (pos >> 6) - a.pre_blocks;
+        const int cx = c % a.ncx, cy = (c / a.ncx) % a.ncy, ct = c / (a.ncx * a.ncy);
+        tma_load_5d(dst, m5, bar, dc * 64, h, cx * a.cW, cy * a.cH, ct * a.cT);
+    }
+}
 
 template <int D>
 struct Lay {
@@ -285,7 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
                 const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_gk,
                 const __grid_constant__ CUtensorMap tm_gv, const __grid_constant__ CUtensorMap tm_gxk,
-                const __grid_constant__ CUtensorMap tm_gxv, const AttnArgs a)
+                const __grid_constant__ CUtensorMap tm_gxv, const __grid_constant__ CUtensorMap tm_q5,
+                const __grid_constant__ CUtensorMap tm_k5, const __grid_constant__ CUtensorMap tm_v5,
+                const AttnArgs a)
 {
     using L = Lay<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -364,8 +396,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Q first: its load overlaps the rest of the set-up
         prefetch_tmap(&tm_q);
         mbar_expect_tx(bar_q, L::kQBytes);
-        for (int dc = 0; dc < D / 64; ++dc)
-            tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
+        if (a.cube) {
+            // two 64-row blocks (the map's box is 64 rows in this mode)
+            for (int dc = 0; dc < D / 64; ++dc)
+                for (int half = 0; half < 2; ++half)
+                    load_rows64(sm + L::kOffQ + dc * (kM * 128) + half * (64 * 128), a, &tm_q, &tm_q5, bar_q, dc, h,
+                                b, row0 + 64 * half);
+        } else {
+            for (int dc = 0; dc < D / 64; ++dc)
+                tma_load_4d(sm + L::kOffQ + dc * (kM * 128), &tm_q, bar_q, dc * 64, h, row0, b);
+        }
     }
     if (warp == 9) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -515,13 +555,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const __nv_bfloat16 *src_c = is_k ? a.xk16 : a.xv16;
         int j = 0;
         // half x of the tile lands at row offset 64 x of every channel chunk
+        const CUtensorMap *tm_x5 = is_k ? &tm_k5 : &tm_v5;
         auto load_half = [&](uint8_t *dst, int kind, int blk, uint64_t *bar) {
             for (int dc = 0; dc < D / 64; ++dc) {
                 uint8_t *d = dst + dc * (kTK * 128);
-                if (kind == TILE_EXACT)
-                    tma_load_4d(d, tm_x, bar, dc * 64, h, blk * kBK, b);
-                else
+                if (kind == TILE_EXACT) {
+                    if (a.cube)
+                        load_rows64(d, a, tm_x, tm_x5, bar, dc, h, b, blk * kBK);
+                    else
+                        tma_load_4d(d, tm_x, bar, dc * 64, h, blk * kBK, b);
+                } else {
                     tma_load_3d(d, tm_c, bar, dc * 64, blk * kBK, bh);
+                }
             }
         };
         // row address of a gathered column: an extra token of this head, or a
@@ -1036,7 +1081,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
                     continue;
                 }
-                const int64_t off = (int64_t)b * a.sb + (int64_t)n * a.sn + (int64_t)h * a.sh + cc * 32;
+                const int64_t off = (int64_t)b * a.sb + (int64_t)pos_token(a, n) * a.sn + (int64_t)h * a.sh + cc * 32;
                 if (a.out_f32) {
                     float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + off);
 #pragma unroll
@@ -1056,7 +1101,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pm[0] = lt > 0.f ? m : -INFINITY;
                     pm[1] = lt;
                 } else if (mine && a.lse != nullptr) {
-                    a.lse[(int64_t)bh * a.N + n] = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+                    a.lse[(int64_t)bh * a.N + pos_token(a, n)] =
+                        lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
                 }
             }
         }
@@ -1402,15 +1448,35 @@ bool make_map_rows(CUtensorMap *m, const void *base, int64_t rows, int d, int64_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 cubes of the latent grid that follows a prefix of P tokens (B = 1):
+// [T, Hs, Ws, H, d] seen through the token strides; box = 64 channels x 1 head
+// x cW x cH x cT tokens, i.e. one cube's 64 token rows of 128 bytes, t-major.
+bool make_map_cube(CUtensorMap *m, const void *base, int P, int H, int d, int gT, int gH, int gW, int cT, int cH,
+                   int cW, int64_t sn, int64_t sh)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const __nv_bfloat16 *g0 = static_cast<const __nv_bfloat16 *>(base) + (int64_t)P * sn;
+    cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)gW, (cuuint64_t)gH, (cuuint64_t)gT};
+    cuuint64_t strides[4] = {(cuuint64_t)sh * 2, (cuuint64_t)sn * 2, (cuuint64_t)gW * sn * 2,
+                             (cuuint64_t)gH * gW * sn * 2};
+    cuuint32_t box[5] = {64, 1, (cuuint32_t)cW, (cuuint32_t)cH, (cuuint32_t)cT};
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<__nv_bfloat16 *>(g0), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch_attn_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                const CUtensorMap &tkc, const CUtensorMap &tvc, const CUtensorMap (&tg)[4],
-                               const AttnArgs &a, int64_t items, cudaStream_t st)
+                               const CUtensorMap (&t5)[3], const AttnArgs &a, int64_t items, cudaStream_t st)
 {
     const size_t smem = Lay<D>::bytes(a.nW);
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<D><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, tg[0], tg[1], tg[2], tg[3], a);
+    attn_kernel<D><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, tg[0], tg[1], tg[2], tg[3], t5[0],
+                                                            t5[1], t5[2], a);
     return cudaGetLastError();
 }
 
@@ -1489,14 +1555,37 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
         to_bf16_kernel<<<g, 256, 0, st>>>(vbar, vc, n);
     }
     CUtensorMap tq, tk, tv, tkc, tvc;
-    if (!make_map_bnhd(&tq, q16, D.B, D.N, D.H, D.d, sb, sn, sh, kM) ||
+    if (!make_map_bnhd(&tq, q16, D.B, D.N, D.H, D.d, sb, sn, sh, D.cube ? kBK : kM) ||
         !make_map_bnhd(&tk, k16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) ||
         !make_map_bnhd(&tv, v16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) ||
         !make_map_cent(&tkc, kc, BH, D.nKB, D.d) || !make_map_cent(&tvc, vc, BH, D.nKB, D.d)) {
         set_error("cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)");
         return cudaErrorInvalidValue;
     }
+    CUtensorMap t5[3] = {tq, tk, tv};   // cube maps (unused without cube tiling)
+    if (D.cube) {
+        const int P = p.prefix_len;
+        if (!make_map_cube(&t5[0], q16, P, D.H, D.d, p.grid_t, p.grid_h, p.grid_w, p.cube_t, p.cube_h, p.cube_w, sn,
+                           sh) ||
+            !make_map_cube(&t5[1], k16, P, D.H, D.d, p.grid_t, p.grid_h, p.grid_w, p.cube_t, p.cube_h, p.cube_w, sn,
+                           sh) ||
+            !make_map_cube(&t5[2], v16, P, D.H, D.d, p.grid_t, p.grid_h, p.grid_w, p.cube_t, p.cube_h, p.cube_w, sn,
+                           sh)) {
+            set_error("cuTensorMapEncodeTiled failed for the cube tiles");
+            return cudaErrorInvalidValue;
+        }
+    }
     AttnArgs a;
+    a.cube = D.cube;
+    a.pre_blocks = D.pre_blocks;
+    a.P = p.prefix_len;
+    a.gH = p.grid_h;
+    a.gW = p.grid_w;
+    a.cT = p.cube_t;
+    a.cH = p.cube_h;
+    a.cW = p.cube_w;
+    a.ncx = D.cube ? p.grid_w / p.cube_w : 1;
+    a.ncy = D.cube ? p.grid_h / p.cube_h : 1;
     a.B = D.B;
     a.H = D.H;
     a.N = D.N;
@@ -1594,8 +1683,8 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
             }
         }
     }
-    cudaError_t e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, tg, a, items, st)
-                              : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, tg, a, items, st);
+    cudaError_t e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
+                              : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st);
     if (e != cudaSuccess) return e;
     if (a.n_dense > 0 && a.dense_split > 1) {
         combine_kernel<<<(unsigned)(BH * (int64_t)a.n_dense), kM, 0, st>>>(a, D.d);

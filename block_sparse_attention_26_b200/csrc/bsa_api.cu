@@ -53,6 +53,8 @@ Dims dims_of(const bsa_params &p)
     D.nW = (int)ceil_div(D.nKB, 32);
     D.rows = (int64_t)p.B * p.H * D.nQB;
     D.E = p.extra_tokens;
+    D.cube = p.method == BSA_VSA;
+    D.pre_blocks = D.cube ? p.prefix_len / 64 : 0;
     return D;
 }
 
@@ -67,10 +69,9 @@ WsLayout ws_layout(const bsa_params &p)
         return at;
     };
     const int64_t BH = (int64_t)D.B * D.H;
-    L.status = take(sizeof(int32_t) * 2);
-    L.scores = take((size_t)D.rows * D.nKB * sizeof(float));
-    L.bitmask = take((size_t)D.rows * D.nW * sizeof(uint32_t));
-    L.counts = take((size_t)D.rows * sizeof(int32_t));
+    Taker T;
+    select_regions(p, D, L, T);
+    off = T.off;
     L.kc16 = take((size_t)BH * D.nKB * D.d * 2);
     L.vc16 = take((size_t)BH * D.nKB * D.d * 2);
     const size_t ecap = D.E > 0 ? (size_t)std::min(D.E, D.nKB) : 0;
@@ -121,7 +122,8 @@ bsa_status check_params(const bsa_params *p)
     if (p->B < 1 || p->H < 1 || p->N < 1) FAIL(BSA_ERR_INVALID_ARG, "B, H, N must be >= 1");
     if (p->d != 64 && p->d != 128) FAIL(BSA_ERR_UNSUPPORTED, "d = %d; supported head dims are 64 and 128", p->d);
     if (p->dtype != BSA_DT_BF16 && p->dtype != BSA_DT_F32) FAIL(BSA_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
-    if (p->method != BSA_SOL && p->method != BSA_SLA) FAIL(BSA_ERR_UNSUPPORTED, "unknown method %d", p->method);
+    if (p->method != BSA_SOL && p->method != BSA_SLA && p->method != BSA_VSA)
+        FAIL(BSA_ERR_UNSUPPORTED, "unknown method %d", p->method);
     if (p->k_block != 64) FAIL(BSA_ERR_UNSUPPORTED, "k_block must be 64");
     if (p->q_block != 64 && p->q_block != 128) FAIL(BSA_ERR_UNSUPPORTED, "q_block must be 64 or 128");
     const int64_t align_elems = p->dtype == BSA_DT_BF16 ? 8 : 4;
@@ -131,8 +133,23 @@ bsa_status check_params(const bsa_params *p)
         FAIL(BSA_ERR_INVALID_ARG, "strides must be multiples of %lld elements (16 bytes)", (long long)align_elems);
     if (p->stride_h < p->d) FAIL(BSA_ERR_INVALID_ARG, "stride_h smaller than d would overlap heads");
     if (isnan(p->tau)) FAIL(BSA_ERR_INVALID_ARG, "tau is NaN");
-    if (p->method == BSA_SLA && !(p->keep_percent > 0.0 && p->keep_percent <= 100.0))
+    if (p->method != BSA_SOL && !(p->keep_percent > 0.0 && p->keep_percent <= 100.0))
         FAIL(BSA_ERR_INVALID_ARG, "keep_percent must be in (0, 100]");
+    if (p->method == BSA_VSA) {
+        if (p->q_block != 64) FAIL(BSA_ERR_UNSUPPORTED, "vsa: query cubes hold 64 tokens (q_block 64)");
+        if (p->B != 1) FAIL(BSA_ERR_UNSUPPORTED, "vsa: B must be 1");
+        if (p->cube_t < 1 || p->cube_h < 1 || p->cube_w < 1 || p->cube_t * p->cube_h * p->cube_w != 64)
+            FAIL(BSA_ERR_UNSUPPORTED, "vsa: cube extents must multiply to 64");
+        if (p->grid_t < 1 || p->grid_h < 1 || p->grid_w < 1 || p->grid_t % p->cube_t || p->grid_h % p->cube_h ||
+            p->grid_w % p->cube_w)
+            FAIL(BSA_ERR_UNSUPPORTED, "vsa: every grid extent must be a multiple of its cube extent");
+        if (p->prefix_len % 64) FAIL(BSA_ERR_UNSUPPORTED, "vsa: prefix_len must be a multiple of 64");
+        if ((int64_t)p->prefix_len + (int64_t)p->grid_t * p->grid_h * p->grid_w != p->N)
+            FAIL(BSA_ERR_INVALID_ARG, "vsa: prefix_len + grid_t * grid_h * grid_w must equal N");
+        if (p->dense_row_end > p->prefix_len) FAIL(BSA_ERR_UNSUPPORTED, "vsa: dense rows must lie in the prefix");
+        if (p->centroid) FAIL(BSA_ERR_UNSUPPORTED, "vsa: the fine stage has no centroid term (centroid 0)");
+        if (p->extra_tokens) FAIL(BSA_ERR_UNSUPPORTED, "vsa: extra_tokens is ignored for vsa; pass 0");
+    }
     if (p->sink_blocks < 0) FAIL(BSA_ERR_INVALID_ARG, "sink_blocks < 0");
     if (p->keep_diag != 0 && p->keep_diag != 1) FAIL(BSA_ERR_INVALID_ARG, "keep_diag must be 0 or 1");
     if (p->prefix_len < 0 || p->prefix_len > p->N) FAIL(BSA_ERR_INVALID_ARG, "prefix_len outside [0, N]");
@@ -194,7 +211,10 @@ void bsa_default_params(bsa_params *p, int32_t method)
     p->keep_percent = 10.0;
     p->sink_blocks = 1;
     p->keep_diag = 1;
-    p->centroid = method == BSA_SLA ? 0 : 1;
+    p->centroid = method == BSA_SOL ? 1 : 0;
+    if (method == BSA_VSA) {
+        p->cube_t = p->cube_h = p->cube_w = 4;
+    }
 }
 
 bsa_status bsa_workspace_size(const bsa_params *p, size_t *bytes, int64_t *max_nnz)

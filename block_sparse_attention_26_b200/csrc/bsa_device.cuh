@@ -130,6 +130,17 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// 5-D variant (cube tiles of the latent grid).
+__device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0,
+                                            int c1, int c2, int c3, int c4)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
+
 // 3-D variant.
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0,
                                             int c1, int c2)
@@ -259,6 +270,26 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ misc
+
+// v[e] for a runtime e in [0, 32) without local memory: a 5-level select tree.
+__device__ __forceinline__ uint32_t select32(const uint32_t *v, int e)
+{
+    uint32_t a16[16], a8[8], a4[4], a2[2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a16[i] = (e & 1) ? v[2 * i + 1] : v[2 * i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a8[i] = (e & 2) ? a16[2 * i + 1] : a16[2 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a4[i] = (e & 4) ? a8[2 * i + 1] : a8[2 * i];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) a2[i] = (e & 8) ? a4[2 * i + 1] : a4[2 * i];
+    return (e & 16) ? a2[1] : a2[0];
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {

@@ -22,6 +22,18 @@ inline int fallback_ctas() { return sm_count(); }
 constexpr int kGlistCap = 2 * 256 + 4;
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Certified Sol routing: uncertain blocks listed per row before the exact pass.
+constexpr int kUcap = 128;
+
+// Per-row data of the certified routing (32 bytes): the decide kernel keeps
+// block b iff raw > hi + c |kbar_b| and drops it iff raw < lo - c |kbar_b|
+// (raw = the tensor-core dot product); the definition's threshold lies in
+// [thr_lo, thr_hi]; mode 1 sends the row to the exact path.
+struct RowInfo {
+    float hi, lo, c, thr_lo, thr_hi;
+    int32_t mode, pad0, pad1;
+};
+
 // Derived sizes of one problem.
 struct Dims {
     int B, H, N, d;
@@ -29,6 +41,8 @@ struct Dims {
     int nQB, nKB, nW;      // nW = 32-bit words of a per-row key-block bitmask
     int64_t rows;          // B * H * nQB
     int E;
+    bool cube;             // cube tiling (BSA_VSA): blocks past the prefix are cubes of the grid
+    int pre_blocks;        // 64-token blocks of the prefix that precede the cubes
 };
 
 Dims dims_of(const bsa_params &p);
@@ -39,6 +53,7 @@ struct WsLayout {
     size_t scores;         // [rows, nKB] f32 block scores (select)
     size_t bitmask;        // [rows, nW] u32 kept-block bitmask (select)
     size_t counts;         // [rows] i32 kept counts (select)
+    size_t scan_tmp;       // [ceil(rows / 4096)] i64 per-tile sums of the counts' scan
     size_t kc16, vc16;     // [B*H, nKB, d] bf16 centroids (attention)
     size_t xk16, xv16;     // [rows, min(E, nKB), d] bf16 modified centroids (extra tokens)
     size_t xbias;          // [rows, min(E, nKB)] f32 their log2 token counts
@@ -54,6 +69,20 @@ struct WsLayout {
     size_t ex_cnt;         // [rows] i32 survivors per row
     size_t ex_ovf;         // [1 + rows] i32 overflowed rows
     size_t ex_scratch;     // [fallback_ctas(), N] u32 fallback keys
+    // certified Sol routing (finite tau)
+    size_t r_k16;          // [B*H, nKB, d] bf16 key centroids (the score GEMM's B operand)
+    size_t r_knorm;        // [B*H, nKBp] f32 their norms, rounded up
+    size_t r_knmax;        // [B*H, nKBp / 32] f32 largest norm per 32-block word
+    size_t r_gram;         // [B*H, nsplit, d, d] f64 partial Gram matrices
+    size_t r_ksum;         // [B*H, nsplit, d] f64 partial sums
+    size_t r_cov;          // [B*H, d, d] f64 centred second moments
+    size_t r_hstat;        // [B*H, d + 3] f64 mean key, tr(G)/n, |m|^2, max |kbar|
+    size_t r_info;         // [rows] RowInfo
+    size_t r_ulist;        // [rows, kUcap] i32 blocks left undecided
+    size_t r_ucnt;         // [rows] i32 their count
+    size_t r_fbl;          // [1 + rows] i32 rows for the exact path
+    size_t r_fbs;          // [fallback_ctas(), nKBp] f32 exact scores of one row
+    int r_nsplit;
     size_t part_o;         // [part_tiles, 128, d] f32 dense-row partial outputs
     size_t part_ml;        // [part_tiles, 128, 2] f32 dense-row partial (max, sum)
     int64_t part_tiles;    // capacity of the partial buffers, in 128-row tiles
@@ -61,6 +90,29 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const bsa_params &p);
+
+// Consecutive 256-byte-aligned regions.
+struct Taker {
+    size_t off = 0;
+    size_t take(size_t bytes)
+    {
+        const size_t at = off;
+        off = align_up(off + bytes, 256);
+        return at;
+    }
+};
+
+// Whether Sol selection takes the certified route (a finite tau); key blocks
+// per head padded to a multiple of 128; split count of the key Gram matrix.
+bool certified_route(const bsa_params &p);
+inline int64_t route_nkbp(const Dims &D) { return ceil_div(D.nKB, 128) * 128; }
+int route_nsplit(const Dims &D);
+// The selection's scratch regions (status, scores, bitmask, counts and the
+// certified route's), taken from T in that order.
+void select_regions(const bsa_params &p, const Dims &D, WsLayout &L, Taker &T);
+// Certified Sol routing: bitmask (forced blocks included) and kept counts.
+cudaError_t launch_route(const bsa_params &p, const Dims &D, const float *qbar, const float *kbar, char *ws,
+                         const WsLayout &L, cudaStream_t st);
 
 // Key-chunk split of `nrows` dense rows (1 = no split), limited to max_partials tiles.
 int dense_split_for(const Dims &D, int nrows, int64_t max_partials);

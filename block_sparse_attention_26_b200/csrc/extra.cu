@@ -270,25 +270,6 @@ struct FLay {
     static_assert(bytes <= 232448, "filter tile exceeds the per-block shared memory limit");
 };
 
-// v[e] for a runtime e in [0, 32) without local memory: a 5-level select tree.
-__device__ __forceinline__ uint32_t select32(const uint32_t *v, int e)
-{
-    uint32_t a16[16], a8[8], a4[4], a2[2];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) a16[i] = (e & 1) ? v[2 * i + 1] : v[2 * i];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a8[i] = (e & 2) ? a16[2 * i + 1] : a16[2 * i];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a4[i] = (e & 4) ? a8[2 * i + 1] : a8[2 * i];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) a2[i] = (e & 8) ? a4[2 * i + 1] : a4[2 * i];
-    return (e & 16) ? a2[1] : a2[0];
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // Warps 0-7 read the scores: warp w takes the rows of TMEM lane quarter w & 3
 // and, of each 128-token tile, key block 2t + (w >> 2).  Warp 8 loads K tiles,

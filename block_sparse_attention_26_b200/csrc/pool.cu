@@ -51,7 +51,20 @@ struct PoolArgs {
     int64_t sb, sn, sh;
     int N, H, d;
     int32_t *count;       // written for the key blocks (tensor 1)
+    // cube tiling: blocks past the prefix's pre_blocks are cubes of the grid
+    int cube, pre_blocks, P, gH, gW, cT, cH, cW, ncx, ncy;
 };
+
+// Token of slot t (0..63) of block i: the prefix's own tokens, or the cube's
+// tokens t-major inside the cube, cubes t-major over the grid.
+__device__ __forceinline__ int block_token(const PoolArgs &a, int i, int t)
+{
+    if (i < a.pre_blocks) return i * 64 + t;
+    const int c = i - a.pre_blocks;
+    const int cx = c % a.ncx, cy = (c / a.ncx) % a.ncy, ct = c / (a.ncx * a.ncy);
+    const int dx = t % a.cW, dy = (t / a.cW) % a.cH, dt = t / (a.cW * a.cH);
+    return a.P + ((ct * a.cT + dt) * a.gH + cy * a.cH + dy) * a.gW + cx * a.cW + dx;
+}
 
 template <typename T, int UNROLL>
 __global__ void __launch_bounds__(128) pool_kernel(PoolArgs a)
@@ -76,6 +89,17 @@ __global__ void __launch_bounds__(128) pool_kernel(PoolArgs a)
 #pragma unroll
         for (int e = 0; e < V; ++e) acc[e] = 0.0;
         int t = 0;
+        if (a.cube) {
+            const T *pb = base + (int64_t)b * a.sb + (int64_t)h * a.sh + c;
+            for (; t + UNROLL <= n; t += UNROLL) {
+                uint4 r[UNROLL];
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) r[u] = ld_nc_v4(pb + (int64_t)block_token(a, i, t + u) * a.sn);
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) Vec<T>::add(acc, r[u]);
+            }
+            for (; t < n; ++t) Vec<T>::add(acc, ld_nc_v4(pb + (int64_t)block_token(a, i, t) * a.sn));
+        }
         for (; t + UNROLL <= n; t += UNROLL) {
             uint4 r[UNROLL];
 #pragma unroll
@@ -122,6 +146,16 @@ cudaError_t launch_pool(const bsa_params &p, const Dims &D, const void *q, const
     a.H = D.H;
     a.d = D.d;
     a.count = blk_count;
+    a.cube = D.cube;
+    a.pre_blocks = D.pre_blocks;
+    a.P = p.prefix_len;
+    a.gH = p.grid_h;
+    a.gW = p.grid_w;
+    a.cT = p.cube_t;
+    a.cH = p.cube_h;
+    a.cW = p.cube_w;
+    a.ncx = D.cube ? p.grid_w / p.cube_w : 1;
+    a.ncy = D.cube ? p.grid_h / p.cube_h : 1;
     dim3 grid(std::max(D.nQB, D.nKB), D.B, 3);
     if (p.dtype == BSA_DT_BF16)
         pool_kernel<__nv_bfloat16, 8><<<grid, 128, 0, st>>>(a);

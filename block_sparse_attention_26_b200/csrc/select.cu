@@ -21,6 +21,7 @@
 //   expand_kernel  bitmask -> ascending CSR column lists (popc prefix per warp).
 #include <math.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "bsa_device.cuh"
@@ -226,30 +227,101 @@ __global__ void __launch_bounds__(256) rows_kernel(RowArgs a)
     if (lane == 0) a.count[r] = total;
 }
 
-// Exclusive scan of counts into int64 row_ptr (single CTA of 1024 threads).
-__global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ count, int64_t rows,
-                                                    int64_t *__restrict__ row_ptr)
+// Exclusive scan of the kept counts into int64 row_ptr, in three launches:
+// each CTA scans a tile of kScanTile rows (4 per thread) and records the
+// tile's total; one CTA scans the totals; every row adds its tile's offset.
+constexpr int kScanTile = 4096;
+
+__global__ void __launch_bounds__(1024) scan_tiles_kernel(const int32_t *__restrict__ count, int64_t rows,
+                                                          int64_t *__restrict__ row_ptr, int64_t *__restrict__ tile_sum)
 {
-    __shared__ int64_t part[1024];
-    const int t = threadIdx.x;
-    const int64_t per = (rows + 1023) / 1024;
-    const int64_t lo = min(rows, t * per), hi = min(rows, lo + per);
-    int64_t s = 0;
-    for (int64_t i = lo; i < hi; ++i) s += count[i];
-    part[t] = s;
+    __shared__ int64_t wsum[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t r0 = (int64_t)blockIdx.x * kScanTile + 4 * threadIdx.x;
+    int64_t v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = r0 + e < rows ? count[r0 + e] : 0;
+    const int64_t s = v[0] + v[1] + v[2] + v[3];
+    int64_t incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) wsum[warp] = incl;
     __syncthreads();
-    for (int off = 1; off < 1024; off <<= 1) {
-        const int64_t v = t >= off ? part[t - off] : 0;
+    if (warp == 0) {
+        int64_t x = wsum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t t = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += t;
+        }
+        wsum[lane] = x;
+    }
+    __syncthreads();
+    int64_t base = (warp > 0 ? wsum[warp - 1] : 0) + incl - s;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        if (r0 + e < rows) row_ptr[r0 + e] = base;
+        base += v[e];
+    }
+    if (threadIdx.x == 1023) tile_sum[blockIdx.x] = wsum[31];
+}
+
+__global__ void __launch_bounds__(1024) scan_tops_kernel(int64_t *__restrict__ tile_sum, int ntiles,
+                                                         int64_t *__restrict__ row_ptr, int64_t rows)
+{
+    __shared__ int64_t wsum[32];
+    __shared__ int64_t carry_s;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) carry_s = 0;
+    __syncthreads();
+    for (int t0 = 0; t0 < ntiles; t0 += 1024) {
+        const int t = t0 + threadIdx.x;
+        const int64_t s = t < ntiles ? tile_sum[t] : 0;
+        int64_t incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
         __syncthreads();
-        part[t] += v;
+        if (warp == 0) {
+            int64_t x = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            wsum[lane] = x;
+        }
+        __syncthreads();
+        const int64_t carry = carry_s;
+        if (t < ntiles) tile_sum[t] = carry + (warp > 0 ? wsum[warp - 1] : 0) + incl - s;
+        __syncthreads();
+        if (threadIdx.x == 0) carry_s = carry + wsum[31];
         __syncthreads();
     }
-    int64_t run = part[t] - s;
-    for (int64_t i = lo; i < hi; ++i) {
-        row_ptr[i] = run;
-        run += count[i];
-    }
-    if (t == 1023) row_ptr[rows] = part[1023];
+    if (threadIdx.x == 0) row_ptr[rows] = carry_s;
+}
+
+__global__ void __launch_bounds__(256) scan_add_kernel(int64_t *__restrict__ row_ptr, int64_t rows,
+                                                       const int64_t *__restrict__ tile_off)
+{
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += (int64_t)gridDim.x * blockDim.x)
+        row_ptr[r] += tile_off[r / kScanTile];
+}
+
+cudaError_t launch_scan(const int32_t *cnt, int64_t rows, int64_t *row_ptr, int64_t *tile_sum, cudaStream_t st)
+{
+    const int ntiles = (int)ceil_div(rows, kScanTile);
+    scan_tiles_kernel<<<(unsigned)ntiles, 1024, 0, st>>>(cnt, rows, row_ptr, tile_sum);
+    scan_tops_kernel<<<1, 1024, 0, st>>>(tile_sum, ntiles, row_ptr, rows);
+    const unsigned g = (unsigned)std::min<int64_t>(ceil_div(rows, 256), (int64_t)sm_count() * 8);
+    scan_add_kernel<<<g, 256, 0, st>>>(row_ptr, rows, tile_sum);
+    return cudaGetLastError();
 }
 
 __global__ void __launch_bounds__(256) expand_kernel(const uint32_t *__restrict__ bitmask,
@@ -293,6 +365,35 @@ __global__ void __launch_bounds__(256) expand_kernel(const uint32_t *__restrict_
 
 }  // namespace
 
+void select_regions(const bsa_params &p, const Dims &D, WsLayout &L, Taker &T)
+{
+    const bool route = certified_route(p);
+    const int64_t BH = (int64_t)D.B * D.H;
+    const size_t rows = (size_t)D.rows;
+    L.status = T.take(sizeof(int32_t) * 2);
+    // block scores: all of them on the fp64 path; on the certified route only
+    // approximate ones, for the extra-token sampler
+    L.scores = T.take(!route || p.extra_tokens > 0 ? rows * D.nKB * sizeof(float) : 0);
+    L.bitmask = T.take(rows * D.nW * sizeof(uint32_t));
+    L.counts = T.take(rows * sizeof(int32_t));
+    L.scan_tmp = T.take((size_t)ceil_div(D.rows, kScanTile) * sizeof(int64_t));
+    const size_t d = (size_t)D.d;
+    const int ns = route ? route_nsplit(D) : 0;
+    L.r_nsplit = ns;
+    L.r_k16 = T.take(route ? (size_t)BH * D.nKB * d * 2 : 0);
+    L.r_knorm = T.take(route ? (size_t)BH * route_nkbp(D) * 4 : 0);
+    L.r_knmax = T.take(route ? (size_t)BH * (route_nkbp(D) / 32) * 4 : 0);
+    L.r_gram = T.take(route ? (size_t)BH * ns * d * d * 8 : 0);
+    L.r_ksum = T.take(route ? (size_t)BH * ns * d * 8 : 0);
+    L.r_cov = T.take(route ? (size_t)BH * d * d * 8 : 0);
+    L.r_hstat = T.take(route ? (size_t)BH * (d + 3) * 8 : 0);
+    L.r_info = T.take(route ? rows * sizeof(RowInfo) : 0);
+    L.r_ulist = T.take(route ? rows * kUcap * 4 : 0);
+    L.r_ucnt = T.take(route ? rows * 4 : 0);
+    L.r_fbl = T.take(route ? (rows + 1) * 4 : 0);
+    L.r_fbs = T.take(route ? (size_t)fallback_ctas() * route_nkbp(D) * 4 : 0);
+}
+
 cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar, const float *kbar,
                           int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity,
                           int32_t *kept_count, char *ws, const WsLayout &L, cudaStream_t st)
@@ -301,6 +402,18 @@ cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar,
     uint32_t *bm = reinterpret_cast<uint32_t *>(ws + L.bitmask);
     int32_t *cnt = reinterpret_cast<int32_t *>(ws + L.counts);
     int32_t *status = reinterpret_cast<int32_t *>(ws + L.status);
+    int64_t *tsum = reinterpret_cast<int64_t *>(ws + L.scan_tmp);
+    const unsigned g2 = (unsigned)ceil_div(D.rows, 8);
+
+    if (certified_route(p)) {
+        cudaError_t e = launch_route(p, D, qbar, kbar, ws, L, st);
+        if (e != cudaSuccess) return e;
+        e = launch_scan(cnt, D.rows, row_ptr, tsum, st);
+        if (e != cudaSuccess) return e;
+        expand_kernel<<<g2, 256, 0, st>>>(bm, cnt, row_ptr, D.rows, D.nW, col_capacity, col_idx, kept_count,
+                                          status);
+        return cudaGetLastError();
+    }
 
     dim3 g1((unsigned)ceil_div(D.nQB, kRows), (unsigned)(D.B * D.H));
     const int smem = (kRows * 128 + kChan * (kKeys + 1)) * (int)sizeof(double);
@@ -328,9 +441,9 @@ cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar,
     a.keep_diag = p.keep_diag;
     a.bitmask = bm;
     a.count = cnt;
-    const unsigned g2 = (unsigned)ceil_div(D.rows, 8);
     rows_kernel<<<g2, 256, 0, st>>>(a);
-    scan_kernel<<<1, 1024, 0, st>>>(cnt, D.rows, row_ptr);
+    cudaError_t es = launch_scan(cnt, D.rows, row_ptr, tsum, st);
+    if (es != cudaSuccess) return es;
     expand_kernel<<<g2, 256, 0, st>>>(bm, cnt, row_ptr, D.rows, D.nW, col_capacity, col_idx,
                                       kept_count, status);
     return cudaGetLastError();
@@ -419,20 +532,12 @@ cudaError_t static_scratch(char **out)
 bool static_select_layout(const bsa_params &p, WsLayout *L, size_t *need)
 {
     const Dims D = dims_of(p);
-    size_t off = 0;
-    auto take = [&](size_t bytes) {
-        const size_t at = off;
-        off = align_up(off + bytes, 256);
-        return at;
-    };
     *L = WsLayout();
-    L->status = take(sizeof(int32_t) * 2);
-    L->scores = take((size_t)D.rows * D.nKB * sizeof(float));
-    L->bitmask = take((size_t)D.rows * D.nW * sizeof(uint32_t));
-    L->counts = take((size_t)D.rows * sizeof(int32_t));
-    L->total = off;
-    *need = off;
-    return off <= kStaticScratchBytes;
+    Taker T;
+    select_regions(p, D, *L, T);
+    L->total = T.off;
+    *need = T.off;
+    return T.off <= kStaticScratchBytes;
 }
 
 cudaError_t launch_select_static(const bsa_params &p, const Dims &D, const float *qbar, const float *kbar,

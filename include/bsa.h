@@ -28,6 +28,14 @@
  *                        sink_conditioning = exact_kv_and_rows).
  *   4. bsa_dense_ref_rows -- dense softmax attention for a range of query rows.
  *
+ * Cube tiling (method BSA_VSA): block b < prefix_len / 64 is the prefix's
+ * b-th run of 64 tokens; block prefix_len / 64 + c is cube c of the grid in
+ * t-major cube order, its 64 tokens taken t-major inside the cube.  Query and
+ * key blocks are the same cubes (q_block = k_block = 64).  Pooled means, rows
+ * of the CSR and the diagonal ("key block = query block") are in that block
+ * order; Q, K, V, O and LSE stay in token order.  Needs B == 1, prefix_len a
+ * multiple of 64, dense rows inside the prefix, centroid 0, extra_tokens 0.
+ *
  * Conventions shared by every call:
  *   - Tensors Q, K, V and O are [B, N, H, d] with element strides stride_b,
  *     stride_n, stride_h and a contiguous channel dimension; all four share the
@@ -73,7 +81,11 @@ typedef enum {
 } bsa_status;
 
 typedef enum { BSA_DT_BF16 = 0, BSA_DT_F32 = 1 } bsa_dtype;
-typedef enum { BSA_SOL = 0, BSA_SLA = 1 } bsa_method;   /* vsa: not provided (needs trained weights) */
+/* BSA_VSA: the fine stage of [DOC]'s vsa method without its learned coarse
+ * branch (the node runs it so when the model lacks that layer): key blocks and
+ * query blocks are 3-D cubes of the latent video grid, the top keep_percent %
+ * of key cubes per query cube are attended exactly, the rest dropped. */
+typedef enum { BSA_SOL = 0, BSA_SLA = 1, BSA_VSA = 2 } bsa_method;
 
 typedef struct {
     int32_t B, H, N, d;            /* batch, heads, tokens, head dim (64 or 128) */
@@ -92,6 +104,10 @@ typedef struct {
     int32_t extra_tokens;          /* E: extra top-scoring tokens per query block, 0..256; 0 disables */
     int32_t centroid;              /* 1: unselected blocks contribute through centroids (Sol);
                                       0: they are dropped (SLA without its trained linear branch) */
+    int32_t grid_t, grid_h, grid_w;  /* BSA_VSA: the latent grid T x Hs x Ws of the tokens after the
+                                        prefix, flattened t-major (prefix_len + T*Hs*Ws == N) */
+    int32_t cube_t, cube_h, cube_w;  /* BSA_VSA: cube extents (4, 4, 4); product 64, each dividing its
+                                        grid extent ([DOC] vsa: 3-D video cube tiling) */
 } bsa_params;
 
 /* Fill *p with the defaults of the node documentation for `method`
@@ -218,6 +234,45 @@ BSA_API bsa_status bsa_device_status(void *ws, void *stream, int32_t *device_sta
  * `ws` (read it with bsa_device_status) and the kernel returns; nothing traps
  * and the context stays usable. */
 BSA_API bsa_status bsa_selftest_bounded_wait(void *ws, int64_t cycles, void *stream);
+
+/* Per-step policy ([DOC] general inputs start_percent, end_percent,
+ * dense_blocks, min_tokens and "constraints and limitations"; [STAR]
+ * "Hybrid"): whether one attention call takes the sparse path or stays dense.
+ * Host-only; nothing is launched.  A dense call runs bsa_dense_ref_rows over
+ * all N rows in place of pool / select / attention. */
+typedef struct {
+    double start_percent;        /* sparse from this fraction of the sampling schedule on ...     */
+    double end_percent;          /* ... up to and including this one (both in [0, 1]; 0.2 / 1.0)   */
+    int32_t min_tokens;          /* sequences shorter than this stay dense (12288)                */
+    int32_t hybrid;              /* 1: the first and last hybrid_guard_steps sampling steps dense */
+    int32_t hybrid_guard_steps;  /* guard steps at each end of the schedule (1)                   */
+    int32_t pad_;
+    const char *dense_blocks;    /* transformer blocks always dense, e.g. "0, 1, 47-49"; NULL or
+                                    "" for none (host string, read during the call only)          */
+} bsa_policy;
+
+typedef enum {
+    BSA_RUN_SPARSE = 0,          /* take the sparse path                                          */
+    BSA_DENSE_SHORT = 1,         /* n_tokens < min_tokens                                         */
+    BSA_DENSE_BLOCK = 2,         /* block_index listed in dense_blocks                            */
+    BSA_DENSE_HYBRID = 3,        /* a guard step of the hybrid schedule                           */
+    BSA_DENSE_WINDOW = 4         /* progress outside [start_percent, end_percent]                 */
+} bsa_decision;
+
+/* Defaults of the node documentation: window [0.2, 1.0], min_tokens 12288,
+ * no dense blocks, hybrid off with one guard step at each end. */
+BSA_API void bsa_default_policy(bsa_policy *pol);
+
+/* Decide one call.  n_tokens: sequence length N (>= 1); block_index: the
+ * transformer block's index, or < 0 when the model reports none (dense_blocks
+ * is then ignored); progress: fraction of the sampling schedule done, in
+ * [0, 1]; step / n_steps: the sampling step (0-based) and their number, needed
+ * only when hybrid is on (BSA_ERR_INVALID_ARG when they cannot place the step,
+ * as the hybrid mode stops when it cannot tell the step).  *decision gets a
+ * bsa_decision; reasons are checked in the order of the enum.  A malformed
+ * dense_blocks list is BSA_ERR_INVALID_ARG. */
+BSA_API bsa_status bsa_policy_decide(const bsa_policy *pol, int32_t n_tokens, int32_t block_index,
+                                     double progress, int32_t step, int32_t n_steps, int32_t *decision);
 
 /* Static description of a status code. */
 BSA_API const char *bsa_status_string(bsa_status s);

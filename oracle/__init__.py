@@ -222,6 +222,36 @@ def attention_rows(q: Raw, k: Raw, v: Raw, Bq: int, Bk: int, kbar, vbar, count, 
     return out, lse
 
 
+def cube_order(w) -> np.ndarray:
+    """Block order of the tokens under 3-D cube tiling ("BlockSparseAttention -
+    ComfyUI Built-in Node Documentation", vsa: 3-D video cube tiling): position p
+    of the block-ordered sequence holds token cube_order(w)[p].  The packed
+    prefix keeps its own order (its 64-token runs are blocks); then come the
+    cubes of the T x Hs x Ws grid in t-major order, each cube's tokens t-major
+    inside it."""
+    P = w.prefix_len
+    T, Hs, Ws = w.grid
+    ct, cy, cx = w.cube
+    order = list(range(P))
+    for t0 in range(0, T, ct):
+        for y0 in range(0, Hs, cy):
+            for x0 in range(0, Ws, cx):
+                for dt in range(ct):
+                    for dy in range(cy):
+                        for dx in range(cx):
+                            order.append(P + ((t0 + dt) * Hs + (y0 + dy)) * Ws + (x0 + dx))
+    return np.asarray(order, np.int64)
+
+
+def reorder(x: Raw, order: np.ndarray) -> Raw:
+    """The tokens of x taken in the given order, as a contiguous [B, N, H, d] Raw."""
+    item = x.arr.itemsize
+    full = np.lib.stride_tricks.as_strided(x.arr, shape=(x.B, x.N, x.H, x.d),
+                                           strides=(x.sb * item, x.sn * item, x.sh * item, item))
+    arr = np.ascontiguousarray(full[:, order])
+    return Raw(arr.reshape(-1), x.dtype, x.N * x.H * x.d, x.H * x.d, x.d, x.B, x.N, x.H, x.d)
+
+
 def mask_to_csr(keep: np.ndarray):
     """CSR (row_ptr [rows+1], col [nnz] ascending, count [rows]) of a 0/1 mask."""
     flat = keep.reshape(-1, keep.shape[-1]).astype(bool)
@@ -245,6 +275,7 @@ class LayerResult:
     thr: np.ndarray
     extra: Optional[np.ndarray]
     ecnt: Optional[np.ndarray]
+    order: Optional[np.ndarray] = None     # vsa: block-order position -> token
 
 
 def routing(w, q: Raw, k: Raw, v: Raw, extra_rows: Optional[Sequence[int]] = None,
@@ -253,12 +284,23 @@ def routing(w, q: Raw, k: Raw, v: Raw, extra_rows: Optional[Sequence[int]] = Non
 
     extra_rows restricts the (expensive) extra-token search to those rows; the
     other rows get an empty list.
+
+    Method "vsa" (the fine stage of the vsa method without its learned coarse
+    branch): blocks are the cubes of cube_order; the top keep_percent % of key
+    cubes per query cube are kept, with the sink and diagonal blocks, as SLA
+    keeps blocks; pooled means and masks are in block order.
     """
+    order = None
+    method = w.method
+    if w.method == "vsa":
+        order = cube_order(w)
+        q, k, v = reorder(q, order), reorder(k, order), reorder(v, order)
+        method = "sla"
     qbar, _ = block_means(q, w.q_block)
     kbar, count = block_means(k, w.k_block)
     vbar, _ = block_means(v, w.k_block)
     S = block_scores(qbar, kbar)
-    keep, thr = select(S, w.N, w.q_block, w.k_block, w.method, w.tau, w.keep_percent,
+    keep, thr = select(S, w.N, w.q_block, w.k_block, method, w.tau, w.keep_percent,
                        w.sink_blocks, w.prefix_len, w.keep_diag)
     extra = ecnt = None
     E = w.extra_tokens
@@ -269,11 +311,18 @@ def routing(w, q: Raw, k: Raw, v: Raw, extra_rows: Optional[Sequence[int]] = Non
         ex, ec, rows = extra_tokens(qbar, k, keep, w.q_block, w.k_block, E, extra_rows)
         extra[rows] = ex
         ecnt[rows] = ec
-    return LayerResult(qbar, kbar, vbar, count, S, keep, thr, extra, ecnt)
+    return LayerResult(qbar, kbar, vbar, count, S, keep, thr, extra, ecnt, order)
 
 
 def layer_rows(w, q: Raw, k: Raw, v: Raw, r: LayerResult, tokens: np.ndarray):
-    """Final outputs (sparse + centroid, dense rows applied) for `tokens`."""
+    """Final outputs (sparse + centroid, dense rows applied) for `tokens`
+    ([m, 3] = (b, h, token))."""
+    if r.order is not None:
+        q, k, v = reorder(q, r.order), reorder(k, r.order), reorder(v, r.order)
+        pos = np.empty_like(r.order)
+        pos[r.order] = np.arange(len(r.order))
+        tokens = tokens.copy()
+        tokens[:, 2] = pos[tokens[:, 2]]
     return attention_rows(q, k, v, w.q_block, w.k_block, r.kbar, r.vbar, r.count,
                           r.keep.reshape(w.rows, w.nKB), tokens, r.extra, r.ecnt,
                           centroid=w.centroid, dense_rows=w.dense_rows)
@@ -285,5 +334,6 @@ def all_tokens(w) -> np.ndarray:
 
 
 __all__ = ["build", "threads", "Raw", "as_raw", "block_means", "block_scores", "forced_blocks",
-           "select", "extra_tokens", "attention_rows", "mask_to_csr", "routing", "layer_rows",
+           "select", "extra_tokens", "attention_rows", "mask_to_csr", "routing", "layer_rows", "cube_order",
+           "reorder",
            "all_tokens", "LayerResult"]

@@ -324,3 +324,68 @@ def test_tiny_cases_match_pure_python_bruteforce(cfg):
     assert (res.keep[0].astype(bool) == np.array(keep_b)).all()
     np.testing.assert_allclose(out[0], np.array(out_b), rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse[0], np.array(lse_b), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- cube tiling (vsa)
+
+def _vsa(**kw):
+    base = dict(name="v", B=1, H=2, d=16, dtype="bf16", method="vsa", q_block=64, k_block=64,
+                keep_percent=30.0, centroid=0)
+    base.update(kw)
+    return Workload(**base)
+
+
+def test_cube_order_blocks_are_the_grid_cubes():
+    """Every block of the cube order is one 4 x 4 x 4 box of the latent grid
+    (its tokens' (t, y, x) span 4 consecutive values on each axis, aligned to
+    4), the prefix keeps its order, and every token appears once."""
+    w = _vsa(N=64 + 8 * 12 * 16, prefix_len=64, grid=(8, 12, 16))
+    order = oracle.cube_order(w)
+    assert sorted(order.tolist()) == list(range(w.N))
+    assert order[:64].tolist() == list(range(64))
+    T, Hs, Ws = w.grid
+    for blk in range(1, w.N // 64):
+        toks = order[64 * blk:64 * blk + 64] - w.prefix_len
+        t, y, x = toks // (Hs * Ws), (toks // Ws) % Hs, toks % Ws
+        for axis in (t, y, x):
+            assert axis.min() % 4 == 0 and axis.max() - axis.min() == 3
+        assert len({(a, b, c) for a, b, c in zip(t, y, x)}) == 64
+        # t-major inside the cube: slot s = 16 dt + 4 dy + dx
+        s = 16 * (t - t.min()) + 4 * (y - y.min()) + (x - x.min())
+        assert s.tolist() == list(range(64))
+
+
+def test_vsa_on_column_cubes_is_sla_with_64_token_blocks():
+    """With a 4 x 4 frame every cube is 64 consecutive tokens, so cube tiling is
+    the identity order and vsa must give exactly SLA with Q64/K64 blocks."""
+    w = _vsa(N=64 * 12, grid=(48, 4, 4), keep_percent=25.0)
+    assert oracle.cube_order(w).tolist() == list(range(w.N))
+    q, k, v = (_rand((1, w.N, w.H, w.d), torch.bfloat16, s) for s in (41, 42, 43))
+    out_v, lse_v, res_v = _oracle_full(w, q, k, v)
+    out_s, lse_s, res_s = _oracle_full(w.replace(method="sla"), q, k, v)
+    assert np.array_equal(res_v.keep, res_s.keep)
+    assert np.array_equal(out_v, out_s) and np.array_equal(lse_v, lse_s)
+
+
+def test_vsa_keep_all_is_dense_attention():
+    w = _vsa(N=64 + 4 * 8 * 8, prefix_len=64, grid=(4, 8, 8), keep_percent=100.0)
+    q, k, v = (_rand((1, w.N, w.H, w.d), torch.bfloat16, s) for s in (44, 45, 46))
+    out, lse, res = _oracle_full(w, q, k, v)
+    ref, ref_lse = _dense_numpy(q, k, v)
+    assert res.keep.all()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def test_vsa_cube_means_are_means_over_the_cube():
+    w = _vsa(N=8 * 8 * 8, grid=(8, 8, 8))
+    k = _rand((1, w.N, w.H, w.d), torch.float32, 47)
+    res = oracle.routing(w, *(oracle.as_raw(k) for _ in range(3)))
+    K = k.double().numpy().reshape(8, 8, 8, w.H, w.d)          # (t, y, x, h, c)
+    c = 0
+    for t0 in range(0, 8, 4):
+        for y0 in range(0, 8, 4):
+            for x0 in range(0, 8, 4):
+                ref = K[t0:t0 + 4, y0:y0 + 4, x0:x0 + 4].mean(axis=(0, 1, 2)).astype(np.float32)
+                np.testing.assert_allclose(res.kbar[0, :, c], ref, rtol=2e-7, atol=0)
+                c += 1

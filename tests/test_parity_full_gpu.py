@@ -31,7 +31,7 @@ def _sample_tokens(w):
     return np.array(toks, np.int64)
 
 
-@pytest.mark.parametrize("name", ["sol_mid", "sla_topk", "sol_sinks", "long"])
+@pytest.mark.parametrize("name", ["sol_mid", "sla_topk", "sol_sinks", "long", "vsa_cubes"])
 def test_full_size_parity(name):
     w = CONFIGS[name]
     q, k, v = make_qkv(w, "cuda")
@@ -51,6 +51,8 @@ def test_full_size_parity(name):
     mask = csr_to_mask(buf.row_ptr, buf.col_idx, w.rows, w.nKB)
     exempt = compare_masks(mask, res, w)
     print(f"{name}: kept fraction {mask.mean():.4f}, exempt blocks {exempt}")
+    if w.method == "sol":
+        assert exempt == 0          # the certified route is exact
     # outputs on the sampled rows
     ref, ref_lse = oracle.layer_rows(w, qr, kr, vr, res, toks)
     got = out[toks[:, 0], toks[:, 2], toks[:, 1]].float().cpu().numpy()

@@ -167,3 +167,58 @@ def test_sigma_zero_rows_keep_only_forced():
     kc = buf.kept_count.cpu().numpy()
     # sink block 0 plus the diagonal block (the same block for query block 0)
     assert kc[0] == 1 and (kc[1:w.nQB] == 2).all()
+
+
+# Sol with a finite tau takes the certified route: its masks equal the
+# definition's bit for bit, with no near-threshold exemption.  The cases below
+# also push rows onto the route's exact paths: keys that are nearly identical
+# (every block undecided by the tensor-core scores: list overflow, exact
+# fallback rows), and pooled values scaled far up or down (bounds near the ends
+# of the f32 range).
+ROUTE = {
+    "near_identical_keys": Workload("near_identical_keys", B=1, H=2, N=3000, d=128, dtype="bf16", method="sol",
+                                    q_block=64, k_block=64, tau=1.0, grid=(3, 20, 50), seed=31),
+    "large_scale": Workload("large_scale", B=1, H=2, N=2500, d=128, dtype="bf16", method="sol", q_block=64,
+                            k_block=64, tau=1.3, grid=(2, 25, 50), seed=32),
+    "tiny_scale": Workload("tiny_scale", B=1, H=2, N=2500, d=64, dtype="bf16", method="sol", q_block=64,
+                           k_block=64, tau=0.7, grid=(2, 25, 50), seed=33),
+    "negative_tau": Workload("negative_tau", B=1, H=2, N=2970, d=128, dtype="bf16", method="sol", q_block=64,
+                             k_block=64, tau=-0.6, prefix_len=130, grid=(2, 20, 71), seed=34),
+}
+
+
+def _route_inputs(name, w):
+    q, k, v = make_qkv(w, "cpu")
+    if name == "near_identical_keys":
+        # one key row for the whole sequence plus a perturbation of a few ulps
+        base = k[:, :1].float()
+        k = (base + 1e-3 * (k.float() - base)).to(k.dtype)
+    elif name == "large_scale":
+        q = q * 2.0 ** 60
+    elif name == "tiny_scale":
+        q = q * 2.0 ** -120
+        k = k * 2.0 ** -4
+    return q.contiguous(), k.contiguous(), v
+
+
+@pytest.mark.parametrize("name", list(ROUTE))
+def test_certified_route_masks_exact(name):
+    w = ROUTE[name]
+    q, k, v = _route_inputs(name, w)
+    p, buf, out, status = gpu_layer(w, q.cuda(), k.cuda(), v.cuda())
+    assert status == 0
+    res = oracle.routing(w, oracle.as_raw(q), oracle.as_raw(k), oracle.as_raw(v))
+    assert np.array_equal(buf.qbar.cpu().numpy(), res.qbar)
+    mask = csr_to_mask(buf.row_ptr, buf.col_idx, w.rows, w.nKB)
+    ora = res.keep.reshape(w.rows, w.nKB)
+    diff = np.argwhere(mask != ora)
+    assert len(diff) == 0, f"{len(diff)} mask differences, e.g. {diff[:5].tolist()}"
+    assert np.array_equal(buf.kept_count.cpu().numpy(), ora.sum(axis=1).astype(np.int32))
+
+
+@pytest.mark.parametrize("name", [n for n, w in SMALL.items() if w.method == "sol" and math.isfinite(w.tau)])
+def test_certified_route_no_exemptions(runs, name):
+    w, _, _, p, buf, _, status, res = runs(name)
+    assert status == 0
+    mask = csr_to_mask(buf.row_ptr, buf.col_idx, w.rows, w.nKB)
+    assert np.array_equal(mask, res.keep.reshape(w.rows, w.nKB))

@@ -37,7 +37,7 @@ class Workload:
     N: int
     d: int
     dtype: str                      # "bf16" | "f32"
-    method: str                     # "sol" | "sla"
+    method: str                     # "sol" | "sla" | "vsa"
     q_block: int
     k_block: int
     tau: float = 1.3
@@ -49,6 +49,7 @@ class Workload:
     extra_tokens: int = 0
     centroid: int = 1
     grid: Optional[Tuple[int, int, int]] = None   # latent grid (T, Hs, Ws); None = iid tokens
+    cube: Tuple[int, int, int] = (4, 4, 4)         # vsa: cube extents (t, y, x)
     seed: int = 0
     field_sigma: float = 4.0
     noise: float = 0.5
@@ -85,7 +86,14 @@ LONG = Workload("long", B=1, H=40, N=207872, d=128, dtype="bf16", method="sol",
                 q_block=64, k_block=64, tau=1.5, prefix_len=512, dense_rows=(256, 512),
                 extra_tokens=0, centroid=1, grid=(24, 90, 96), seed=5000)
 
-CONFIGS = {w.name: w for w in (TINY_SOL, SOL_MID, SLA_TOPK, SOL_SINKS, LONG)}
+# Cube tiling (the vsa method's fine stage without its learned coarse branch)
+# on the SLA workload's grid, whose extents are multiples of 4; keep_percent 10,
+# the value the FastH3-VSA checkpoint is trained at.
+VSA_CUBES = Workload("vsa_cubes", B=1, H=24, N=46080, d=128, dtype="bf16", method="vsa",
+                     q_block=64, k_block=64, keep_percent=10.0, centroid=0,
+                     grid=(12, 48, 80), seed=6000)
+
+CONFIGS = {w.name: w for w in (TINY_SOL, SOL_MID, SLA_TOPK, SOL_SINKS, LONG, VSA_CUBES)}
 
 
 def _gaussian_transfer(n: int, sigma: float, device) -> torch.Tensor:
