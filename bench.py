@@ -332,6 +332,70 @@ def launches_per_step(w) -> int:
             + 1 + (1 if dense_split else 0))
 
 
+def run_producer(args, w, dev):
+    """--producer: the QKV projection with pooling in its epilogue
+    (bsa_qkv_pool) against the same work unfused: cuBLAS (torch.matmul) for
+    X W^T, then bsa_pool reading Q, K and V back.  d_model = H * d."""
+    import block_sparse_attention_26_b200 as bsa
+    dm = w.H * w.d
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 9)
+    x = torch.randn((w.B, w.N, dm), generator=g, device=dev).to(torch.bfloat16)
+    W = (torch.randn((3 * w.H * w.d, dm), generator=g, device=dev) / dm ** 0.5).to(torch.bfloat16)
+    q, k, v = (torch.empty((w.B, w.N, w.H, w.d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    p = bsa.params_for(w, q)
+    nQB, nKB, _ = bsa.dims(p)
+    qbar = torch.empty((w.B, w.H, nQB, w.d), dtype=torch.float32, device=dev)
+    kbar = torch.empty((w.B, w.H, nKB, w.d), dtype=torch.float32, device=dev)
+    vbar = torch.empty_like(kbar)
+    cnt = torch.empty((nKB,), dtype=torch.int32, device=dev)
+    ws = torch.zeros(4096, dtype=torch.uint8, device=dev)
+    y = torch.empty((w.B, w.N, 3, w.H, w.d), dtype=torch.bfloat16, device=dev)
+    yq, yk, yv = y[:, :, 0], y[:, :, 1], y[:, :, 2]
+    py = bsa.params_for(w, yq)
+    stream = torch.cuda.current_stream(dev)
+
+    def fused():
+        bsa.bsa_qkv_pool(p, x, W, q, k, v, qbar, kbar, vbar, cnt, ws, stream)
+
+    def unfused(ev=None):
+        torch.matmul(x, W.t(), out=y.view(w.B, w.N, 3 * w.H * w.d))
+        if ev:
+            ev.record(stream)
+        bsa.bsa_pool(py, yq, yk, yv, qbar, kbar, vbar, cnt, stream)
+
+    def timed(fn, mid=False):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        em = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e0.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            fn(em[i]) if mid else fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        total = e0.elapsed_time(e1) / args.steps
+        part = statistics.mean(s.elapsed_time(m) for s, m in zip(starts, em)) if mid else None
+        return total, part
+
+    with ClockSampler(int(str(dev).split(":")[-1]) if ":" in str(dev) else 0) as clocks:
+        t_fused, _ = timed(fused)
+        t_unf, t_gemm = timed(unfused, mid=True)
+    assert bsa.bsa_device_status(ws) == 0
+    flop = 2.0 * w.B * w.N * dm * 3 * w.H * w.d
+    peaks, src = _peaks()
+    line = {"metric": "qkv projection + pooling ms (producer)", "workload": w.name, "d_model": dm,
+            "fused_ms": t_fused, "unfused_ms": t_unf, "unfused_gemm_ms": t_gemm, "unfused_pool_ms": t_unf - t_gemm,
+            "fused_tflops": flop / (t_fused * 1e-3) / 1e12, "cublas_tflops": flop / (t_gemm * 1e-3) / 1e12,
+            "fused_frac_of_bf16_peak": flop / (t_fused * 1e-3) / 1e12 / float(peaks["bf16_tflops"]),
+            "peak_source": f"{src} bf16_tflops", "steps": args.steps, "warmup": args.warmup,
+            "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -343,6 +407,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--heads", type=int, default=0, help="override H (profiling a smaller case)")
+    ap.add_argument("--producer", action="store_true",
+                    help="time the QKV projection with pooling in its epilogue against cuBLAS + bsa_pool")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -368,6 +434,9 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.producer:
+        run_producer(args, w, dev)
+        return
     pg = None
     if world > 1:
         import datetime

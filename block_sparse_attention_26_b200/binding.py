@@ -74,6 +74,7 @@ def _load() -> ctypes.CDLL:
     lib.bsa_workspace_size.argtypes = [PP, ctypes.POINTER(SZ), ctypes.POINTER(I64)]
     lib.bsa_pool.argtypes = [PP, P, P, P, P, P, P, P, P]
     lib.bsa_select.argtypes = [PP, P, P, P, P, P, I64, P, P, P, P, SZ, P]
+    lib.bsa_qkv_pool.argtypes = [PP, P, I32, P, P, P, P, P, P, P, P, P, P]
     lib.bsa_select_static.argtypes = [PP, P, P, P, P, I64, P, P]
     lib.bsa_attention.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.bsa_attention_prepare.argtypes = lib.bsa_attention.argtypes
@@ -90,7 +91,7 @@ def _load() -> ctypes.CDLL:
     lib.bsa_status_string.restype = ctypes.c_char_p
     lib.bsa_last_error.argtypes = []
     lib.bsa_last_error.restype = ctypes.c_char_p
-    for f in ("bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_select_static", "bsa_attention",
+    for f in ("bsa_workspace_size", "bsa_pool", "bsa_qkv_pool", "bsa_select", "bsa_select_static", "bsa_attention",
               "bsa_attention_prepare", "bsa_attention_run", "bsa_dense_ref_rows", "bsa_device_status",
               "bsa_selftest_bounded_wait"):
         getattr(lib, f).restype = I32
@@ -99,7 +100,7 @@ def _load() -> ctypes.CDLL:
 
 lib = _load()
 
-EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_select", "bsa_select_static",
+EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_qkv_pool", "bsa_select", "bsa_select_static",
             "bsa_attention", "bsa_attention_prepare", "bsa_attention_run", "bsa_dense_ref_rows",
             "bsa_device_status", "bsa_selftest_bounded_wait", "bsa_default_policy", "bsa_policy_decide",
             "bsa_status_string", "bsa_last_error")
@@ -181,6 +182,12 @@ def bsa_workspace_size(p: bsa_params):
 def bsa_pool(p, q, k, v, qbar, kbar, vbar, blk_count, stream=None):
     _check(lib.bsa_pool(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(qbar), _ptr(kbar), _ptr(vbar),
                         _ptr(blk_count), _stream(stream)), "bsa_pool")
+
+
+def bsa_qkv_pool(p, x, w_qkv, q, k, v, qbar, kbar, vbar, blk_count, ws=None, stream=None):
+    _check(lib.bsa_qkv_pool(ctypes.byref(p), _ptr(x), int(x.shape[-1]), _ptr(w_qkv), _ptr(q), _ptr(k), _ptr(v),
+                            _ptr(qbar), _ptr(kbar), _ptr(vbar), _ptr(blk_count), _ptr(ws), _stream(stream)),
+           "bsa_qkv_pool")
 
 
 def bsa_select(p, qbar, kbar, k, row_ptr, col_idx, kept_count, extra_idx, extra_count, ws,

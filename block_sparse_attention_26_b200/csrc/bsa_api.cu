@@ -245,6 +245,30 @@ bsa_status bsa_pool(const bsa_params *p, const void *q, const void *k, const voi
     return from_cuda(launch_pool(*p, D, q, k, v, qbar, kbar, vbar, blk_count, (cudaStream_t)stream), "bsa_pool");
 }
 
+bsa_status bsa_qkv_pool(const bsa_params *p, const void *x, int32_t d_model, const void *w_qkv, void *q, void *k,
+                        void *v, float *qbar, float *kbar, float *vbar, int32_t *blk_count, void *ws, void *stream)
+{
+    g_err[0] = 0;
+    TRY(check_params(p));
+    if (p->dtype != BSA_DT_BF16) FAIL(BSA_ERR_UNSUPPORTED, "bsa_qkv_pool: bf16 only");
+    if (p->method == BSA_VSA) FAIL(BSA_ERR_UNSUPPORTED, "bsa_qkv_pool: cube tiling pools cubes; use bsa_pool");
+    if (d_model < 64 || d_model % 64) FAIL(BSA_ERR_UNSUPPORTED, "bsa_qkv_pool: d_model must be a multiple of 64");
+    if ((p->H * p->d) % 256) FAIL(BSA_ERR_UNSUPPORTED, "bsa_qkv_pool: H * d must be a multiple of 256");
+    TRY(check_tensor(x, "x"));
+    TRY(check_tensor(w_qkv, "w_qkv"));
+    TRY(check_tensor(q, "q"));
+    TRY(check_tensor(k, "k"));
+    TRY(check_tensor(v, "v"));
+    TRY(check_tensor(qbar, "qbar"));
+    TRY(check_tensor(kbar, "kbar"));
+    TRY(check_tensor(vbar, "vbar"));
+    if (ws != nullptr && !aligned16(ws)) FAIL(BSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    const Dims D = dims_of(*p);
+    return from_cuda(launch_qkv_pool(*p, D, x, d_model, w_qkv, q, k, v, qbar, kbar, vbar, blk_count,
+                                     static_cast<int32_t *>(ws), (cudaStream_t)stream),
+                     "bsa_qkv_pool");
+}
+
 bsa_status bsa_select(const bsa_params *p, const float *qbar, const float *kbar, const void *k,
                       int64_t *row_ptr, int32_t *col_idx, int64_t col_capacity, int32_t *kept_count,
                       int32_t *extra_idx, int32_t *extra_count, void *ws, size_t ws_bytes, void *stream)

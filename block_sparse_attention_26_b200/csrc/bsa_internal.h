@@ -141,6 +141,11 @@ cudaError_t launch_select_static(const bsa_params &p, const Dims &D, const float
                                  int32_t *kept_count, const WsLayout &L, cudaStream_t st);
 size_t static_scratch_bytes();
 
+// The QKV projection with pooling in its epilogue (bsa_qkv_pool).
+cudaError_t launch_qkv_pool(const bsa_params &p, const Dims &D, const void *x, int d_model, const void *w, void *q,
+                            void *k, void *v, float *qbar, float *kbar, float *vbar, int32_t *blk_count,
+                            int32_t *status, cudaStream_t st);
+
 // Extra tokens (E > 0): survivor buffer capacity per row, and the launch.
 int64_t extra_buffer_capacity();
 cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, const void *k,

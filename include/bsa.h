@@ -130,6 +130,24 @@ BSA_API bsa_status bsa_workspace_size(const bsa_params *p, size_t *bytes, int64_
 BSA_API bsa_status bsa_pool(const bsa_params *p, const void *q, const void *k, const void *v,
                     float *qbar, float *kbar, float *vbar, int32_t *blk_count, void *stream);
 
+/* Steps before 1 and 1 in one kernel: the QKV projection with pooling folded
+ * into its epilogue ([STAR] "Sol": a producer with fused preprocessing that
+ * reuses the current input statistics).  [Q | K | V] = X W^T in bf16 with
+ * fp32 accumulation, and the block means of the rounded outputs exactly as
+ * bsa_pool computes them (fp64 sums in token order, rounded once to f32),
+ * without reading Q, K and V back.
+ *   x         : [B, N, d_model] bf16, contiguous (d_model a multiple of 64).
+ *   w_qkv     : [3 * H * d, d_model] bf16, contiguous: the rows of Q's heads,
+ *               then K's, then V's, d rows per head (a linear layer's weight).
+ *   q, k, v   : out [B, N, H, d] bf16 with p's strides.
+ *   qbar, kbar, vbar, blk_count: out, as for bsa_pool.
+ *   ws        : NULL, or a workspace whose status word receives kernel errors.
+ * Needs bf16, H * d a multiple of 256, and a method other than BSA_VSA (cubes
+ * are not runs of tokens); no bias term. */
+BSA_API bsa_status bsa_qkv_pool(const bsa_params *p, const void *x, int32_t d_model, const void *w_qkv,
+                                void *q, void *k, void *v, float *qbar, float *kbar, float *vbar,
+                                int32_t *blk_count, void *ws, void *stream);
+
 /* Step 2, selection ([DOC] "sol-attn inputs" tau, "sla inputs" keep_percent,
  * general inputs extra_tokens).
  *   qbar, kbar  : pooled means from bsa_pool.
