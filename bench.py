@@ -315,6 +315,7 @@ def _config_json(w, world, split="replicas", heads=None):
             "keep_percent": w.keep_percent if w.method == "sla" else None,
             "prefix_len": w.prefix_len, "dense_rows": list(w.dense_rows), "extra_tokens": w.extra_tokens,
             "centroid": w.centroid, "grid": list(w.grid) if w.grid else None,
+            "qk_fp8": bool(getattr(w, "qk_fp8", False)),
             "parallelism": par,
             "l2": "inputs larger than L2 (126 MB); no flush" if 3 * w.B * w.N * w.H * w.d * 2 > 126e6
             else "L2 flushed between steps"}
@@ -407,6 +408,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--heads", type=int, default=0, help="override H (profiling a smaller case)")
+    ap.add_argument("--qk-fp8", action="store_true", help="fine pass with S = Q K^T in fp8 (e4m3)")
     ap.add_argument("--producer", action="store_true",
                     help="time the QKV projection with pooling in its epilogue against cuBLAS + bsa_pool")
     args = ap.parse_args()
@@ -417,6 +419,8 @@ def main():
     w_job = CONFIGS[args.config]
     if args.heads > 0:
         w_job = w_job.replace(H=args.heads)
+    if args.qk_fp8:
+        w_job = w_job.replace(qk_fp8=True)
     split = args.split if world > 1 else "replicas"
     if split == "replicas":
         w_job = rank_workload(w_job, rank, world)
@@ -554,7 +558,7 @@ def main():
         "higher_is_better": True,
         "scaling": "strong" if split == "heads" and world > 1 else "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "dtype": ("bf16 (Q K^T in e4m3)" if w.qk_fp8 else "bf16") if w.dtype == "bf16" else "f32",
         "data": "synthetic (smooth Gaussian-filtered fields + noise, seeded)",
         "config": _config_json(w_job, world, split, [h0, h1]),
         "ms_per_layer": ms_step,

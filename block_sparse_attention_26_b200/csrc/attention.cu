@@ -53,6 +53,8 @@
 
 #include <algorithm>
 
+#include <cuda_fp8.h>
+
 #include "bsa_device.cuh"
 #include "bsa_internal.h"
 
@@ -101,6 +103,8 @@ struct TileInfo {
     float last_bias;      // centroid: log2 of the partial block's size
     int32_t pad;
     uint64_t cmask[2][2]; // centroid / gathered: [query block][half] active columns
+    float ksc[2];         // fp8 Q K^T: scale of each half's keys (1 otherwise)
+    int32_t pad2[2];
 };
 
 struct AttnArgs {
@@ -143,6 +147,9 @@ struct AttnArgs {
     // cube tiling (vsa): positions are in block order (the prefix's 64-token
     // blocks, then the grid's cubes); tiles of cubes come through 5-D maps
     int cube, pre_blocks, P, gH, gW, cT, cH, cW, ncx, ncy;
+    // fp8 Q K^T: scales of Q per 64 tokens, of K per key block, of the centroids per 64
+    const float *sq8, *sk8, *skc8;
+    int nb64, nch64;
 };
 
 // Token of block-order position p (identity without cube tiling).
@@ -172,14 +179,17 @@ __device__ __forceinline__ void load_rows64(uint8_t *dst, const AttnArgs &a, con
     }
 }
 
-template <int D>
+template <int D, bool QK8 = false>
 struct Lay {
-    static constexpr int kQBytes = kM * D * 2;
-    static constexpr int kTileBytes = kTK * D * 2;              // one K or V tile (128 keys)
-    static constexpr int kHalfBytes = kBK * 128;                // one 64-key box of one channel chunk
+    // Q and K tiles hold 1 byte per channel with fp8 Q K^T (QK8), else 2
+    static constexpr int kQKElem = QK8 ? 1 : 2;
+    static constexpr int kQBytes = kM * D * kQKElem;
+    static constexpr int kKTileBytes = kTK * D * kQKElem;       // one K tile (128 keys)
+    static constexpr int kTileBytes = kTK * D * 2;              // one V tile (128 keys)
+    static constexpr int kHalfBytes = kBK * 128;                // one 64-key box of one 128-byte channel chunk
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
-    static constexpr int kOffV = kOffK + kKS * kTileBytes;
+    static constexpr int kOffV = kOffK + kKS * kKTileBytes;
     static constexpr int kOffKind = kOffV + kVS * kTileBytes;
     static constexpr int kOffInfo = kOffKind + 16;
     static constexpr int kOffBar = kOffInfo + kVS * (int)sizeof(TileInfo);
@@ -224,6 +234,28 @@ __device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint64_t adesc, uint6
         "setp.ne.b32 p, %4, 0;\n\t"
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// The same with fp8 (e4m3) operands, K = 32 per instruction.
+__device__ __forceinline__ void umma_ss_f8_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Instruction descriptor, kind::f8f6f4 with e4m3 A and B (K-major) and f32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
+{
+    return (1u << 4)                       // D format f32
+           | (0u << 7)                     // A format e4m3
+           | (0u << 10)                    // B format e4m3
+           | ((uint32_t)(N >> 3) << 17)    // N / 8
+           | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]: A (M x K, bf16 pairs per 32-bit column) from TMEM.
@@ -309,7 +341,7 @@ __device__ __forceinline__ void named_bar(int id, int count)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <int D>
+template <int D, bool QK8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
@@ -319,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tm_k5, const __grid_constant__ CUtensorMap tm_v5,
                 const AttnArgs a)
 {
-    using L = Lay<D>;
+    using L = Lay<D, QK8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~(uintptr_t)1023);
@@ -396,7 +428,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Q first: its load overlaps the rest of the set-up
         prefetch_tmap(&tm_q);
         mbar_expect_tx(bar_q, L::kQBytes);
-        if (a.cube) {
+        if (QK8) {
+            // 128 rows of 128 fp8 channels: one box
+            tma_load_4d(sm + L::kOffQ, &tm_q, bar_q, 0, h, row0, b);
+        } else if (a.cube) {
             // two 64-row blocks (the map's box is 64 rows in this mode)
             for (int dc = 0; dc < D / 64; ++dc)
                 for (int half = 0; half < 2; ++half)
@@ -557,6 +592,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // half x of the tile lands at row offset 64 x of every channel chunk
         const CUtensorMap *tm_x5 = is_k ? &tm_k5 : &tm_v5;
         auto load_half = [&](uint8_t *dst, int kind, int blk, uint64_t *bar) {
+            if (QK8 && is_k) {
+                // 64 keys of 128 fp8 channels: one box
+                if (kind == TILE_EXACT)
+                    tma_load_4d(dst, tm_x, bar, 0, h, blk * kBK, b);
+                else
+                    tma_load_3d(dst, tm_c, bar, 0, blk * kBK, bh);
+                return;
+            }
             for (int dc = 0; dc < D / 64; ++dc) {
                 uint8_t *d = dst + dc * (kTK * 128);
                 if (kind == TILE_EXACT) {
@@ -593,6 +636,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                     TRACE(1, j);
                     for (int x = 0; x < 2; ++x) {
+                        float ksc = 1.f;
+                        if (QK8 && blk[x] >= 0)
+                            ksc = kind == TILE_EXACT ? a.sk8[(int64_t)bh * a.nKB + blk[x]]
+                                                     : a.skc8[(int64_t)bh * a.nch64 + blk[x]];
+                        info[s].ksc[x] = ksc;
                         info[s].blk[x] = blk[x];
                         info[s].h[x].x = kind;
                         info[s].h[x].y = (int32_t)who[x];
@@ -604,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     info[s].last_bias = last_bias;
                 }
             }
-            uint8_t *dst = ring + s * L::kTileBytes;
+            uint8_t *dst = ring + s * (is_k ? L::kKTileBytes : L::kTileBytes);
             if (kind == TILE_GATHER && !is_k)
                 for (int c = lane; c < kTK; c += 32) {
                     // bias 0 for extra tokens, log2 of the remaining count for modified centroids
@@ -667,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (kind == TILE_END) {
                     mbar_arrive(&full[s]);
                 } else {
-                    mbar_expect_tx(&full[s], L::kTileBytes);
+                    mbar_expect_tx(&full[s], is_k ? L::kKTileBytes : L::kTileBytes);
                     load_half(dst, kind, blk[0], &full[s]);
                     load_half(dst + L::kHalfBytes, kind, blk[1], &full[s]);
                 }
@@ -819,6 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The whole warp runs it (warp-uniform operands); one elected lane issues.
         {
             const uint32_t idesc_s = idesc_bf16_f32(kM, kTK, 0, 0);
+            const uint32_t idesc_s8 = idesc_e4m3_f32(kM, kTK);
             const uint32_t idesc_o = idesc_bf16_f32(kM, D, 0, 1);
             const uint32_t q_addr = smem_u32(sm + L::kOffQ);
             const uint32_t k_addr = smem_u32(sm + L::kOffK);
@@ -846,12 +895,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     return false;
                 }
                 if (!a.gather_tma && kind == TILE_GATHER) fence_async_smem();   // rows by cp.async
+                if (QK8) {
+                    // 128 fp8 channels per 128-byte row, 32 per instruction
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd =
-                        sdesc_sw128(k_addr + ks * L::kTileBytes + (kk >> 2) * (kTK * 128) + (kk & 3) * 32, 16, 1024);
-                    umma_ss_w(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 32; ++kk) {
+                        const uint64_t ad = sdesc_sw128(q_addr + kk * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(k_addr + ks * L::kKTileBytes + kk * 32, 16, 1024);
+                        umma_ss_f8_w(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s8, kk > 0 ? 1u : 0u);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(
+                            k_addr + ks * L::kKTileBytes + (kk >> 2) * (kTK * 128) + (kk & 3) * 32, 16, 1024);
+                        umma_ss_w(tmem + kColS + 128 * (ns & 1), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    }
                 }
                 umma_commit_w(&s_full[ns & 1]);
                 if (lane == 0) TRACE(2, ns);
@@ -893,7 +952,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = threadIdx.x & 127;                         // tile row == TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const int qsel = (a.Bq == 64 && !dense) ? (r >> 6) : 0;
-        const float scale = a.scale_log2;
+        // fp8 Q K^T: S is in units of (Q scale of the row's 64 tokens) x (K scale of the half)
+        const float scale_q =
+            QK8 ? a.scale_log2 * a.sq8[(int64_t)bh * a.nb64 + min(row0 + r, a.N - 1) / 64] : a.scale_log2;
         const uint32_t col_o = kColO + 128 * hf;
         uint64_t *pf = p_full + 2 * hf;
         float m_ref = -INFINITY, l = 0.f;
@@ -910,6 +971,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 hq = ti->h[hf];
             const int kind = hq.x;
             if (kind == TILE_END) break;
+            const float scale = QK8 ? scale_q * ti->ksc[hf] : scale_q;
             if (r == 0) TRACE(4 + 3 * hf, j);
             float s[64];
             const uint32_t col_s = kColS + 128 * (j & 1) + 64 * hf;   // this half's S, then its P
@@ -1384,6 +1446,118 @@ __global__ void inputs_to_bf16_kernel(const float *__restrict__ src, __nv_bfloat
     }
 }
 
+// ------------------------------------------------------------------ fp8 Q K^T
+
+// e4m3 copy of 64 rows of one head ([B, N, H, 128] bf16 in, contiguous
+// [B, N, H, 128] fp8 out) with one scale per (b, h, 64-token block): the
+// block's largest |x| maps to 448, the largest finite e4m3 value (scale 1
+// for an all-zero block); x8 = round-to-nearest(x / scale), saturating.
+// One CTA per (b * H + h, block); thread t: row t / 4, channels 32 (t % 4) ...
+__global__ void __launch_bounds__(256) quant_rows_kernel(const __nv_bfloat16 *__restrict__ src, int64_t sb,
+                                                         int64_t sn, int64_t sh, int N, int H, int nb64,
+                                                         uint8_t *__restrict__ dst, float *__restrict__ scale)
+{
+    __shared__ float wmax[8];
+    const int64_t bh = blockIdx.y;
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    const int blk = blockIdx.x;
+    const int row = threadIdx.x >> 2, c0 = 32 * (threadIdx.x & 3);
+    const int n = blk * 64 + row;
+    float x[32];
+    if (n < N) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(src + (int64_t)b * sb + (int64_t)n * sn + (int64_t)h * sh + c0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 w = p[i];
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                x[8 * i + 2 * e] = __uint_as_float(ww[e] << 16);
+                x[8 * i + 2 * e + 1] = __uint_as_float(ww[e] & 0xffff0000u);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(x[e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = wmax[0];
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+    const float sc = m > 0.f ? m / 448.f : 1.f;
+    const float inv = 1.f / sc;
+    if (threadIdx.x == 0) scale[bh * nb64 + blk] = sc;
+    if (n >= N) return;
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * i] * inv, x[4 * i + 1] * inv),
+                                                                 __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+            make_float2(x[4 * i + 2] * inv, x[4 * i + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+        pk[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    uint4 *o = reinterpret_cast<uint4 *>(dst + (((int64_t)b * N + n) * H + h) * 128 + c0);
+    o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
+// e4m3 centroids [BH, nKB, 128] from the f32 means, one scale per 64 centroids.
+__global__ void __launch_bounds__(256) quant_cent_kernel(const float *__restrict__ kbar, int nKB, int nch,
+                                                         uint8_t *__restrict__ dst, float *__restrict__ scale)
+{
+    __shared__ float wmax[8];
+    const int64_t bh = blockIdx.y;
+    const int ch = blockIdx.x;
+    const int row = threadIdx.x >> 2, c0 = 32 * (threadIdx.x & 3);
+    const int j = ch * 64 + row;
+    float x[32];
+    if (j < nKB) {
+        const float4 *p = reinterpret_cast<const float4 *>(kbar + ((int64_t)bh * nKB + j) * 128 + c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 v = p[i];
+            x[4 * i] = v.x;
+            x[4 * i + 1] = v.y;
+            x[4 * i + 2] = v.z;
+            x[4 * i + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = 0.f;
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(x[e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = wmax[0];
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+    const float sc = m > 0.f ? m / 448.f : 1.f;
+    const float inv = 1.f / sc;
+    if (threadIdx.x == 0) scale[bh * nch + ch] = sc;
+    if (j >= nKB) return;
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * i] * inv, x[4 * i + 1] * inv),
+                                                                 __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+            make_float2(x[4 * i + 2] * inv, x[4 * i + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+        pk[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    uint4 *o = reinterpret_cast<uint4 *>(dst + ((int64_t)bh * nKB + j) * 128 + c0);
+    o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
 // ------------------------------------------------------------------ tensor maps
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -1415,6 +1589,34 @@ bool make_map_bnhd(CUtensorMap *m, const void *base, int B, int N, int H, int d,
     cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Bytes (fp8) [B, N, H, d] contiguous; box = 128 channels x 1 head x rows tokens x 1.
+bool make_map_u8_bnhd(CUtensorMap *m, const void *base, int B, int N, int H, int d, int rows)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d, (cuuint64_t)H * d, (cuuint64_t)N * H * d};
+    cuuint32_t box[4] = {128, 1, (cuuint32_t)rows, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Bytes (fp8) [BH, nKB, d] centroids; box = 128 channels x 64 centroids x 1.
+bool make_map_u8_cent(CUtensorMap *m, const void *base, int BH, int nKB, int d)
+{
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)nKB, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)nKB * d};
+    cuuint32_t box[3] = {128, 64, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1467,16 +1669,17 @@ bool make_map_cube(CUtensorMap *m, const void *base, int P, int H, int d, int gT
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool QK8>
 cudaError_t launch_attn_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                const CUtensorMap &tkc, const CUtensorMap &tvc, const CUtensorMap (&tg)[4],
                                const CUtensorMap (&t5)[3], const AttnArgs &a, int64_t items, cudaStream_t st)
 {
-    const size_t smem = Lay<D>::bytes(a.nW);
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = Lay<D, QK8>::bytes(a.nW);
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attn_kernel<D><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, tg[0], tg[1], tg[2], tg[3], t5[0],
-                                                            t5[1], t5[2], a);
+    attn_kernel<D, QK8><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, tg[0], tg[1], tg[2], tg[3],
+                                                                 t5[0], t5[1], t5[2], a);
     return cudaGetLastError();
 }
 
@@ -1554,8 +1757,30 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
         to_bf16_kernel<<<g, 256, 0, st>>>(kbar, kc, n);
         to_bf16_kernel<<<g, 256, 0, st>>>(vbar, vc, n);
     }
+    const bool f8 = p.qk_fp8 != 0;
+    uint8_t *q8 = reinterpret_cast<uint8_t *>(ws + L.q8), *k8 = reinterpret_cast<uint8_t *>(ws + L.k8);
+    uint8_t *kc8 = reinterpret_cast<uint8_t *>(ws + L.kc8);
+    float *sq8 = reinterpret_cast<float *>(ws + L.sq8), *sk8 = reinterpret_cast<float *>(ws + L.sk8);
+    float *skc8 = reinterpret_cast<float *>(ws + L.skc8);
+    const int nb64 = (int)ceil_div(D.N, 64), nch64 = (int)ceil_div(D.nKB, 64);
+    if (f8 && prep) {
+        // Q per 64 tokens, K per key block (also 64 tokens), centroids per 64
+        quant_rows_kernel<<<dim3((unsigned)nb64, (unsigned)BH), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(q16), sb, sn, sh, D.N, D.H, nb64, q8, sq8);
+        quant_rows_kernel<<<dim3((unsigned)nb64, (unsigned)BH), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(k16), sb, sn, sh, D.N, D.H, nb64, k8, sk8);
+        if (use_cent)
+            quant_cent_kernel<<<dim3((unsigned)nch64, (unsigned)BH), 256, 0, st>>>(kbar, D.nKB, nch64, kc8, skc8);
+    }
     CUtensorMap tq, tk, tv, tkc, tvc;
-    if (!make_map_bnhd(&tq, q16, D.B, D.N, D.H, D.d, sb, sn, sh, D.cube ? kBK : kM) ||
+    if (f8) {
+        if (!make_map_u8_bnhd(&tq, q8, D.B, D.N, D.H, D.d, kM) || !make_map_u8_bnhd(&tk, k8, D.B, D.N, D.H, D.d, kBK) ||
+            !make_map_bnhd(&tv, v16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) ||
+            !make_map_u8_cent(&tkc, kc8, BH, D.nKB, D.d) || !make_map_cent(&tvc, vc, BH, D.nKB, D.d)) {
+            set_error("cuTensorMapEncodeTiled failed for the fp8 tiles");
+            return cudaErrorInvalidValue;
+        }
+    } else if (!make_map_bnhd(&tq, q16, D.B, D.N, D.H, D.d, sb, sn, sh, D.cube ? kBK : kM) ||
         !make_map_bnhd(&tk, k16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) ||
         !make_map_bnhd(&tv, v16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) ||
         !make_map_cent(&tkc, kc, BH, D.nKB, D.d) || !make_map_cent(&tvc, vc, BH, D.nKB, D.d)) {
@@ -1576,6 +1801,11 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
         }
     }
     AttnArgs a;
+    a.sq8 = sq8;
+    a.sk8 = sk8;
+    a.skc8 = skc8;
+    a.nb64 = nb64;
+    a.nch64 = nch64;
     a.cube = D.cube;
     a.pre_blocks = D.pre_blocks;
     a.P = p.prefix_len;
@@ -1683,8 +1913,9 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
             }
         }
     }
-    cudaError_t e = D.d == 64 ? launch_attn_kernel<64>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
-                              : launch_attn_kernel<128>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st);
+    cudaError_t e = D.d == 64 ? launch_attn_kernel<64, false>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
+                    : p.qk_fp8  ? launch_attn_kernel<128, true>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
+                                : launch_attn_kernel<128, false>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st);
     if (e != cudaSuccess) return e;
     if (a.n_dense > 0 && a.dense_split > 1) {
         combine_kernel<<<(unsigned)(BH * (int64_t)a.n_dense), kM, 0, st>>>(a, D.d);

@@ -95,6 +95,15 @@ WsLayout ws_layout(const bsa_params &p)
     L.ex_cnt = take(ex ? (size_t)D.rows * 4 : 0);
     L.ex_ovf = take(ex ? (size_t)(D.rows + 1) * 4 : 0);
     L.ex_scratch = take(ex ? (size_t)fallback_ctas() * D.N * 4 : 0);
+    // fp8 Q / K (qk_fp8): e4m3 copies and one scale per 64 tokens (per 64 centroids)
+    const bool f8 = p.qk_fp8 != 0;
+    const size_t ntok = (size_t)D.B * D.N * D.H * D.d;
+    L.q8 = take(f8 ? ntok : 0);
+    L.k8 = take(f8 ? ntok : 0);
+    L.sq8 = take(f8 ? (size_t)BH * ceil_div(D.N, 64) * 4 : 0);
+    L.sk8 = take(f8 ? (size_t)BH * D.nKB * 4 : 0);
+    L.kc8 = take(f8 ? (size_t)BH * D.nKB * D.d : 0);
+    L.skc8 = take(f8 ? (size_t)BH * ceil_div(D.nKB, 64) * 4 : 0);
     L.part_tiles = dense_partial_tiles(D, p.dense_row_end - p.dense_row_begin);
     L.part_o = take((size_t)L.part_tiles * 128 * D.d * sizeof(float));
     L.part_ml = take((size_t)L.part_tiles * 128 * 2 * sizeof(float));
@@ -135,6 +144,11 @@ bsa_status check_params(const bsa_params *p)
     if (isnan(p->tau)) FAIL(BSA_ERR_INVALID_ARG, "tau is NaN");
     if (p->method != BSA_SOL && !(p->keep_percent > 0.0 && p->keep_percent <= 100.0))
         FAIL(BSA_ERR_INVALID_ARG, "keep_percent must be in (0, 100]");
+    if (p->qk_fp8 != 0 && p->qk_fp8 != 1) FAIL(BSA_ERR_INVALID_ARG, "qk_fp8 must be 0 or 1");
+    if (p->qk_fp8) {
+        if (p->dtype != BSA_DT_BF16 || p->d != 128 || p->extra_tokens != 0 || p->method == BSA_VSA)
+            FAIL(BSA_ERR_UNSUPPORTED, "qk_fp8 needs bf16 inputs, d = 128, extra_tokens 0 and method Sol or SLA");
+    }
     if (p->method == BSA_VSA) {
         if (p->q_block != 64) FAIL(BSA_ERR_UNSUPPORTED, "vsa: query cubes hold 64 tokens (q_block 64)");
         if (p->B != 1) FAIL(BSA_ERR_UNSUPPORTED, "vsa: B must be 1");

@@ -83,6 +83,11 @@ struct WsLayout {
     size_t r_fbl;          // [1 + rows] i32 rows for the exact path
     size_t r_fbs;          // [fallback_ctas(), nKBp] f32 exact scores of one row
     int r_nsplit;
+    size_t q8, k8;         // [B, N, H, d] e4m3 copies of Q and K (qk_fp8)
+    size_t sq8;            // [B*H, ceil(N / 64)] f32 scales of Q per 64 tokens
+    size_t sk8;            // [B*H, nKB] f32 scales of K per key block
+    size_t kc8;            // [B*H, nKB, d] e4m3 centroids
+    size_t skc8;           // [B*H, ceil(nKB / 64)] f32 scales of the centroids per 64
     size_t part_o;         // [part_tiles, 128, d] f32 dense-row partial outputs
     size_t part_ml;        // [part_tiles, 128, 2] f32 dense-row partial (max, sum)
     int64_t part_tiles;    // capacity of the partial buffers, in 128-row tiles

@@ -108,6 +108,11 @@ typedef struct {
                                         prefix, flattened t-major (prefix_len + T*Hs*Ws == N) */
     int32_t cube_t, cube_h, cube_w;  /* BSA_VSA: cube extents (4, 4, 4); product 64, each dividing its
                                         grid extent ([DOC] vsa: 3-D video cube tiling) */
+    int32_t qk_fp8;                /* 1: the fine pass takes S = Q K^T in fp8 (e4m3, one scale per 64
+                                      tokens of Q and of K and per 64 centroids), P V in bf16 -- the
+                                      B200 form of [STAR] "attention modes" qk_int8_pv_fp16; needs
+                                      bf16 inputs, d = 128, extra_tokens 0, method Sol or SLA */
+    int32_t reserved_;
 } bsa_params;
 
 /* Fill *p with the defaults of the node documentation for `method`

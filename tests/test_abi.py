@@ -32,12 +32,13 @@ def test_header_declarations_are_exported():
 
 
 def test_params_struct_layout():
-    # int32 x4, int64 x3, int32 x4, double x2, int32 x13 (+4 padding)
-    assert ctypes.sizeof(bsa.bsa_params) == 128
+    # int32 x4, int64 x3, int32 x4, double x2, int32 x15 (+4 padding)
+    assert ctypes.sizeof(bsa.bsa_params) == 136
     assert bsa.bsa_params.tau.offset == 56
     assert bsa.bsa_params.centroid.offset == 96
     assert bsa.bsa_params.grid_t.offset == 100
     assert bsa.bsa_params.cube_w.offset == 120
+    assert bsa.bsa_params.qk_fp8.offset == 124
 
 
 def _p(**kw):

@@ -1,0 +1,72 @@
+"""The fp8 form of the fine pass (qk_fp8: S = Q K^T from e4m3 Q and K with one
+scale per 64 tokens, P V in bf16; "minimax-h3-chunk-star7" README, "attention
+modes", qk_int8_pv_fp16 -- the B200 analogue in fp8) against the CPU oracle's
+exact attention, with the relaxed tolerance FP8_MAX_ABS / FP8_MEAN_ABS.
+
+e4m3 keeps 3 fraction bits (unit roundoff 2^-4, against bf16's 2^-8), so each
+logit moves by up to about 2^-3 * sum_c |q_c k_c| / sqrt(d) in the worst case
+and by roughly 2^-4 * sqrt(2 sum_c (q_c k_c)^2 / 3) / sqrt(d) typically; the
+output moves by about that much times the spread of the attended values.  The
+bars below are the measured errors on these inputs with headroom, about ten
+times the bf16 bars.  Selection does not change (it uses the pooled means), so
+masks are compared bit for bit as for bf16.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.gpu_helpers import compare_masks, csr_to_mask, gpu_layer
+from workloads import CONFIGS, Workload, make_qkv, sample_heads, sample_query_blocks
+
+pytestmark = pytest.mark.gpu
+
+FP8_MAX_ABS = 2e-1
+FP8_MEAN_ABS = 2e-2
+
+CASES = {
+    "fp8_sol": Workload("fp8_sol", B=1, H=2, N=3000, d=128, dtype="bf16", method="sol", q_block=64, k_block=64,
+                        tau=1.3, grid=(3, 20, 50), seed=101, qk_fp8=True),
+    "fp8_sinks": Workload("fp8_sinks", B=1, H=2, N=2120, d=128, dtype="bf16", method="sol", q_block=64, k_block=64,
+                          tau=1.3, prefix_len=200, dense_rows=(72, 200), grid=(3, 16, 40), seed=102, qk_fp8=True),
+    "fp8_sla": Workload("fp8_sla", B=1, H=2, N=2880, d=128, dtype="bf16", method="sla", q_block=128, k_block=64,
+                        keep_percent=15.0, centroid=0, grid=(4, 24, 30), seed=103, qk_fp8=True),
+}
+
+
+def _check(w, q, k, v, toks=None):
+    p, buf, out, status = gpu_layer(w, q, k, v)
+    assert status == 0
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    raw = [oracle.as_raw(t) for t in (qc, kc, vc)]
+    res = oracle.routing(w, *raw)
+    mask = csr_to_mask(buf.row_ptr, buf.col_idx, w.rows, w.nKB)
+    compare_masks(mask, res, w)
+    if toks is None:
+        toks = oracle.all_tokens(w)
+    ref, _ = oracle.layer_rows(w, *raw, res, toks)
+    got = out[toks[:, 0], toks[:, 2], toks[:, 1]].float().cpu().numpy()
+    err = np.abs(got.astype(np.float64) - ref)
+    print(f"{w.name}: fp8 max abs err {err.max():.3e}, mean {err.mean():.3e}")
+    assert np.isfinite(got).all()
+    assert err.max() <= FP8_MAX_ABS and err.mean() <= FP8_MEAN_ABS, (err.max(), err.mean())
+    return err
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_fp8_matches_oracle_within_relaxed_tolerance(name):
+    w = CASES[name]
+    q, k, v = (t.cuda() for t in make_qkv(w, "cpu"))
+    _check(w, q, k, v)
+
+
+def test_fp8_full_size_sampled():
+    w = CONFIGS["sol_mid"].replace(qk_fp8=True)
+    q, k, v = make_qkv(w, "cuda")
+    g = np.random.default_rng(5)
+    toks = []
+    for h in sample_heads(w):
+        for i in sample_query_blocks(w, 32):
+            lo, hi = i * w.q_block, min(w.N, (i + 1) * w.q_block)
+            toks += [(0, h, int(n)) for n in sorted({lo, hi - 1} | set(g.integers(lo, hi, 6).tolist()))]
+    _check(w, q, k, v, np.array(toks, np.int64))

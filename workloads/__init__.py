@@ -50,6 +50,7 @@ class Workload:
     centroid: int = 1
     grid: Optional[Tuple[int, int, int]] = None   # latent grid (T, Hs, Ws); None = iid tokens
     cube: Tuple[int, int, int] = (4, 4, 4)         # vsa: cube extents (t, y, x)
+    qk_fp8: bool = False                           # fine pass with S = Q K^T in fp8 (e4m3)
     seed: int = 0
     field_sigma: float = 4.0
     noise: float = 0.5
