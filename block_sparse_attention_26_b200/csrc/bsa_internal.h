@@ -78,8 +78,6 @@ struct WsLayout {
     size_t r_cov;          // [B*H, d, d] f64 centred second moments
     size_t r_hstat;        // [B*H, d + 3] f64 mean key, tr(G)/n, |m|^2, max |kbar|
     size_t r_info;         // [rows] RowInfo
-    size_t r_ulist;        // [rows, kUcap] i32 blocks left undecided
-    size_t r_ucnt;         // [rows] i32 their count
     size_t r_fbl;          // [1 + rows] i32 rows for the exact path
     size_t r_fbs;          // [fallback_ctas(), nKBp] f32 exact scores of one row
     int r_nsplit;

@@ -30,9 +30,9 @@
 //                       the accumulation).  A block whose score interval lies
 //                       wholly above the threshold interval is kept, wholly
 //                       below it dropped; the few others (about 9 of 3248 per
-//                       row on the long workload) are listed.
-//   exact               the listed blocks' S_b exactly as the definition
-//                       computes them; decided against [thr_lo, thr_hi].  A
+//                       row on the long workload) are listed and, at the end
+//                       of the CTA, get their S_b exactly as the definition
+//                       computes them, decided against [thr_lo, thr_hi].  A
 //                       row with a block inside that interval, more listed
 //                       blocks than the list holds, or a std that may be zero
 //                       goes to
@@ -71,7 +71,7 @@ struct RouteArgs {
     float *knmax;     // [BH, nKBp / 32] largest norm of each 32-block word
     double *gram, *ksum, *cov, *hstat;   // hstat: [BH, d + 3]
     RowInfo *info;
-    int32_t *ulist, *ucnt, *fbl;
+    int32_t *fbl;
     float *fbs;
     uint32_t *bitmask;
     int32_t *count;
@@ -243,13 +243,15 @@ __device__ __forceinline__ float block_max(float v)
 
 // Per head: m = s / n, C = G / n - m m^T, and the scalars tr(G)/n, |m|^2 and
 // the largest key-centroid norm (hstat[bh] = {m[0..D), tr(G)/n, |m|^2, max
-// |kbar_b|}).  Partials are added in split order.
+// |kbar_b|}).  Partials are added in split order.  Grid (D * D / 256, BH): CTA x
+// takes entries 256 x .. 256 x + 255 of C (each CTA forms m itself); CTA 0 of a
+// head also writes hstat.
 template <int D>
 __global__ void __launch_bounds__(256) gram_reduce_kernel(RouteArgs a)
 {
     __shared__ double m[D];
     __shared__ double diag[D];
-    const int64_t bh = blockIdx.x;
+    const int64_t bh = blockIdx.y;
     const double n = (double)a.nKB;
     for (int c = threadIdx.x; c < D; c += blockDim.x) {
         double s = 0.0;
@@ -258,7 +260,8 @@ __global__ void __launch_bounds__(256) gram_reduce_kernel(RouteArgs a)
     }
     __syncthreads();
     double *cov = a.cov + bh * D * D;
-    for (int idx = threadIdx.x; idx < D * D; idx += blockDim.x) {
+    {
+        const int idx = blockIdx.x * 256 + threadIdx.x;
         const int r = idx / D, c = idx % D;
         // only the tiles on and above the diagonal of 64 x 64 blocks were computed
         const int src = (r >> 6) > (c >> 6) ? c * D + r : idx;
@@ -266,9 +269,13 @@ __global__ void __launch_bounds__(256) gram_reduce_kernel(RouteArgs a)
         for (int sp = 0; sp < a.nsplit; ++sp) g += a.gram[(bh * a.nsplit + sp) * D * D + src];
         g /= n;
         cov[idx] = g - m[r] * m[c];
-        if (r == c) diag[r] = g;
     }
-    __syncthreads();
+    if (blockIdx.x != 0) return;
+    for (int c = threadIdx.x; c < D; c += blockDim.x) {
+        double g = 0.0;
+        for (int sp = 0; sp < a.nsplit; ++sp) g += a.gram[(bh * a.nsplit + sp) * D * D + c * D + c];
+        diag[c] = g / n;
+    }
     float kmax = 0.f;
     for (int j = threadIdx.x; j < a.nKB; j += blockDim.x) kmax = fmaxf(kmax, a.knorm[bh * a.nKBp + j]);
     kmax = block_max(kmax);
@@ -422,6 +429,85 @@ __global__ void __launch_bounds__(D * 4) rowstat_kernel(RouteArgs a)
     }
 }
 
+// ------------------------------------------------------------------ exact scores
+
+// S_b exactly as the definition computes it: fp64 FMA per channel in channel
+// order from 0, divided by sqrt(d) in fp64, rounded to f32.  The chain is
+// serial; the key row is loaded 32 values ahead of it.
+template <int D, typename QT>
+__device__ __forceinline__ float exact_score(const QT *qd, const float *k, double rs)
+{
+    constexpr int CH = 8;              // float4 per chunk (32 values)
+    constexpr int NCH = D / (4 * CH);
+    const float4 *k4 = reinterpret_cast<const float4 *>(k);
+    float4 cur[CH], nxt[CH];
+#pragma unroll
+    for (int e = 0; e < CH; ++e) cur[e] = __ldg(k4 + e);
+    double acc = 0.0;
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+        if (ch + 1 < NCH) {
+#pragma unroll
+            for (int e = 0; e < CH; ++e) nxt[e] = __ldg(k4 + (ch + 1) * CH + e);
+        }
+#pragma unroll
+        for (int e = 0; e < CH; ++e) {
+            const int c = 4 * (ch * CH + e);
+            acc = __fma_rn((double)qd[c], (double)cur[e].x, acc);
+            acc = __fma_rn((double)qd[c + 1], (double)cur[e].y, acc);
+            acc = __fma_rn((double)qd[c + 2], (double)cur[e].z, acc);
+            acc = __fma_rn((double)qd[c + 3], (double)cur[e].w, acc);
+        }
+        if (ch + 1 < NCH) {
+#pragma unroll
+            for (int e = 0; e < CH; ++e) cur[e] = nxt[e];
+        }
+    }
+    return __double2float_rn(__ddiv_rn(acc, rs));
+}
+
+// Two of them at once (independent chains, one instruction stream).
+template <int D>
+__device__ __forceinline__ void exact_score2(const float *q, const float *k0, const float *k1, double rs, float *s0,
+                                             float *s1)
+{
+    const float4 *a4 = reinterpret_cast<const float4 *>(k0);
+    const float4 *b4 = reinterpret_cast<const float4 *>(k1);
+    const float4 *q4 = reinterpret_cast<const float4 *>(q);
+    double x = 0.0, y = 0.0;
+    float4 ka = __ldg(a4), kb = __ldg(b4);
+#pragma unroll 4
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 na = c4 + 1 < D / 4 ? __ldg(a4 + c4 + 1) : ka;
+        const float4 nb = c4 + 1 < D / 4 ? __ldg(b4 + c4 + 1) : kb;
+        const float4 qv = q4[c4];
+        x = __fma_rn((double)qv.x, (double)ka.x, x);
+        y = __fma_rn((double)qv.x, (double)kb.x, y);
+        x = __fma_rn((double)qv.y, (double)ka.y, x);
+        y = __fma_rn((double)qv.y, (double)kb.y, y);
+        x = __fma_rn((double)qv.z, (double)ka.z, x);
+        y = __fma_rn((double)qv.z, (double)kb.z, y);
+        x = __fma_rn((double)qv.w, (double)ka.w, x);
+        y = __fma_rn((double)qv.w, (double)kb.w, y);
+        ka = na;
+        kb = nb;
+    }
+    *s0 = __double2float_rn(__ddiv_rn(x, rs));
+    *s1 = __double2float_rn(__ddiv_rn(y, rs));
+}
+
+template <typename QT>
+__device__ __forceinline__ float exact_score_d(const QT *qd, const float *k, int d, double rs)
+{
+    return d == 128 ? exact_score<128>(qd, k, rs) : exact_score<64>(qd, k, rs);
+}
+
+__device__ __forceinline__ void push_fallback(const RouteArgs &a, int64_t r)
+{
+    const int pos = atomicAdd(&a.fbl[0], 1);
+    a.fbl[1 + pos] = (int32_t)r;
+}
+
 // ------------------------------------------------------------------ decide
 
 template <int D>
@@ -433,9 +519,11 @@ struct DLay {
     static constexpr int kOffK = kQBytes;
     static constexpr int kOffBar = kOffK + kStages * kKBytes;   // k_full[S], k_empty[S], s_full[2], s_free[2], done
     static constexpr int kOffMisc = kOffBar + (2 * kStages + 5) * 8;
-    static constexpr int kOffUcnt = kOffMisc + 16;             // [kTM] i32
-    static constexpr size_t bytes = (size_t)kOffUcnt + kTM * 4 + 1024;
-    static_assert(bytes <= 232448, "decide tile exceeds the per-block shared memory limit");
+    static constexpr int kOffUcnt = kOffMisc + 16;             // [kTM] i32 undecided blocks per row
+    static constexpr int kOffAmb = kOffUcnt + kTM * 4;         // [kTM] i32 a row's exact pass was inconclusive
+    static constexpr int kOffUl = kOffAmb + kTM * 4;           // [kTM][kUcap] u16 the undecided blocks
+    static constexpr int kOffKx = kOffUl + kTM * kUcap * 2;    // [nKBp / 32] f32 largest key norm per word
+    static size_t bytes(int nwp) { return (size_t)kOffKx + (size_t)nwp * 4 + 1024; }
 };
 
 // Warps 0-7 read the scores (warp w: TMEM lane quarter w & 3, columns 64 (w >> 2)
@@ -458,6 +546,9 @@ __global__ void __launch_bounds__(320, 1) decide_kernel(const __grid_constant__ 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kOffMisc);
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(sm + L::kOffMisc + 4);
     int32_t *ucnt_s = reinterpret_cast<int32_t *>(sm + L::kOffUcnt);
+    int32_t *amb_s = reinterpret_cast<int32_t *>(sm + L::kOffAmb);
+    uint16_t *ul_s = reinterpret_cast<uint16_t *>(sm + L::kOffUl);
+    float *kx_s = reinterpret_cast<float *>(sm + L::kOffKx);
 
     const int r = threadIdx.x & (kTM - 1);
     const bool live = i0 + r < a.nQB;
@@ -494,6 +585,10 @@ __global__ void __launch_bounds__(320, 1) decide_kernel(const __grid_constant__ 
         }
         fence_async_smem();
         ucnt_s[r] = 0;
+        amb_s[r] = 0;
+    } else if (warp < 8) {
+        const float *src = a.knmax + (int64_t)bh * (a.nKBp / 32);
+        for (int i = threadIdx.x - 128; i < a.nKBp / 32; i += 128) kx_s[i] = src[i];
     }
     tc_fence_before();
     __syncthreads();
@@ -549,9 +644,8 @@ __global__ void __launch_bounds__(320, 1) decide_kernel(const __grid_constant__ 
         const Forced fo = forced_of(a, min(i0 + r, a.nQB - 1));
         const float inv_rs = (float)(1.0 / sqrt((double)D));
         const float *kn_head = a.knorm + (int64_t)bh * a.nKBp;
-        const float *kx_head = a.knmax + (int64_t)bh * (a.nKBp / 32);
         uint32_t *bm = a.bitmask + row * a.nW;
-        int32_t *ul = a.ulist + row * kUcap;
+        uint16_t *ul = ul_s + r * kUcap;
         const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
         for (int t = 0; t < ntiles; ++t) {
             const int sb = t & 1;
@@ -583,7 +677,7 @@ __global__ void __launch_bounds__(320, 1) decide_kernel(const __grid_constant__ 
                 // word-wide bounds from the word's largest key norm: every block of
                 // the word has l_b >= lmin and u_b <= umax, so most scores are
                 // decided by two compares; the rest get their own bounds
-                const float kmx = __ldg(kx_head + wi);
+                const float kmx = kx_s[wi];
                 const float lmin = fmaf(-info.c, kmx, info.lo);
                 const float umax = fmaf(info.c, kmx, info.hi);
                 uint32_t kw = 0u, slow = 0u;
@@ -608,12 +702,58 @@ __global__ void __launch_bounds__(320, 1) decide_kernel(const __grid_constant__ 
                 bm[wi] = kw & valid;
                 for (uint32_t m = uw; m != 0u; m &= m - 1u) {
                     const int pos = atomicAdd(&ucnt_s[r], 1);
-                    if (pos < kUcap) ul[pos] = 32 * wi + __ffs(m) - 1;
+                    if (pos < kUcap) ul[pos] = (uint16_t)(32 * wi + __ffs(m) - 1);
                 }
             }
         }
         named_bar_sync(1, 256);
-        if (g == 0 && live) a.ucnt[row] = info.mode == 0 ? ucnt_s[r] : kUcap + 1;
+        // The undecided blocks' scores exactly as the definition computes them
+        // (the two threads of a row take alternate entries), decided against
+        // [thr_lo, thr_hi]; a row with an inconclusive block, more undecided
+        // blocks than the list holds, or mode 1 goes to the exact path.  The
+        // rows' f32 queries are staged in the K ring, idle once every tile has
+        // been read (the MMA warp's last S is in registers by now).
+        float *qs = reinterpret_cast<float *>(sm + L::kOffK);   // [kTM][D + 4]
+        constexpr int QP = D + 4;
+        for (int idx = threadIdx.x; idx < kTM * D / 4; idx += 256) {
+            const int rr = idx / (D / 4), c4 = idx % (D / 4);
+            const float4 v = i0 + rr < a.nQB
+                                 ? *reinterpret_cast<const float4 *>(a.qbar + ((int64_t)bh * a.nQB + i0 + rr) * D + 4 * c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(qs + rr * QP + 4 * c4) = v;
+        }
+        named_bar_sync(1, 256);
+        if (live) {
+            const int u = ucnt_s[r];
+            if (info.mode != 0 || u > kUcap) {
+                if (g == 0) push_fallback(a, row);
+            } else {
+                const float *qrow = qs + r * QP;
+                const float *kb = a.kbar + (int64_t)bh * a.nKB * D;
+                const double rs = sqrt((double)D);
+                bool amb = false;
+                auto decide1 = [&](int j, float sv) {
+                    if (sv > info.thr_hi)
+                        atomicOr(&bm[j >> 5], 1u << (j & 31));
+                    else if (!(sv <= info.thr_lo))
+                        amb = true;
+                };
+                int idx = g;
+                for (; idx + 2 < u; idx += 4) {
+                    // two independent chains side by side
+                    const int j0 = ul[idx], j1 = ul[idx + 2];
+                    float s0, s1;
+                    exact_score2<D>(qrow, kb + (int64_t)j0 * D, kb + (int64_t)j1 * D, rs, &s0, &s1);
+                    decide1(j0, s0);
+                    decide1(j1, s1);
+                }
+                for (; idx < u; idx += 2) {
+                    const int j = ul[idx];
+                    decide1(j, exact_score<D>(qrow, kb + (int64_t)j * D, rs));
+                }
+                if (amb && atomicExch(&amb_s[r], 1) == 0) push_fallback(a, row);
+            }
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -625,112 +765,6 @@ __global__ void __launch_bounds__(320, 1) decide_kernel(const __grid_constant__ 
 
 // ------------------------------------------------------------------ exact
 
-// S_b exactly as the definition computes it: fp64 FMA per channel in channel
-// order from 0, divided by sqrt(d) in fp64, rounded to f32.  The chain is
-// serial; the key row is loaded 32 values ahead of it.
-template <int D>
-__device__ __forceinline__ float exact_score(const double *qd, const float *k, double rs)
-{
-    constexpr int CH = 8;              // float4 per chunk (32 values)
-    constexpr int NCH = D / (4 * CH);
-    const float4 *k4 = reinterpret_cast<const float4 *>(k);
-    float4 cur[CH], nxt[CH];
-#pragma unroll
-    for (int e = 0; e < CH; ++e) cur[e] = __ldg(k4 + e);
-    double acc = 0.0;
-#pragma unroll
-    for (int ch = 0; ch < NCH; ++ch) {
-        if (ch + 1 < NCH) {
-#pragma unroll
-            for (int e = 0; e < CH; ++e) nxt[e] = __ldg(k4 + (ch + 1) * CH + e);
-        }
-#pragma unroll
-        for (int e = 0; e < CH; ++e) {
-            const int c = 4 * (ch * CH + e);
-            acc = __fma_rn(qd[c], (double)cur[e].x, acc);
-            acc = __fma_rn(qd[c + 1], (double)cur[e].y, acc);
-            acc = __fma_rn(qd[c + 2], (double)cur[e].z, acc);
-            acc = __fma_rn(qd[c + 3], (double)cur[e].w, acc);
-        }
-        if (ch + 1 < NCH) {
-#pragma unroll
-            for (int e = 0; e < CH; ++e) cur[e] = nxt[e];
-        }
-    }
-    return __double2float_rn(__ddiv_rn(acc, rs));
-}
-
-__device__ __forceinline__ float exact_score_d(const double *qd, const float *k, int d, double rs)
-{
-    return d == 128 ? exact_score<128>(qd, k, rs) : exact_score<64>(qd, k, rs);
-}
-
-__device__ __forceinline__ void push_fallback(const RouteArgs &a, int64_t r)
-{
-    const int pos = atomicAdd(&a.fbl[0], 1);
-    a.fbl[1 + pos] = (int32_t)r;
-}
-
-// The listed blocks' exact scores against [thr_lo, thr_hi]: one CTA per 32
-// rows, its 256 threads spread over all the rows' entries.
-constexpr int kExactRows = 32;
-
-__global__ void __launch_bounds__(256) exact_kernel(RouteArgs a)
-{
-    __shared__ double qs[kExactRows][128];
-    __shared__ int pref[kExactRows + 1];
-    __shared__ float tlo[kExactRows], thi[kExactRows];
-    __shared__ int amb[kExactRows];
-    const int64_t r0 = (int64_t)blockIdx.x * kExactRows;
-    const int nr = (int)(a.rows - r0 < kExactRows ? a.rows - r0 : kExactRows);
-    if (threadIdx.x < 32) {
-        const int i = threadIdx.x;
-        int u = 0;
-        if (i < nr) {
-            const RowInfo info = a.info[r0 + i];
-            u = a.ucnt[r0 + i];
-            if (info.mode != 0 || u > kUcap) {
-                push_fallback(a, r0 + i);
-                u = 0;
-            }
-            tlo[i] = info.thr_lo;
-            thi[i] = info.thr_hi;
-        }
-        amb[i] = 0;
-        int incl = u;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (i >= o) incl += y;
-        }
-        pref[i + 1] = incl;
-        if (i == 0) pref[0] = 0;
-    }
-    for (int idx = threadIdx.x; idx < nr * a.d; idx += blockDim.x) {
-        const int i = idx / a.d, c = idx % a.d;
-        qs[i][c] = (double)a.qbar[(r0 + i) * a.d + c];
-    }
-    __syncthreads();
-    const int total = pref[kExactRows];
-    const double rs = sqrt((double)a.d);
-    for (int t = threadIdx.x; t < total; t += blockDim.x) {
-        int i = 0;
-#pragma unroll
-        for (int step = 16; step > 0; step >>= 1)
-            if (pref[i + step] <= t) i += step;
-        const int64_t r = r0 + i;
-        const int j = a.ulist[r * kUcap + (t - pref[i])];
-        const int64_t bh = r / a.nQB;
-        const float s = exact_score_d(qs[i], a.kbar + (bh * a.nKB + j) * a.d, a.d, rs);
-        if (s > thi[i])
-            atomicOr(&a.bitmask[r * a.nW + (j >> 5)], 1u << (j & 31));
-        else if (!(s <= tlo[i]))
-            amb[i] = 1;
-    }
-    __syncthreads();
-    if (threadIdx.x < nr && amb[threadIdx.x]) push_fallback(a, r0 + threadIdx.x);
-}
-
 // ------------------------------------------------------------------ fallback
 
 // Rows whose threshold could not be bracketed tightly enough: every score
@@ -740,39 +774,78 @@ __global__ void __launch_bounds__(256) exact_kernel(RouteArgs a)
 // the CTA's global scratch row.
 constexpr int kFbSmem = 16384;
 
-__global__ void __launch_bounds__(256) fallback_rows_kernel(RouteArgs a)
+__global__ void __launch_bounds__(512) fallback_rows_kernel(RouteArgs a)
 {
     extern __shared__ float fb_smem[];
     __shared__ double qd[128];
     __shared__ float thr_s;
     __shared__ int keep_s;
+    __shared__ double red_d[16], red_s[16];
+    __shared__ int red_i[16];
     const int nfb = a.fbl[0];
     float *srow = a.nKBp <= kFbSmem ? fb_smem : a.fbs + (int64_t)blockIdx.x * a.nKBp;
     const double rs = sqrt((double)a.d);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int f = blockIdx.x; f < nfb; f += gridDim.x) {
         const int64_t r = a.fbl[1 + f];
         const int64_t bh = r / a.nQB;
         __syncthreads();
         for (int c = threadIdx.x; c < a.d; c += blockDim.x) qd[c] = (double)a.qbar[r * a.d + c];
         __syncthreads();
-        for (int j = threadIdx.x; j < a.nKB; j += blockDim.x)
-            srow[j] = exact_score_d(qd, a.kbar + (bh * a.nKB + j) * a.d, a.d, rs);
+        // every score exactly, and in the same pass the smallest exponent of a
+        // nonzero score and the sum of |score| (for the exactness test below)
+        int emin = 1 << 20;
+        double sabs = 0.0, ssum = 0.0;
+        for (int j = threadIdx.x; j < a.nKB; j += blockDim.x) {
+            const float sv = exact_score_d(qd, a.kbar + (bh * a.nKB + j) * a.d, a.d, rs);
+            srow[j] = sv;
+            if (sv != 0.f) emin = min(emin, ilogbf(sv));
+            sabs += fabs((double)sv);
+            ssum += (double)sv;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
+            sabs += __shfl_xor_sync(0xffffffffu, sabs, o);
+            ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+        }
+        if (lane == 0) {
+            red_i[warp] = emin;
+            red_d[warp] = sabs;
+            red_s[warp] = ssum;
+        }
         __syncthreads();
         if (threadIdx.x == 0) {
+            const int nwarp = (int)(blockDim.x >> 5);
+            int e = red_i[0];
+            double sa = red_d[0];
+            for (int w = 1; w < nwarp; ++w) {
+                e = min(e, red_i[w]);
+                sa += red_d[w];
+            }
+            // Every score is a multiple of 2^(e - 23).  If the sum of |scores|
+            // stays below 2^(e - 23 + 53) (here with a factor 2 to spare), every
+            // partial sum in any order is exactly representable in fp64, so the
+            // definition's sequential sum equals a sum in any order.
+            const bool exact_sum = e == (1 << 20) || sa < ldexp(1.0, e - 23 + 52);
             const int n = a.nKB;
             double mu = 0.0;
-            int j = 0;
-            for (; j + 8 <= n; j += 8) {
-                float v[8];
+            if (exact_sum) {
+                for (int w = 0; w < nwarp; ++w) mu += red_s[w];
+            } else {
+                int j = 0;
+                for (; j + 8 <= n; j += 8) {
+                    float v[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = srow[j + e];
+                    for (int e = 0; e < 8; ++e) v[e] = srow[j + e];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mu = __dadd_rn(mu, (double)v[e]);
+                    for (int e = 0; e < 8; ++e) mu = __dadd_rn(mu, (double)v[e]);
+                }
+                for (; j < n; ++j) mu = __dadd_rn(mu, (double)srow[j]);
             }
-            for (; j < n; ++j) mu = __dadd_rn(mu, (double)srow[j]);
             mu = __ddiv_rn(mu, (double)n);
             double var = 0.0;
-            j = 0;
+            int j = 0;
             for (; j + 8 <= n; j += 8) {
                 double e2[8];
 #pragma unroll
@@ -859,7 +932,7 @@ cudaError_t launch_route_d(const RouteArgs &a, cudaStream_t st)
     route_prep_kernel<<<(unsigned)ceil_div(BH * a.nKBp, 8), 256, 0, st>>>(a);
     knmax_kernel<<<(unsigned)ceil_div(BH * (a.nKBp / 32), 256), 256, 0, st>>>(a);
     gram_kernel<D><<<dim3((unsigned)(a.nsplit * (D == 128 ? 3 : 1)), (unsigned)BH), 256, 0, st>>>(a);
-    gram_reduce_kernel<D><<<(unsigned)BH, 256, 0, st>>>(a);
+    gram_reduce_kernel<D><<<dim3(D * D / 256, (unsigned)BH), 256, 0, st>>>(a);
     const int rs_smem = D * D * 8 + D * kTM * 4 + (D + 3) * 8;
     cudaError_t e = cudaFuncSetAttribute(rowstat_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, rs_smem);
     if (e != cudaSuccess) return e;
@@ -870,18 +943,21 @@ cudaError_t launch_route_d(const RouteArgs &a, cudaStream_t st)
         set_error("cuTensorMapEncodeTiled failed for the routing scores");
         return cudaErrorInvalidValue;
     }
-    const int bytes = (int)DLay<D>::bytes;
+    const int bytes = (int)DLay<D>::bytes(a.nKBp / 32);
+    if (bytes > 232448) {
+        set_error("routing: too many key blocks for the score tiles' shared memory");
+        return cudaErrorInvalidValue;
+    }
     e = cudaFuncSetAttribute(decide_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     decide_kernel<D><<<gt, 320, bytes, st>>>(tm, a);
     const unsigned g8 = (unsigned)ceil_div(a.rows, 8);
-    exact_kernel<<<(unsigned)ceil_div(a.rows, kExactRows), 256, 0, st>>>(a);
     const int fb_smem = a.nKBp <= kFbSmem ? a.nKBp * 4 : 0;
     if (fb_smem > 48 * 1024) {
         e = cudaFuncSetAttribute(fallback_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fb_smem);
         if (e != cudaSuccess) return e;
     }
-    fallback_rows_kernel<<<(unsigned)fallback_ctas(), 256, fb_smem, st>>>(a);
+    fallback_rows_kernel<<<(unsigned)fallback_ctas(), 512, fb_smem, st>>>(a);
     route_count_kernel<<<g8, 256, 0, st>>>(a);
     return cudaGetLastError();
 }
@@ -922,8 +998,6 @@ cudaError_t launch_route(const bsa_params &p, const Dims &D, const float *qbar, 
     a.cov = reinterpret_cast<double *>(ws + L.r_cov);
     a.hstat = reinterpret_cast<double *>(ws + L.r_hstat);
     a.info = reinterpret_cast<RowInfo *>(ws + L.r_info);
-    a.ulist = reinterpret_cast<int32_t *>(ws + L.r_ulist);
-    a.ucnt = reinterpret_cast<int32_t *>(ws + L.r_ucnt);
     a.fbl = reinterpret_cast<int32_t *>(ws + L.r_fbl);
     a.fbs = reinterpret_cast<float *>(ws + L.r_fbs);
     a.bitmask = reinterpret_cast<uint32_t *>(ws + L.bitmask);

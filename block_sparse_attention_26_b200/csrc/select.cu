@@ -324,6 +324,11 @@ cudaError_t launch_scan(const int32_t *cnt, int64_t rows, int64_t *row_ptr, int6
     return cudaGetLastError();
 }
 
+// One warp per row, its words 32 at a time: every lane counts its word's bits
+// and a warp scan gives every word its first output slot.  A sparse word (at
+// most 4 bits) is written by its own lane, a bit per step; a dense word (the
+// kept blocks near the diagonal) by the whole warp at once, lane l testing bit
+// l -- so a few dense words do not hold the other lanes for 32 steps.
 __global__ void __launch_bounds__(256) expand_kernel(const uint32_t *__restrict__ bitmask,
                                                      const int32_t *__restrict__ count,
                                                      const int64_t *__restrict__ row_ptr,
@@ -332,6 +337,7 @@ __global__ void __launch_bounds__(256) expand_kernel(const uint32_t *__restrict_
                                                      int32_t *__restrict__ kept_count,
                                                      int32_t *status)
 {
+    constexpr int kSparse = 4;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * 8 + warp;
     if (r >= rows) return;
@@ -341,10 +347,11 @@ __global__ void __launch_bounds__(256) expand_kernel(const uint32_t *__restrict_
         if (start + count[r] > capacity) report(status, BSA_DEV_CAPACITY, (int32_t)(r & 0x7fffffff));
     }
     const uint32_t *bm = bitmask + r * nW;
+    const uint32_t lt = (1u << lane) - 1u;
     int64_t base = start;
     for (int w0 = 0; w0 < nW; w0 += 32) {
         const int w = w0 + lane;
-        uint32_t word = w < nW ? bm[w] : 0u;
+        const uint32_t word = w < nW ? bm[w] : 0u;
         const int pc = __popc(word);
         int incl = pc;
 #pragma unroll
@@ -352,12 +359,22 @@ __global__ void __launch_bounds__(256) expand_kernel(const uint32_t *__restrict_
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        int64_t pos = base + (incl - pc);
-        while (word) {
-            const int bit = __ffs(word) - 1;
-            word &= word - 1;
-            if (pos < capacity) col[pos] = w * 32 + bit;
-            ++pos;
+        const int64_t first = base + (incl - pc);
+        // sparse words: each lane its own
+        if (pc <= kSparse) {
+            int64_t pos = first;
+            for (uint32_t m = word; m != 0u; m &= m - 1u, ++pos)
+                if (pos < capacity) col[pos] = w * 32 + __ffs(m) - 1;
+        }
+        // dense words: the warp takes them one by one
+        for (uint32_t dense = __ballot_sync(0xffffffffu, pc > kSparse); dense != 0u; dense &= dense - 1u) {
+            const int src = __ffs(dense) - 1;
+            const uint32_t wd = __shfl_sync(0xffffffffu, word, src);
+            const int64_t f = __shfl_sync(0xffffffffu, first, src);
+            if ((wd >> lane) & 1u) {
+                const int64_t pos = f + __popc(wd & lt);
+                if (pos < capacity) col[pos] = (w0 + src) * 32 + lane;
+            }
         }
         base += __shfl_sync(0xffffffffu, incl, 31);
     }
@@ -388,8 +405,6 @@ void select_regions(const bsa_params &p, const Dims &D, WsLayout &L, Taker &T)
     L.r_cov = T.take(route ? (size_t)BH * d * d * 8 : 0);
     L.r_hstat = T.take(route ? (size_t)BH * (d + 3) * 8 : 0);
     L.r_info = T.take(route ? rows * sizeof(RowInfo) : 0);
-    L.r_ulist = T.take(route ? rows * kUcap * 4 : 0);
-    L.r_ucnt = T.take(route ? rows * 4 : 0);
     L.r_fbl = T.take(route ? (rows + 1) * 4 : 0);
     L.r_fbs = T.take(route ? (size_t)fallback_ctas() * route_nkbp(D) * 4 : 0);
 }

@@ -173,8 +173,9 @@ def test_sigma_zero_rows_keep_only_forced():
 # definition's bit for bit, with no near-threshold exemption.  The cases below
 # also push rows onto the route's exact paths: keys that are nearly identical
 # (every block undecided by the tensor-core scores: list overflow, exact
-# fallback rows), and pooled values scaled far up or down (bounds near the ends
-# of the f32 range).
+# fallback rows), pooled values scaled far up or down (bounds near the ends of
+# the f32 range), and one enormous key block (rows sent to the exact path, with
+# scores whose fp64 sum depends on its order).
 ROUTE = {
     "near_identical_keys": Workload("near_identical_keys", B=1, H=2, N=3000, d=128, dtype="bf16", method="sol",
                                     q_block=64, k_block=64, tau=1.0, grid=(3, 20, 50), seed=31),
@@ -182,6 +183,8 @@ ROUTE = {
                             k_block=64, tau=1.3, grid=(2, 25, 50), seed=32),
     "tiny_scale": Workload("tiny_scale", B=1, H=2, N=2500, d=64, dtype="bf16", method="sol", q_block=64,
                            k_block=64, tau=0.7, grid=(2, 25, 50), seed=33),
+    "huge_block": Workload("huge_block", B=1, H=2, N=2500, d=128, dtype="bf16", method="sol", q_block=64,
+                           k_block=64, tau=1.3, grid=(2, 25, 50), seed=35),
     "negative_tau": Workload("negative_tau", B=1, H=2, N=2970, d=128, dtype="bf16", method="sol", q_block=64,
                              k_block=64, tau=-0.6, prefix_len=130, grid=(2, 20, 71), seed=34),
 }
@@ -198,6 +201,12 @@ def _route_inputs(name, w):
     elif name == "tiny_scale":
         q = q * 2.0 ** -120
         k = k * 2.0 ** -4
+    elif name == "huge_block":
+        # one key block of head 0 at 2^110: the tensor-core products could
+        # overflow, so every row of that head takes the exact path, whose scores
+        # then span far more than fp64 can sum exactly in any order
+        k = k.clone()
+        k[:, 640:704, 0] = k[:, 640:704, 0] * 2.0 ** 110
     return q.contiguous(), k.contiguous(), v
 
 
