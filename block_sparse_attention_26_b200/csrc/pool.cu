@@ -56,14 +56,21 @@ struct PoolArgs {
 };
 
 // Token of slot t (0..63) of block i: the prefix's own tokens, or the cube's
-// tokens t-major inside the cube, cubes t-major over the grid.
-__device__ __forceinline__ int block_token(const PoolArgs &a, int i, int t)
+// tokens t-major inside the cube, cubes t-major over the grid.  As the cube's
+// first token plus a slot offset that does not depend on the cube.
+__device__ __forceinline__ int cube_origin(const PoolArgs &a, int i)
 {
-    if (i < a.pre_blocks) return i * 64 + t;
+    if (i < a.pre_blocks) return i * 64;
     const int c = i - a.pre_blocks;
     const int cx = c % a.ncx, cy = (c / a.ncx) % a.ncy, ct = c / (a.ncx * a.ncy);
+    return a.P + (ct * a.cT * a.gH + cy * a.cH) * a.gW + cx * a.cW;
+}
+
+__device__ __forceinline__ int slot_offset(const PoolArgs &a, int i, int t)
+{
+    if (i < a.pre_blocks) return t;
     const int dx = t % a.cW, dy = (t / a.cW) % a.cH, dt = t / (a.cW * a.cH);
-    return a.P + ((ct * a.cT + dt) * a.gH + cy * a.cH + dy) * a.gW + cx * a.cW + dx;
+    return (dt * a.gH + dy) * a.gW + dx;
 }
 
 template <typename T, int UNROLL>
@@ -81,6 +88,14 @@ __global__ void __launch_bounds__(128) pool_kernel(PoolArgs a)
     const T *base = static_cast<const T *>(z == 0 ? a.src[0] : (z == 1 ? a.src[1] : a.src[2]));
     float *dst = z == 0 ? a.dst[0] : (z == 1 ? a.dst[1] : a.dst[2]);
     const int cols = a.H * a.d / V;
+    __shared__ int slot_off[64];
+    int origin = 0;
+    if (a.cube) {
+        // the block's token offsets once per CTA (integer divisions are slow)
+        if (threadIdx.x < 64) slot_off[threadIdx.x] = slot_offset(a, i, threadIdx.x);
+        origin = cube_origin(a, i);
+        __syncthreads();
+    }
     for (int col = threadIdx.x; col < cols; col += blockDim.x) {
         const int h = (col * V) / a.d;
         const int c = (col * V) % a.d;
@@ -90,15 +105,15 @@ __global__ void __launch_bounds__(128) pool_kernel(PoolArgs a)
         for (int e = 0; e < V; ++e) acc[e] = 0.0;
         int t = 0;
         if (a.cube) {
-            const T *pb = base + (int64_t)b * a.sb + (int64_t)h * a.sh + c;
+            const T *pb = base + (int64_t)b * a.sb + (int64_t)origin * a.sn + (int64_t)h * a.sh + c;
             for (; t + UNROLL <= n; t += UNROLL) {
                 uint4 r[UNROLL];
 #pragma unroll
-                for (int u = 0; u < UNROLL; ++u) r[u] = ld_nc_v4(pb + (int64_t)block_token(a, i, t + u) * a.sn);
+                for (int u = 0; u < UNROLL; ++u) r[u] = ld_nc_v4(pb + (int64_t)slot_off[t + u] * a.sn);
 #pragma unroll
                 for (int u = 0; u < UNROLL; ++u) Vec<T>::add(acc, r[u]);
             }
-            for (; t < n; ++t) Vec<T>::add(acc, ld_nc_v4(pb + (int64_t)block_token(a, i, t) * a.sn));
+            for (; t < n; ++t) Vec<T>::add(acc, ld_nc_v4(pb + (int64_t)slot_off[t] * a.sn));
         }
         for (; t + UNROLL <= n; t += UNROLL) {
             uint4 r[UNROLL];
