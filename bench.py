@@ -101,6 +101,15 @@ def max_over_ranks(value: float, pg, device) -> float:
     return float(t)
 
 
+def sum_over_ranks(value: int, pg, device) -> int:
+    """A count over the whole job (all_reduce SUM); identity on one rank."""
+    if pg is None:
+        return int(value)
+    t = torch.tensor([int(value)], dtype=torch.int64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.SUM)
+    return int(t)
+
+
 def job_throughput(w, world: int, ms_per_step: float, split: str = "replicas") -> float:
     """Whole-job dense-equivalent TFLOP/s over the slowest rank's time: all
     ranks' layers (replicas), or the one layer whose heads the ranks share."""
@@ -321,18 +330,6 @@ def _config_json(w, world, split="replicas", heads=None):
             else "L2 flushed between steps"}
 
 
-def launches_per_step(w) -> int:
-    """Kernels of ours one step launches: pool 1; select: scores, rows, scan,
-    expand (+ theta, filter, finalize, fallback with extra tokens); attention
-    preparation: bf16 centroids (2), bf16 copies of f32 inputs (3), modified
-    centroids and gather lists (2, extra tokens); fine pass 1 (+ the dense-row
-    merge when dense rows are split over keys)."""
-    dense_split = w.dense_rows[1] > w.dense_rows[0] and w.N > 256 * 64
-    return (1 + 4 + (4 if w.extra_tokens > 0 else 0)
-            + (2 if w.centroid else 0) + (3 if w.dtype == "f32" else 0) + (2 if w.extra_tokens > 0 else 0)
-            + 1 + (1 if dense_split else 0))
-
-
 def run_producer(args, w, dev):
     """--producer: the QKV projection with pooling in its epilogue
     (bsa_qkv_pool) against the same work unfused: cuBLAS (torch.matmul) for
@@ -495,14 +492,17 @@ def main():
         pg.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
+        launches0 = bsa.bsa_launch_count()
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         stop.record(stream)
         torch.cuda.synchronize(dev)
+        launches = bsa.bsa_launch_count() - launches0   # the library's own kernels, as it counted them
     if pg:
         pg.barrier()
     total_ms = max_over_ranks(start.elapsed_time(stop), pg, dev)
+    launches = sum_over_ranks(launches, pg, dev)
     status = bsa.bsa_device_status(buf.ws, stream)
     if status != 0:
         raise SystemExit(f"device status {status} after the timed steps")
@@ -578,7 +578,8 @@ def main():
                             "select_flop": select_flops(w),
                             "select_tflops": select_flops(w) / (ph_ms["select"] * 1e-3) / 1e12},
         "extra_tokens_per_row": (float(buf.extra_count.float().mean()) if buf.extra_count is not None else 0.0),
-        "gpu_launches": launches_per_step(w) * args.steps,
+        "gpu_launches": launches,
+        "workspace_bytes": int(buf.ws.numel() * buf.ws.element_size()),
         "clocks": clocks.summary(),
         "e2e": e2e,
     }

@@ -42,7 +42,7 @@ class bsa_params(ctypes.Structure):
         ("extra_tokens", ctypes.c_int32), ("centroid", ctypes.c_int32),
         ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
         ("cube_t", ctypes.c_int32), ("cube_h", ctypes.c_int32), ("cube_w", ctypes.c_int32),
-        ("qk_fp8", ctypes.c_int32), ("reserved_", ctypes.c_int32),
+        ("qk_fp8", ctypes.c_int32), ("modcent_per_row", ctypes.c_int32),
     ]
 
 
@@ -81,6 +81,8 @@ def _load() -> ctypes.CDLL:
     lib.bsa_attention_prepare.argtypes = lib.bsa_attention.argtypes
     lib.bsa_attention_run.argtypes = lib.bsa_attention.argtypes
     lib.bsa_selftest_bounded_wait.argtypes = [P, I64, P]
+    lib.bsa_launch_count.argtypes = []
+    lib.bsa_launch_count.restype = I64
     lib.bsa_dense_ref_rows.argtypes = [PP, P, P, P, I32, I32, P, P, P, SZ, P]
     lib.bsa_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
     PolP = ctypes.POINTER(bsa_policy)
@@ -103,7 +105,8 @@ lib = _load()
 
 EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_qkv_pool", "bsa_select", "bsa_select_static",
             "bsa_attention", "bsa_attention_prepare", "bsa_attention_run", "bsa_dense_ref_rows",
-            "bsa_device_status", "bsa_selftest_bounded_wait", "bsa_default_policy", "bsa_policy_decide",
+            "bsa_device_status", "bsa_selftest_bounded_wait", "bsa_launch_count", "bsa_default_policy",
+            "bsa_policy_decide",
             "bsa_status_string", "bsa_last_error")
 
 
@@ -128,7 +131,8 @@ def _stream(stream) -> ctypes.c_void_p:
 def make_params(q: torch.Tensor, method: str = "sol", *, q_block: Optional[int] = None,
                 tau: float = 1.3, keep_percent: float = 10.0, sink_blocks: int = 1,
                 keep_diag: int = 1, prefix_len: int = 0, dense_rows=(0, 0), extra_tokens: int = 0,
-                centroid: Optional[int] = None, grid=None, cube=(4, 4, 4), qk_fp8: bool = False) -> bsa_params:
+                centroid: Optional[int] = None, grid=None, cube=(4, 4, 4), qk_fp8: bool = False,
+                modcent_per_row: int = 0) -> bsa_params:
     """Parameters for a [B, N, H, d] query tensor `q` (strides taken from q).
     method "vsa" needs `grid` = (T, Hs, Ws) of the tokens after the prefix."""
     m = {"sol": BSA_SOL, "sla": BSA_SLA, "vsa": BSA_VSA}[method]
@@ -148,6 +152,7 @@ def make_params(q: torch.Tensor, method: str = "sol", *, q_block: Optional[int] 
     if centroid is not None:
         p.centroid = centroid
     p.qk_fp8 = int(bool(qk_fp8))
+    p.modcent_per_row = int(modcent_per_row)
     if m == BSA_VSA:
         if grid is None:
             raise ValueError("method vsa needs the latent grid (T, Hs, Ws)")
@@ -164,7 +169,7 @@ def params_for(w, q: torch.Tensor) -> bsa_params:
                        sink_blocks=w.sink_blocks, keep_diag=w.keep_diag, prefix_len=w.prefix_len,
                        dense_rows=tuple(w.dense_rows), extra_tokens=w.extra_tokens, centroid=w.centroid,
                        grid=getattr(w, "grid", None), cube=getattr(w, "cube", (4, 4, 4)),
-                       qk_fp8=getattr(w, "qk_fp8", False))
+                       qk_fp8=getattr(w, "qk_fp8", False), modcent_per_row=getattr(w, "modcent_per_row", 0))
 
 
 def dims(p: bsa_params):
@@ -229,6 +234,11 @@ def bsa_attention_run(p, q, k, v, kbar, vbar, blk_count, row_ptr, col_idx, extra
                                  _ptr(blk_count), _ptr(row_ptr), _ptr(col_idx), _ptr(extra_idx),
                                  _ptr(extra_count), _ptr(out), _ptr(lse), _ptr(ws),
                                  ws.numel() * ws.element_size(), _stream(stream)), "bsa_attention_run")
+
+
+def bsa_launch_count() -> int:
+    """Kernels the library has launched since it was loaded."""
+    return int(lib.bsa_launch_count())
 
 
 def bsa_selftest_bounded_wait(ws, cycles: int, stream=None):

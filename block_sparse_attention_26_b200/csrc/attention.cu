@@ -134,10 +134,11 @@ struct AttnArgs {
     const int32_t *extra_idx;    // [rows, E] ascending token indices
     const int32_t *extra_count;  // [rows]
     const __nv_bfloat16 *kx, *vx;              // K and V inputs (bf16), output strides
-    const __nv_bfloat16 *xk16, *xv16;          // [rows, Ecap, d] modified centroids
-    const float *xbias;                        // [rows, Ecap] log2 of their token counts
+    const __nv_bfloat16 *xk16, *xv16;          // [mc_cap, d] modified centroids
+    const float *xbias;                        // [mc_cap] log2 of their token counts
     const int32_t *xcnt;                       // [rows] modified centroids per row
-    const uint32_t *xaff;                      // [rows, nW] blocks that gave extra tokens
+    const int64_t *xoff;                       // [rows] where row r's start
+    const int32_t *slot;                       // [mc_cap] their places in xk16 / xv16
     // gathers by TMA (tile::gather4) when K and V are one uniform 2-D array of token
     // rows: row of (b, n, h) = b grow_b + n grow_n + h grow_h; else by cp.async
     int gather_tma;
@@ -314,6 +315,17 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b)
     return d;
 }
 
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 __device__ __forceinline__ float fmax3(float x, float y, float z)
 {
     float r;
@@ -467,6 +479,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ec0 = min(__shfl_sync(0xffffffffu, len, 10), a.E);
         const int ec1 = nq > 1 ? min(__shfl_sync(0xffffffffu, len, 11), a.E) : 0;
         const int U = __shfl_sync(0xffffffffu, len, 12);
+        int64_t xo = 0;
+        if (a.E > 0 && lane >= 13 && lane < 13 + nq) xo = a.xoff[rbase + lane - 13];
+        const int64_t xo0 = __shfl_sync(0xffffffffu, xo, 13), xo1 = __shfl_sync(0xffffffffu, xo, 14);
         __syncwarp();
         // the column lists of both query blocks (contiguous in the CSR), 16 in flight per lane
         for (int64_t pb = p0; pb < p2; pb += 512) {
@@ -484,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int u = 0; u < 16; ++u) {
                     const int e = 32 * (u & 7) + lane;
                     const int q = u >> 3;
-                    xb[u] = e < (q ? nx1 : nx0) ? a.xbias[(rbase + q) * a.Ecap + e] : 0.f;
+                    xb[u] = e < (q ? nx1 : nx0) ? a.xbias[(q ? xo1 : xo0) + e] : 0.f;
                 }
 #pragma unroll
                 for (int u = 0; u < 17; ++u) {
@@ -523,25 +538,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p0 >= p2) {   // no kept block at all: the lists did not ride along
                 for (int q = 0; q < nq; ++q)
                     for (int e = lane; e < (q ? nx1 : nx0); e += 32)
-                        gl_bias[q * kMaxE + e] = a.xbias[(rbase + q) * a.Ecap + e];
+                        gl_bias[q * kMaxE + e] = a.xbias[(q ? xo1 : xo0) + e];
                 for (int i = lane; i < U; i += 32) {
                     const uint32_t v = a.glist[sidx * kGlistCap + i];
                     gl_code[i] = v & 0x3fffffffu;
                     gl_who[i] = (uint8_t)(v >> 30);
                 }
             }
-            for (int q = 0; q < nq; ++q)
-                for (int w = lane; w < a.nW; w += 32) aff[q * a.nW + w] = a.xaff[(rbase + q) * a.nW + w];
+            // blocks that gave extra tokens, per query block, from the union list
+            __syncwarp();
+            for (int i = lane; i < U; i += 32) {
+                const uint32_t who = gl_who[i];
+                const int kb = (int)(gl_code[i] >> 6);
+                if (who & 1u) atomicOr(&aff[kb >> 5], 1u << (kb & 31));
+                if (who & 2u) atomicOr(&aff[a.nW + (kb >> 5)], 1u << (kb & 31));
+            }
             // gathered columns: the union of the query blocks' extra tokens (merged
             // by glist_kernel, padded to a multiple of 4), then each query block's
             // modified centroids
             const int m0 = nx0, m1 = nx1;
             for (int e = lane; e < m0; e += 32) {
-                gl_code[U + e] = 0x80000000u | (uint32_t)e;
+                gl_code[U + e] = 0x80000000u | (uint32_t)a.slot[xo0 + e];
                 gl_who[U + e] = 1;
             }
             for (int e = lane; e < m1; e += 32) {
-                gl_code[U + m0 + e] = 0xC0000000u | (uint32_t)e;
+                gl_code[U + m0 + e] = 0xC0000000u | (uint32_t)a.slot[xo1 + e];
                 gl_who[U + m0 + e] = 2;
             }
             if (lane == 0) {
@@ -613,12 +634,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         // row address of a gathered column: an extra token of this head, or a
-        // modified centroid (bit 31 set; query block in bit 30, entry in bits 0-29)
+        // modified centroid (bit 31 set; query block in bit 30, its slot in bits 0-29)
         auto row_src = [&](uint32_t code) -> const __nv_bfloat16 * {
-            if (code & 0x80000000u) {
-                const int q = (code >> 30) & 1, e = (int)(code & 0x3fffffffu);
-                return src_c + ((rbase + q) * a.Ecap + e) * D;
-            }
+            if (code & 0x80000000u) return src_c + (int64_t)(code & 0x3fffffffu) * D;
             return src_x + (int64_t)b * a.sb + (int64_t)code * a.sn + (int64_t)h * a.sh;
         };
         auto push = [&](int kind, const int (&blk)[2], const uint32_t (&who)[2], const int (&nc)[2],
@@ -674,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < 4; ++i) {
                     const uint32_t code = gl_code[c + i < gln ? gl0 + c + i : gl0 + gln - 1];
                     if (i == 0) cent = (code & 0x80000000u) != 0u;
-                    rw[i] = cent ? (int)((rbase + ((code >> 30) & 1u)) * a.Ecap + (code & 0x3fffffffu))
+                    rw[i] = cent ? (int)(code & 0x3fffffffu)
                                  : (int)(b * a.grow_b + h * a.grow_h + (int64_t)code * a.grow_n);
                 }
 #pragma unroll
@@ -1245,98 +1263,261 @@ __device__ __forceinline__ void load_bf16_vec(const __nv_bfloat16 *p, float (&f)
     }
 }
 
-// Per query block with extra tokens: the blocks they came from, and for each
-// such block that keeps tokens a centroid over its remaining tokens, (n k - sum
-// of the extra keys) / (n - e) in fp64 from the f32 block mean, stored in bf16
-// with bias log2(n - e).  One warp per row.
-// CPL = d / 32 channels per lane; each lane reads its channels of a token with
-// one vector load, four tokens in flight.
-template <int CPL>
-__global__ void __launch_bounds__(256) modcent_kernel(const int32_t *__restrict__ extra_idx,
-                                                      const int32_t *__restrict__ extra_count,
-                                                      const float *__restrict__ kbar, const float *__restrict__ vbar,
-                                                      const __nv_bfloat16 *__restrict__ k,
-                                                      const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
-                                                      int64_t sh, int64_t rows, int H, int N, int nQB, int nKB, int nW,
-                                                      int E, int Ecap, __nv_bfloat16 *__restrict__ xk,
-                                                      __nv_bfloat16 *__restrict__ xv, float *__restrict__ xbias,
-                                                      int32_t *__restrict__ xcnt, uint32_t *__restrict__ xaff)
+// Modified centroids of the blocks that gave extra tokens: for query block r and
+// a block b that gave e of its n tokens to r's list and keeps some, the centroid
+// of its remaining tokens, (n kbar_b - sum of the extra keys) / (n - e), with
+// bias log2(n - e); the same for V.  Row r's entries, in ascending block order,
+// are numbered idx = xoff[r] .. xoff[r] + xcnt[r] - 1 (as many as the capacity
+// holds); the centroids themselves are stored grouped by source block, entry
+// idx at slot[idx].  Steps: count each row's entries (mc_count_kernel) and scan;
+// per (b, h) and group of query blocks, count the entries that fit per source
+// block and scan (mc_group_kernel<1>), then list them (mc_group_kernel<2>), with
+// counters in shared memory; form each block's entries from its K and V rows,
+// read once into shared memory (mc_build_kernel).
+
+struct McArgs {
+    const int32_t *extra_idx, *extra_count;
+    int64_t rows;
+    int H, N, nQB, nKB, E;
+    int G, rpg;                  // query-block groups per (b, h), query blocks per group
+    int32_t *xcnt;
+    const int64_t *xoff;
+    int32_t *cnt3;               // [B*H, nKB, G] entries that fit, per (source block, group)
+    const int64_t *off3;         // [B*H*nKB*G + 1] its exclusive scan
+    uint64_t *ent;               // [cap] left-out tokens of each entry (bit t: token 64 b + t), by block
+    int32_t *slot;               // [cap] where entry idx sits in ent and in the centroid arrays
+    float *xbias;                // [cap] by idx
+    int64_t cap;
+    int32_t *status;
+};
+
+// Walks row r's ascending extra-token list (one warp; E <= 256, so 8 tokens a
+// lane, all loaded at once) by runs of tokens from one block, in token order:
+// f(blk, mask, e, rank) once per run, on one lane, rank = the run's place among
+// the row's runs whose block keeps tokens (-1 for a run that takes the whole
+// block).  In each 32-token chunk a run starts where the block changes (one
+// ballot); its tokens' bits are OR-ed into its first lane by a segmented
+// shuffle-down; a run that reaches the chunk's last lane and goes on in the next
+// chunk is carried over.  A token outside [0, N) belongs to no run (it is
+// reported).  Returns the count of ranked runs.
+template <typename F>
+__device__ __forceinline__ int walk_runs(const McArgs &a, int64_t r, int lane, F &&f)
 {
-    constexpr int d = 32 * CPL;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t r = (int64_t)blockIdx.x * 8 + warp;
-    if (r >= rows) return;
-    const int bh = (int)(r / nQB);
-    const int b = bh / H, h = bh % H;
-    const int c0 = lane * CPL;
-    for (int w = lane; w < nW; w += 32) xaff[r * nW + w] = 0u;
-    __syncwarp();
-    const int n = extra_count[r];
-    const int32_t *ex = extra_idx + r * E;
-    const __nv_bfloat16 *kh = k + (int64_t)b * sb + (int64_t)h * sh + c0;
-    const __nv_bfloat16 *vh = v + (int64_t)b * sb + (int64_t)h * sh + c0;
-    int nent = 0;
-    for (int i = 0; i < n;) {
-        const int blk = ex[i] >> 6;
-        int jend = i;
-        while (jend < n && (ex[jend] >> 6) == blk) ++jend;
-        if (lane == 0) xaff[r * nW + (blk >> 5)] |= 1u << (blk & 31);
-        const int nb = min(64, N - blk * 64);
-        const int rem = nb - (jend - i);
-        if (rem > 0) {
-            const float *kb = kbar + ((int64_t)bh * nKB + blk) * d + c0;
-            const float *vb = vbar + ((int64_t)bh * nKB + blk) * d + c0;
-            double sk[CPL], sv[CPL];
+    static_assert(kMaxE == 256, "8 tokens per lane");
+    const int n = min(a.extra_count[r], a.E);
+    const int32_t *ex = a.extra_idx + r * a.E;
+    int tk[8];
 #pragma unroll
-            for (int j = 0; j < CPL; ++j) {
-                sk[j] = (double)nb * (double)kb[j];
-                sv[j] = (double)nb * (double)vb[j];
-            }
-            // block sum minus the extra tokens, in token order
-            int t = i;
-            for (; t + 4 <= jend; t += 4) {
-                float fk[4][CPL], fv[4][CPL];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    load_bf16_vec<CPL>(kh + (int64_t)ex[t + u] * sn, fk[u]);
-                    load_bf16_vec<CPL>(vh + (int64_t)ex[t + u] * sn, fv[u]);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-#pragma unroll
-                    for (int j = 0; j < CPL; ++j) {
-                        sk[j] -= (double)fk[u][j];
-                        sv[j] -= (double)fv[u][j];
-                    }
-            }
-            for (; t < jend; ++t) {
-                float fk[CPL], fv[CPL];
-                load_bf16_vec<CPL>(kh + (int64_t)ex[t] * sn, fk);
-                load_bf16_vec<CPL>(vh + (int64_t)ex[t] * sn, fv);
-#pragma unroll
-                for (int j = 0; j < CPL; ++j) {
-                    sk[j] -= (double)fk[j];
-                    sv[j] -= (double)fv[j];
-                }
-            }
-            __nv_bfloat16 ok[CPL], ov[CPL];
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) {
-                ok[j] = __float2bfloat16_rn((float)(sk[j] / rem));
-                ov[j] = __float2bfloat16_rn((float)(sv[j] / rem));
-            }
-            __nv_bfloat16 *dk = xk + (r * Ecap + nent) * d + c0, *dv = xv + (r * Ecap + nent) * d + c0;
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) {
-                dk[j] = ok[j];
-                dv[j] = ov[j];
-            }
-            if (lane == 0) xbias[r * Ecap + nent] = log2f((float)rem);
-            ++nent;
+    for (int u = 0; u < 8; ++u) {
+        const int i = 32 * u + lane;
+        tk[u] = i < n ? ex[i] : -1;
+        if (i < n && (tk[u] < 0 || tk[u] >= a.N)) {
+            report(a.status, BSA_DEV_INTERNAL, 3);
+            tk[u] = -1;
         }
-        i = jend;
     }
-    if (lane == 0) xcnt[r] = nent;
+    int ranked = 0;
+    int cblk = -1, ce = 0;   // the run carried over from the previous chunk
+    uint64_t cmask = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        if (32 * u >= n) break;
+        const int tok = tk[u];
+        const int blk = tok >= 0 ? tok >> 6 : -1 - lane;   // lanes without a token stand alone
+        const int prev = __shfl_up_sync(0xffffffffu, blk, 1);
+        const uint32_t bnd = __ballot_sync(0xffffffffu, lane == 0 || blk != prev);
+        const uint32_t above = bnd & ~((2u << lane) - 1u);   // (2u << 31 wraps to 0: all ones)
+        const int end = above ? __ffs(above) - 2 : 31;       // last lane of this lane's run
+        const int o = tok & 63;
+        uint32_t lo = tok >= 0 && o < 32 ? 1u << o : 0u, hi = tok >= 0 && o >= 32 ? 1u << (o - 32) : 0u;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t vlo = __shfl_down_sync(0xffffffffu, lo, off);
+            const uint32_t vhi = __shfl_down_sync(0xffffffffu, hi, off);
+            if (lane + off <= end) {
+                lo |= vlo;
+                hi |= vhi;
+            }
+        }
+        const bool first = (bnd >> lane) & 1u;
+        uint64_t mask = ((uint64_t)hi << 32) | lo;
+        int e = end - lane + 1;
+        if (lane == 0 && blk == cblk) {
+            e += ce;
+            mask |= cmask;
+        }
+        const int nxt = u < 7 ? __shfl_sync(0xffffffffu, tk[u < 7 ? u + 1 : u], 0) : -1;
+        const bool cont = tok >= 0 && end == 31 && nxt >= 0 && (nxt >> 6) == blk;
+        const bool emit = tok >= 0 && first && !cont;
+        const bool keeps = emit && min(64, a.N - blk * 64) - e > 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, keeps);
+        if (emit) f(blk, mask, e, keeps ? ranked + __popc(bal & ((1u << lane) - 1u)) : -1);
+        ranked += __popc(bal);
+        const uint32_t cl = __ballot_sync(0xffffffffu, cont && first);
+        if (cl) {
+            const int src = __ffs(cl) - 1;
+            cblk = __shfl_sync(0xffffffffu, blk, src);
+            ce = __shfl_sync(0xffffffffu, e, src);
+            cmask = __shfl_sync(0xffffffffu, mask, src);
+        } else {
+            cblk = -1;
+            ce = 0;
+            cmask = 0;
+        }
+    }
+    return ranked;
+}
+
+// Each row's entry count (one warp per row).
+__global__ void __launch_bounds__(256) mc_count_kernel(McArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= a.rows) return;
+    const int cnt = walk_runs(a, r, lane, [](int, uint64_t, int, int) {});
+    if (lane == 0) a.xcnt[r] = cnt;
+}
+
+// One CTA per ((b, h), group g of query blocks), a warp per row, one counter per
+// source block in shared memory.  kMode 1: the entries that fit, per source
+// block, into cnt3; 2: list them -- ent and slot from the scanned counts, the
+// biases -- and cut each row's count to what fits.
+template <int kMode>
+__global__ void __launch_bounds__(256) mc_group_kernel(McArgs a)
+{
+    extern __shared__ int32_t cs[];   // [nKB]
+    const int64_t bh = blockIdx.x / a.G;
+    const int g = (int)(blockIdx.x % a.G);
+    const int i0 = g * a.rpg, i1 = min(a.nQB, i0 + a.rpg);
+    const int64_t b3 = bh * a.nKB;
+    for (int blk = threadIdx.x; blk < a.nKB; blk += blockDim.x)
+        cs[blk] = kMode == 1 ? 0 : (int32_t)a.off3[(b3 + blk) * a.G + g];
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = i0 + warp; i < i1; i += (int)(blockDim.x >> 5)) {
+        const int64_t r = bh * a.nQB + i;
+        const int64_t x0 = a.xoff[r];
+        const int cnt = walk_runs(a, r, lane, [&](int blk, uint64_t mask, int e, int rank) {
+            if (rank < 0 || x0 + rank >= a.cap) return;
+            if (kMode == 1) {
+                atomicAdd(&cs[blk], 1);
+            } else {
+                const int sl = atomicAdd(&cs[blk], 1);
+                a.ent[sl] = mask;
+                a.slot[x0 + rank] = sl;
+                a.xbias[x0 + rank] = log2f((float)(min(64, a.N - blk * 64) - e));
+            }
+        });
+        if (kMode == 2 && lane == 0) {
+            const int64_t fit = a.cap - x0;
+            const int kept = (int)(fit < 0 ? 0 : (fit < cnt ? fit : cnt));
+            a.xcnt[r] = kept;
+            if (kept < cnt) report(a.status, BSA_DEV_CAPACITY, 2);
+        }
+    }
+    if (kMode == 1) {
+        __syncthreads();
+        for (int blk = threadIdx.x; blk < a.nKB; blk += blockDim.x) a.cnt3[(b3 + blk) * a.G + g] = cs[blk];
+    }
+}
+
+// One CTA per (source block, b, h) -- the heads of one block side by side, so
+// that CTAs running together read neighbouring parts of the same token rows --
+// and 2 d threads.  The block's K and V rows go to shared memory once; then each
+// entry listed under the block is formed by 2 d / 8 lanes, a lane owning 8
+// channels of K or of V: in f32, the block's sum n kbar_b minus its left-out
+// tokens in token order, times 1/(n - e), rounded to bf16, written at the entry's
+// slot (a block's slots are consecutive).
+template <int D>
+__global__ void __launch_bounds__(2 * D) mc_build_kernel(McArgs a, const float *__restrict__ kbar,
+                                                         const float *__restrict__ vbar,
+                                                         const __nv_bfloat16 *__restrict__ k,
+                                                         const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
+                                                         int64_t sh, __nv_bfloat16 *__restrict__ xk,
+                                                         __nv_bfloat16 *__restrict__ xv)
+{
+    constexpr int kThr = 2 * D;
+    constexpr int kCpr = D / 8;                 // 16-byte chunks per row
+    constexpr int kLpe = 2 * kCpr;              // lanes per entry
+    constexpr int kEpw = 32 / kLpe;             // entries per warp at a time
+    constexpr int kWarps = kThr / 32;
+    __shared__ __align__(16) __nv_bfloat16 rows_s[2][64][D];
+    __shared__ uint64_t es[kThr];
+    __shared__ float rinv[65];
+    const int64_t BH = a.rows / a.nQB;
+    const int blk = (int)(blockIdx.x / BH);
+    const int64_t bh = blockIdx.x % BH;
+    const int64_t e0 = a.off3[(bh * a.nKB + blk) * a.G];
+    const int n_ent = (int)(a.off3[(bh * a.nKB + blk + 1) * a.G] - e0);
+    if (n_ent == 0) return;
+    const int b = (int)(bh / a.H), h = (int)(bh % a.H);
+    const int nb = min(64, a.N - blk * 64);
+    // 2 tensors x 64 rows x kCpr chunks = 8 per thread, all in flight at once
+    uint4 ld[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int x = threadIdx.x + kThr * u;
+        const int t = x / (64 * kCpr), row = (x / kCpr) % 64, c16 = x % kCpr;
+        const __nv_bfloat16 *src = (t ? v : k) + (int64_t)b * sb + (int64_t)(blk * 64 + row) * sn +
+                                   (int64_t)h * sh + c16 * 8;
+        if (row < nb) ld[u] = __ldg(reinterpret_cast<const uint4 *>(src));
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int x = threadIdx.x + kThr * u;
+        const int t = x / (64 * kCpr), row = (x / kCpr) % 64, c16 = x % kCpr;
+        if (row < nb) *reinterpret_cast<uint4 *>(&rows_s[t][row][c16 * 8]) = ld[u];
+    }
+    if (threadIdx.x <= 64) rinv[threadIdx.x] = threadIdx.x > 0 ? 1.f / (float)threadIdx.x : 0.f;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sub = lane / kLpe, l = lane % kLpe;
+    const int t = l / kCpr, c0 = (l % kCpr) * 8;
+    float2 base[4];
+    {
+        const float4 *m = reinterpret_cast<const float4 *>((t ? vbar : kbar) + (bh * a.nKB + blk) * D + c0);
+        const float4 m0 = m[0], m1 = m[1];
+        const float fn = (float)nb;
+        base[0] = make_float2(fn * m0.x, fn * m0.y);
+        base[1] = make_float2(fn * m0.z, fn * m0.w);
+        base[2] = make_float2(fn * m1.x, fn * m1.y);
+        base[3] = make_float2(fn * m1.z, fn * m1.w);
+    }
+    __nv_bfloat16 *dst = (t ? xv : xk) + e0 * D + c0;
+    for (int i0 = 0; i0 < n_ent; i0 += kThr) {
+        __syncthreads();   // (the first also publishes the rows and rinv)
+        if (i0 + (int)threadIdx.x < n_ent) es[threadIdx.x] = a.ent[e0 + i0 + threadIdx.x];
+        __syncthreads();
+        const int m = min(kThr, n_ent - i0);
+        for (int i = warp * kEpw + sub; i < m; i += kWarps * kEpw) {
+            const uint64_t em = es[i];
+            float2 sum[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sum[j] = base[j];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t mk = (uint32_t)(em >> (32 * half));
+                while (mk) {
+                    const int bit = 32 * half + __ffs(mk) - 1;
+                    mk &= mk - 1;
+                    const uint4 w = *reinterpret_cast<const uint4 *>(&rows_s[t][bit][c0]);
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        sum[j] = fsub2(sum[j], make_float2(__uint_as_float(wv[j] << 16),
+                                                           __uint_as_float(wv[j] & 0xffff0000u)));
+                }
+            }
+            const float ri = rinv[nb - __popcll(em)];
+            const float2 r2 = make_float2(ri, ri);
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 y = fmul2(sum[j], r2);
+                o[j] = pack_bf16x2(y.x, y.y);
+            }
+            *reinterpret_cast<uint4 *>(dst + (int64_t)(i0 + i) * D) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
 }
 
 // Per sparse tile of the fine pass (query blocks qb0 and qb0 + 1 for 64-row
@@ -1363,8 +1544,22 @@ __global__ void __launch_bounds__(128) glist_kernel(const int32_t *__restrict__ 
     const int64_t r0 = bh * nQB + qb0;
     const int n0 = min(extra_count[r0], E), n1 = nq > 1 ? min(extra_count[r0 + 1], E) : 0;
     int32_t *A = sA[warp], *B = sB[warp];
-    for (int i = lane; i < n0; i += 32) A[i] = extra_idx[r0 * E + i];
-    for (int i = lane; i < n1; i += 32) B[i] = extra_idx[(r0 + 1) * E + i];
+    {
+        // both lists, every load in flight before the first store
+        int va[kMaxE / 32], vb[kMaxE / 32];
+#pragma unroll
+        for (int u = 0; u < kMaxE / 32; ++u) {
+            const int i = 32 * u + lane;
+            va[u] = i < n0 ? extra_idx[r0 * E + i] : 0;
+            vb[u] = i < n1 ? extra_idx[(r0 + 1) * E + i] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kMaxE / 32; ++u) {
+            const int i = 32 * u + lane;
+            if (i < n0) A[i] = va[u];
+            if (i < n1) B[i] = vb[u];
+        }
+    }
     __syncwarp();
     auto lower_bound = [](const int32_t *X, int n, int key) {
         int lo = 0, hi = n;
@@ -1678,6 +1873,7 @@ cudaError_t launch_attn_kernel(const CUtensorMap &tq, const CUtensorMap &tk, con
     cudaError_t e =
         cudaFuncSetAttribute(attn_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    count_launch();
     attn_kernel<D, QK8><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, tg[0], tg[1], tg[2], tg[3],
                                                                  t5[0], t5[1], t5[2], a);
     return cudaGetLastError();
@@ -1737,8 +1933,11 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
         __nv_bfloat16 *dk = reinterpret_cast<__nv_bfloat16 *>(ws + L.k16);
         __nv_bfloat16 *dv = reinterpret_cast<__nv_bfloat16 *>(ws + L.v16);
         if (prep) {
+            count_launch();
             inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(q), dq, D.B, D.N, D.H, D.d, sb, sn, sh);
+            count_launch();
             inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(k), dk, D.B, D.N, D.H, D.d, sb, sn, sh);
+            count_launch();
             inputs_to_bf16_kernel<<<g, 256, 0, st>>>(static_cast<const float *>(v), dv, D.B, D.N, D.H, D.d, sb, sn, sh);
         }
         q16 = dq;
@@ -1754,7 +1953,9 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     if (use_cent && prep) {
         const int64_t n = (int64_t)BH * D.nKB * D.d;
         const unsigned g = (unsigned)std::min<int64_t>(ceil_div(n, 256), (int64_t)sm_count() * 8);
+        count_launch();
         to_bf16_kernel<<<g, 256, 0, st>>>(kbar, kc, n);
+        count_launch();
         to_bf16_kernel<<<g, 256, 0, st>>>(vbar, vc, n);
     }
     const bool f8 = p.qk_fp8 != 0;
@@ -1765,10 +1966,13 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     const int nb64 = (int)ceil_div(D.N, 64), nch64 = (int)ceil_div(D.nKB, 64);
     if (f8 && prep) {
         // Q per 64 tokens, K per key block (also 64 tokens), centroids per 64
+        count_launch();
         quant_rows_kernel<<<dim3((unsigned)nb64, (unsigned)BH), 256, 0, st>>>(
             static_cast<const __nv_bfloat16 *>(q16), sb, sn, sh, D.N, D.H, nb64, q8, sq8);
+        count_launch();
         quant_rows_kernel<<<dim3((unsigned)nb64, (unsigned)BH), 256, 0, st>>>(
             static_cast<const __nv_bfloat16 *>(k16), sb, sn, sh, D.N, D.H, nb64, k8, sk8);
+        if (use_cent) count_launch();
         if (use_cent)
             quant_cent_kernel<<<dim3((unsigned)nch64, (unsigned)BH), 256, 0, st>>>(kbar, D.nKB, nch64, kc8, skc8);
     }
@@ -1851,21 +2055,64 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     a.xv16 = reinterpret_cast<const __nv_bfloat16 *>(ws + L.xv16);
     a.xbias = reinterpret_cast<const float *>(ws + L.xbias);
     a.xcnt = reinterpret_cast<const int32_t *>(ws + L.xcnt);
-    a.xaff = reinterpret_cast<const uint32_t *>(ws + L.xaff);
+    a.xoff = reinterpret_cast<const int64_t *>(ws + L.xoff);
+    a.slot = reinterpret_cast<const int32_t *>(ws + L.mc_slot);
     if (a.E > 0 && p.dtype != BSA_DT_BF16) {
         // the gathers read rows through the input strides
         set_error("extra tokens need bf16 inputs");
         return cudaErrorInvalidValue;
     }
     if (a.E > 0 && prep) {
-        auto mc = D.d == 128 ? modcent_kernel<4> : modcent_kernel<2>;
-        mc<<<(unsigned)ceil_div(D.rows, 8), 256, 0, st>>>(
-            extra_idx, extra_count, kbar, vbar, static_cast<const __nv_bfloat16 *>(k),
-            static_cast<const __nv_bfloat16 *>(v), sb, sn, sh, D.rows, D.H, D.N, D.nQB, D.nKB, D.nW, D.E,
-            a.Ecap, reinterpret_cast<__nv_bfloat16 *>(ws + L.xk16), reinterpret_cast<__nv_bfloat16 *>(ws + L.xv16),
-            reinterpret_cast<float *>(ws + L.xbias), reinterpret_cast<int32_t *>(ws + L.xcnt),
-            reinterpret_cast<uint32_t *>(ws + L.xaff));
+        McArgs m;
+        m.extra_idx = extra_idx;
+        m.extra_count = extra_count;
+        m.rows = D.rows;
+        m.H = D.H;
+        m.N = D.N;
+        m.nQB = D.nQB;
+        m.nKB = D.nKB;
+        m.E = D.E;
+        m.G = mc_groups(D);
+        m.rpg = (int)ceil_div(D.nQB, m.G);
+        m.xcnt = reinterpret_cast<int32_t *>(ws + L.xcnt);
+        m.xoff = reinterpret_cast<const int64_t *>(ws + L.xoff);
+        m.cnt3 = reinterpret_cast<int32_t *>(ws + L.mc_cnt3);
+        m.off3 = reinterpret_cast<const int64_t *>(ws + L.mc_off3);
+        m.ent = reinterpret_cast<uint64_t *>(ws + L.mc_ent);
+        m.slot = reinterpret_cast<int32_t *>(ws + L.mc_slot);
+        m.xbias = reinterpret_cast<float *>(ws + L.xbias);
+        m.cap = L.mc_cap;
+        m.status = a.status;
+        const int64_t n3 = BH * D.nKB * m.G;
+        int64_t *tile = reinterpret_cast<int64_t *>(ws + L.mc_tile);
+        const size_t gsm = (size_t)D.nKB * 4;
+        cudaError_t e;
+        if ((e = cudaFuncSetAttribute(mc_group_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm)) !=
+                cudaSuccess ||
+            (e = cudaFuncSetAttribute(mc_group_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm)) !=
+                cudaSuccess)
+            return e;
+        count_launch();
+        mc_count_kernel<<<(unsigned)ceil_div(D.rows, 8), 256, 0, st>>>(m);
+        if ((e = launch_scan(m.xcnt, D.rows, reinterpret_cast<int64_t *>(ws + L.xoff), tile, st)) != cudaSuccess)
+            return e;
+        count_launch();
+        mc_group_kernel<1><<<(unsigned)(BH * m.G), 256, gsm, st>>>(m);
+        if ((e = launch_scan(m.cnt3, n3, reinterpret_cast<int64_t *>(ws + L.mc_off3), tile, st)) != cudaSuccess)
+            return e;
+        count_launch();
+        mc_group_kernel<2><<<(unsigned)(BH * m.G), 256, gsm, st>>>(m);
+        count_launch();
+        if (D.d == 128)
+            mc_build_kernel<128><<<(unsigned)(BH * D.nKB), 256, 0, st>>>(
+                m, kbar, vbar, static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), sb, sn,
+                sh, reinterpret_cast<__nv_bfloat16 *>(ws + L.xk16), reinterpret_cast<__nv_bfloat16 *>(ws + L.xv16));
+        else
+            mc_build_kernel<64><<<(unsigned)(BH * D.nKB), 128, 0, st>>>(
+                m, kbar, vbar, static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), sb, sn,
+                sh, reinterpret_cast<__nv_bfloat16 *>(ws + L.xk16), reinterpret_cast<__nv_bfloat16 *>(ws + L.xv16));
         const int64_t ntiles = (int64_t)BH * ceil_div(D.N, kM);
+        count_launch();
         glist_kernel<<<(unsigned)ceil_div(ntiles, 4), 128, 0, st>>>(
             extra_idx, extra_count, D.E, D.nQB, D.Bq, (int)ceil_div(D.N, kM), ntiles,
             reinterpret_cast<uint32_t *>(ws + L.glist), reinterpret_cast<int32_t *>(ws + L.glcnt));
@@ -1887,7 +2134,7 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     if (items == 0 || !run) return cudaGetLastError();
     // gather maps: token rows of K and V as one 2-D array when the strides allow it
     // (the row pitch min(sn, sh) divides every stride and holds a whole row), and the
-    // modified centroids [rows x Ecap, d]
+    // modified centroids [mc_cap, d]
     CUtensorMap tg[4] = {tk, tv, tk, tv};
     a.gather_tma = 0;
     a.grow_b = a.grow_n = a.grow_h = 0;
@@ -1896,7 +2143,7 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
         if (rs >= D.d && sb % rs == 0 && sn % rs == 0 && sh % rs == 0) {
             const int64_t nrows_k = (int64_t)(D.B - 1) * (sb / rs) + (int64_t)(D.N - 1) * (sn / rs) +
                                     (int64_t)(D.H - 1) * (sh / rs) + 1;
-            const int64_t nrows_x = D.rows * (int64_t)a.Ecap;
+            const int64_t nrows_x = L.mc_cap;
             if (nrows_k < INT32_MAX && nrows_x < INT32_MAX && make_map_rows(&tg[0], k16, nrows_k, D.d, rs) &&
                 make_map_rows(&tg[1], v16, nrows_k, D.d, rs) &&
                 make_map_rows(&tg[2], ws + L.xk16, nrows_x, D.d, D.d) &&
@@ -1918,6 +2165,7 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
                                 : launch_attn_kernel<128, false>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st);
     if (e != cudaSuccess) return e;
     if (a.n_dense > 0 && a.dense_split > 1) {
+        count_launch();
         combine_kernel<<<(unsigned)(BH * (int64_t)a.n_dense), kM, 0, st>>>(a, D.d);
         e = cudaGetLastError();
     }

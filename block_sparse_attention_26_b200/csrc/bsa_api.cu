@@ -24,6 +24,10 @@ void set_error(const char *fmt, ...)
     va_end(ap);
 }
 
+static std::atomic<int64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 int sm_count()
 {
     static std::atomic<int> cache[64];
@@ -69,32 +73,43 @@ WsLayout ws_layout(const bsa_params &p)
         return at;
     };
     const int64_t BH = (int64_t)D.B * D.H;
+    // the selection's scratch: its regions, then the extra-token passes'
     Taker T;
     select_regions(p, D, L, T);
-    off = T.off;
+    const bool ex = D.E > 0;
+    L.ex_theta = T.take(ex ? (size_t)D.rows * 4 : 0);
+    L.ex_smax = T.take(ex ? (size_t)D.rows * 4 : 0);
+    L.ex_cut = T.take(ex ? (size_t)D.rows * 16 : 0);
+    L.ex_buf = T.take(ex ? (size_t)D.rows * extra_buffer_capacity() * 8 : 0);
+    L.ex_cnt = T.take(ex ? (size_t)D.rows * 4 : 0);
+    L.ex_ovf = T.take(ex ? (size_t)(D.rows + 1) * 4 : 0);
+    L.ex_scratch = T.take(ex ? (size_t)fallback_ctas() * D.N * 4 : 0);
+    const size_t select_end = T.off;
+    // the attention calls' scratch, over the same bytes after the status word
+    off = align_up(L.status + 2 * sizeof(int32_t), 256);
     L.kc16 = take((size_t)BH * D.nKB * D.d * 2);
     L.vc16 = take((size_t)BH * D.nKB * D.d * 2);
-    const size_t ecap = D.E > 0 ? (size_t)std::min(D.E, D.nKB) : 0;
-    L.xk16 = take((size_t)D.rows * ecap * D.d * 2);
-    L.xv16 = take((size_t)D.rows * ecap * D.d * 2);
-    L.xbias = take((size_t)D.rows * ecap * 4);
-    L.xcnt = take(D.E > 0 ? (size_t)D.rows * 4 : 0);
-    L.xaff = take(D.E > 0 ? (size_t)D.rows * D.nW * 4 : 0);
+    const int64_t ecap = ex ? std::min(D.E, D.nKB) : 0;
+    const int64_t per_row = p.modcent_per_row > 0 ? std::min<int64_t>(p.modcent_per_row, ecap) : ecap;
+    L.mc_cap = D.rows * per_row;
+    const int64_t n3 = ex ? BH * D.nKB * mc_groups(D) : 0;
+    L.xk16 = take((size_t)L.mc_cap * D.d * 2);
+    L.xv16 = take((size_t)L.mc_cap * D.d * 2);
+    L.xbias = take((size_t)L.mc_cap * 4);
+    L.xcnt = take(ex ? (size_t)D.rows * 4 : 0);
+    L.xoff = take(ex ? (size_t)(D.rows + 1) * 8 : 0);
+    L.mc_slot = take((size_t)L.mc_cap * 4);
+    L.mc_ent = take((size_t)L.mc_cap * 8);
+    L.mc_cnt3 = take((size_t)n3 * 4);
+    L.mc_off3 = take(ex ? (size_t)(n3 + 1) * 8 : 0);
+    L.mc_tile = take(ex ? (size_t)ceil_div(std::max<int64_t>(D.rows, n3), 4096) * 8 : 0);
     const size_t ftiles = (size_t)BH * (size_t)((D.N + 127) / 128);
-    L.glist = take(D.E > 0 ? ftiles * kGlistCap * 4 : 0);
-    L.glcnt = take(D.E > 0 ? ftiles * 4 : 0);
+    L.glist = take(ex ? ftiles * kGlistCap * 4 : 0);
+    L.glcnt = take(ex ? ftiles * 4 : 0);
     const size_t in16 = p.dtype == BSA_DT_F32 ? (size_t)D.B * D.N * D.H * D.d * 2 : 0;
     L.q16 = take(in16);
     L.k16 = take(in16);
     L.v16 = take(in16);
-    const bool ex = D.E > 0;
-    L.ex_theta = take(ex ? (size_t)D.rows * 4 : 0);
-    L.ex_smax = take(ex ? (size_t)D.rows * 4 : 0);
-    L.ex_cut = take(ex ? (size_t)D.rows * 16 : 0);
-    L.ex_buf = take(ex ? (size_t)D.rows * extra_buffer_capacity() * 8 : 0);
-    L.ex_cnt = take(ex ? (size_t)D.rows * 4 : 0);
-    L.ex_ovf = take(ex ? (size_t)(D.rows + 1) * 4 : 0);
-    L.ex_scratch = take(ex ? (size_t)fallback_ctas() * D.N * 4 : 0);
     // fp8 Q / K (qk_fp8): e4m3 copies and one scale per 64 tokens (per 64 centroids)
     const bool f8 = p.qk_fp8 != 0;
     const size_t ntok = (size_t)D.B * D.N * D.H * D.d;
@@ -107,7 +122,7 @@ WsLayout ws_layout(const bsa_params &p)
     L.part_tiles = dense_partial_tiles(D, p.dense_row_end - p.dense_row_begin);
     L.part_o = take((size_t)L.part_tiles * 128 * D.d * sizeof(float));
     L.part_ml = take((size_t)L.part_tiles * 128 * 2 * sizeof(float));
-    L.total = off;
+    L.total = std::max(off, select_end);
     return L;
 }
 
@@ -170,6 +185,16 @@ bsa_status check_params(const bsa_params *p)
     if (p->dense_row_begin < 0 || p->dense_row_end < p->dense_row_begin || p->dense_row_end > p->N)
         FAIL(BSA_ERR_INVALID_ARG, "dense rows must satisfy 0 <= begin <= end <= N");
     if (p->extra_tokens < 0 || p->extra_tokens > 256) FAIL(BSA_ERR_INVALID_ARG, "extra_tokens outside [0, 256]");
+    if (p->modcent_per_row < 0) FAIL(BSA_ERR_INVALID_ARG, "modcent_per_row < 0");
+    if (p->extra_tokens > 0) {
+        // modified-centroid slots are 30-bit fields of the fine pass's column codes
+        const Dims D = dims_of(*p);
+        const int64_t ecap = std::min(D.E, D.nKB);
+        const int64_t per_row = p->modcent_per_row > 0 ? std::min<int64_t>(p->modcent_per_row, ecap) : ecap;
+        if (D.rows * per_row >= (int64_t)1 << 30)
+            FAIL(BSA_ERR_UNSUPPORTED, "modified-centroid capacity %lld >= 2^30 entries; lower modcent_per_row",
+                 (long long)(D.rows * per_row));
+    }
     if (p->centroid != 0 && p->centroid != 1) FAIL(BSA_ERR_INVALID_ARG, "centroid must be 0 or 1");
     const int64_t nKB = ceil_div(p->N, p->k_block);
     if (nKB > 65536) FAIL(BSA_ERR_UNSUPPORTED, "N too large: at most 65536 key blocks");
@@ -417,12 +442,15 @@ bsa_status bsa_attention_run(const bsa_params *p, const void *q, const void *k, 
                           ws, ws_bytes, stream, 2);
 }
 
+int64_t bsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
 bsa_status bsa_selftest_bounded_wait(void *ws, int64_t cycles, void *stream)
 {
     g_err[0] = 0;
     if (ws == nullptr) FAIL(BSA_ERR_INVALID_ARG, "ws is NULL");
     if (!aligned16(ws)) FAIL(BSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
     if (cycles < 1 || cycles > 2000000000LL) FAIL(BSA_ERR_INVALID_ARG, "cycles outside [1, 2e9]");
+    count_launch();
     bounded_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(static_cast<int32_t *>(ws), (long long)cycles);
     return from_cuda(cudaGetLastError(), "bsa_selftest_bounded_wait");
 }

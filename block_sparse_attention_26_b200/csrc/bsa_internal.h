@@ -2,6 +2,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include <algorithm>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -47,7 +49,9 @@ struct Dims {
 
 Dims dims_of(const bsa_params &p);
 
-// Byte offsets of the workspace regions (each 256-byte aligned).
+// Byte offsets of the workspace regions (each 256-byte aligned).  The status
+// word comes first; the selection's scratch and the attention calls' scratch
+// both start after it and share the same bytes (neither reads the other's).
 struct WsLayout {
     size_t status;         // DevStatus
     size_t scores;         // [rows, nKB] f32 block scores (select)
@@ -55,10 +59,19 @@ struct WsLayout {
     size_t counts;         // [rows] i32 kept counts (select)
     size_t scan_tmp;       // [ceil(rows / 4096)] i64 per-tile sums of the counts' scan
     size_t kc16, vc16;     // [B*H, nKB, d] bf16 centroids (attention)
-    size_t xk16, xv16;     // [rows, min(E, nKB), d] bf16 modified centroids (extra tokens)
-    size_t xbias;          // [rows, min(E, nKB)] f32 their log2 token counts
-    size_t xcnt;           // [rows] i32 modified centroids per row
-    size_t xaff;           // [rows, nW] u32 blocks that gave extra tokens
+    // modified centroids (extra tokens): row r's entries are idx = xoff[r] ..
+    // xoff[r] + xcnt[r] - 1; the centroids are stored grouped by source block, entry
+    // idx at slot[idx]
+    int64_t mc_cap;        // capacity, in entries (rows x the per-row average asked for)
+    size_t xk16, xv16;     // [mc_cap, d] bf16 modified centroids, by slot
+    size_t xbias;          // [mc_cap] f32 their log2 token counts, by idx
+    size_t xcnt;           // [rows] i32 modified centroids per row (cut to what fits)
+    size_t xoff;           // [rows + 1] i64 exclusive scan of the uncut counts
+    size_t mc_slot;        // [mc_cap] i32 slot of each idx
+    size_t mc_ent;         // [mc_cap] u64 left-out tokens of each slot
+    size_t mc_cnt3;        // [B*H, nKB, groups] i32 entries per (source block, query-block group)
+    size_t mc_off3;        // [B*H*nKB*groups + 1] i64 its exclusive scan
+    size_t mc_tile;        // scan tile sums for the two scans
     size_t glist;          // [sparse tiles, kGlistCap] u32 extra-token union per fine-pass tile
     size_t glcnt;          // [sparse tiles] i32 its length
     size_t q16, k16, v16;  // [B, N, H, d] bf16 copies of f32 inputs (attention, f32 only)
@@ -149,10 +162,26 @@ cudaError_t launch_qkv_pool(const bsa_params &p, const Dims &D, const void *x, i
                             void *k, void *v, float *qbar, float *kbar, float *vbar, int32_t *blk_count,
                             int32_t *status, cudaStream_t st);
 
+// Query-block groups per (b, h) in the modified-centroid listing (about eight
+// CTAs per SM over the whole problem).
+inline int mc_groups(const Dims &D)
+{
+    const int64_t bh = (int64_t)D.B * D.H;
+    const int64_t g = ceil_div(8 * (int64_t)sm_count(), bh);
+    return (int)std::max<int64_t>(1, std::min<int64_t>(g, D.nQB));
+}
+
+// Exclusive scan of `rows` int32 counts into int64 row_ptr[rows + 1] (tile_sum:
+// ceil(rows / 4096) int64 of scratch).
+cudaError_t launch_scan(const int32_t *cnt, int64_t rows, int64_t *row_ptr, int64_t *tile_sum, cudaStream_t st);
+
 // Extra tokens (E > 0): survivor buffer capacity per row, and the launch.
 int64_t extra_buffer_capacity();
 cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, const void *k,
                          int32_t *extra_idx, int32_t *extra_count, char *ws, const WsLayout &L, cudaStream_t st);
+
+// Counts one kernel launch of this library (read by bsa_launch_count).
+void count_launch();
 
 // Thread-local host error text.
 void set_error(const char *fmt, ...);

@@ -792,6 +792,7 @@ cudaError_t launch_filter(dim3 grid, const CUtensorMap &tm, const ExArgs &a, cud
     const int bytes = (int)FLay<D>::bytes;
     cudaError_t e = cudaFuncSetAttribute(filter_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
+    count_launch();
     filter_kernel<D><<<grid, 320, bytes, st>>>(tm, a);
     return cudaGetLastError();
 }
@@ -838,6 +839,7 @@ cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, 
     cudaError_t e = cudaMemsetAsync(a.ovf, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return e;
     const unsigned g8 = (unsigned)ceil_div(D.rows, 8);
+    count_launch();
     theta_kernel<<<g8, 256, 0, st>>>(a);
     CUtensorMap tm;
     if (!make_k_map(&tm, k, D, p.stride_b, p.stride_n, p.stride_h)) {
@@ -851,7 +853,9 @@ cudaError_t launch_extra(const bsa_params &p, const Dims &D, const float *qbar, 
         e = launch_filter<128>(grid, tm, a, st);
     }
     if (e != cudaSuccess) return e;
+    count_launch();
     finalize_kernel<<<g8, 256, 0, st>>>(a);
+    count_launch();
     fallback_kernel<<<(unsigned)fallback_ctas(), 256, 0, st>>>(a);
     return cudaGetLastError();
 }

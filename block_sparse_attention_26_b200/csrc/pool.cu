@@ -172,6 +172,7 @@ cudaError_t launch_pool(const bsa_params &p, const Dims &D, const void *q, const
     a.ncx = D.cube ? p.grid_w / p.cube_w : 1;
     a.ncy = D.cube ? p.grid_h / p.cube_h : 1;
     dim3 grid(std::max(D.nQB, D.nKB), D.B, 3);
+    count_launch();
     if (p.dtype == BSA_DT_BF16)
         pool_kernel<__nv_bfloat16, 8><<<grid, 128, 0, st>>>(a);
     else

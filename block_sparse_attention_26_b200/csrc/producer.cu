@@ -353,6 +353,7 @@ cudaError_t launch_qkv_pool(const bsa_params &p, const Dims &D, const void *x, i
     cudaError_t e = cudaFuncSetAttribute(qkv_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(a.ntiles, sm_count());
+    count_launch();
     qkv_pool_kernel<<<grid, kPThreads, smem, st>>>(tx, tw, tq, tk, tv, a);
     return cudaGetLastError();
 }

@@ -929,14 +929,19 @@ template <int D>
 cudaError_t launch_route_d(const RouteArgs &a, cudaStream_t st)
 {
     const int64_t BH = (int64_t)a.B * a.H;
+    count_launch();
     route_prep_kernel<<<(unsigned)ceil_div(BH * a.nKBp, 8), 256, 0, st>>>(a);
+    count_launch();
     knmax_kernel<<<(unsigned)ceil_div(BH * (a.nKBp / 32), 256), 256, 0, st>>>(a);
+    count_launch();
     gram_kernel<D><<<dim3((unsigned)(a.nsplit * (D == 128 ? 3 : 1)), (unsigned)BH), 256, 0, st>>>(a);
+    count_launch();
     gram_reduce_kernel<D><<<dim3(D * D / 256, (unsigned)BH), 256, 0, st>>>(a);
     const int rs_smem = D * D * 8 + D * kTM * 4 + (D + 3) * 8;
     cudaError_t e = cudaFuncSetAttribute(rowstat_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, rs_smem);
     if (e != cudaSuccess) return e;
     const dim3 gt((unsigned)ceil_div(a.nQB, kTM), (unsigned)BH);
+    count_launch();
     rowstat_kernel<D><<<gt, D * 4, rs_smem, st>>>(a);
     CUtensorMap tm;
     if (!make_k16_map(&tm, a.k16, (int)BH, a.nKB, D)) {
@@ -950,6 +955,7 @@ cudaError_t launch_route_d(const RouteArgs &a, cudaStream_t st)
     }
     e = cudaFuncSetAttribute(decide_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
+    count_launch();
     decide_kernel<D><<<gt, 320, bytes, st>>>(tm, a);
     const unsigned g8 = (unsigned)ceil_div(a.rows, 8);
     const int fb_smem = a.nKBp <= kFbSmem ? a.nKBp * 4 : 0;
@@ -957,7 +963,9 @@ cudaError_t launch_route_d(const RouteArgs &a, cudaStream_t st)
         e = cudaFuncSetAttribute(fallback_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, fb_smem);
         if (e != cudaSuccess) return e;
     }
+    count_launch();
     fallback_rows_kernel<<<(unsigned)fallback_ctas(), 512, fb_smem, st>>>(a);
+    count_launch();
     route_count_kernel<<<g8, 256, 0, st>>>(a);
     return cudaGetLastError();
 }

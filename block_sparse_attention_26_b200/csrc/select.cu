@@ -314,15 +314,6 @@ __global__ void __launch_bounds__(256) scan_add_kernel(int64_t *__restrict__ row
         row_ptr[r] += tile_off[r / kScanTile];
 }
 
-cudaError_t launch_scan(const int32_t *cnt, int64_t rows, int64_t *row_ptr, int64_t *tile_sum, cudaStream_t st)
-{
-    const int ntiles = (int)ceil_div(rows, kScanTile);
-    scan_tiles_kernel<<<(unsigned)ntiles, 1024, 0, st>>>(cnt, rows, row_ptr, tile_sum);
-    scan_tops_kernel<<<1, 1024, 0, st>>>(tile_sum, ntiles, row_ptr, rows);
-    const unsigned g = (unsigned)std::min<int64_t>(ceil_div(rows, 256), (int64_t)sm_count() * 8);
-    scan_add_kernel<<<g, 256, 0, st>>>(row_ptr, rows, tile_sum);
-    return cudaGetLastError();
-}
 
 // One warp per row, its words 32 at a time: every lane counts its word's bits
 // and a warp scan gives every word its first output slot.  A sparse word (at
@@ -382,6 +373,19 @@ __global__ void __launch_bounds__(256) expand_kernel(const uint32_t *__restrict_
 
 }  // namespace
 
+cudaError_t launch_scan(const int32_t *cnt, int64_t rows, int64_t *row_ptr, int64_t *tile_sum, cudaStream_t st)
+{
+    const int ntiles = (int)ceil_div(rows, kScanTile);
+    count_launch();
+    scan_tiles_kernel<<<(unsigned)ntiles, 1024, 0, st>>>(cnt, rows, row_ptr, tile_sum);
+    count_launch();
+    scan_tops_kernel<<<1, 1024, 0, st>>>(tile_sum, ntiles, row_ptr, rows);
+    const unsigned g = (unsigned)std::min<int64_t>(ceil_div(rows, 256), (int64_t)sm_count() * 8);
+    count_launch();
+    scan_add_kernel<<<g, 256, 0, st>>>(row_ptr, rows, tile_sum);
+    return cudaGetLastError();
+}
+
 void select_regions(const bsa_params &p, const Dims &D, WsLayout &L, Taker &T)
 {
     const bool route = certified_route(p);
@@ -425,6 +429,7 @@ cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar,
         if (e != cudaSuccess) return e;
         e = launch_scan(cnt, D.rows, row_ptr, tsum, st);
         if (e != cudaSuccess) return e;
+        count_launch();
         expand_kernel<<<g2, 256, 0, st>>>(bm, cnt, row_ptr, D.rows, D.nW, col_capacity, col_idx, kept_count,
                                           status);
         return cudaGetLastError();
@@ -434,6 +439,7 @@ cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar,
     const int smem = (kRows * 128 + kChan * (kKeys + 1)) * (int)sizeof(double);
     cudaError_t e = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    count_launch();
     scores_kernel<<<g1, 256, smem, st>>>(qbar, kbar, D.nQB, D.nKB, D.d, S);
 
     RowArgs a;
@@ -456,9 +462,11 @@ cudaError_t launch_select(const bsa_params &p, const Dims &D, const float *qbar,
     a.keep_diag = p.keep_diag;
     a.bitmask = bm;
     a.count = cnt;
+    count_launch();
     rows_kernel<<<g2, 256, 0, st>>>(a);
     cudaError_t es = launch_scan(cnt, D.rows, row_ptr, tsum, st);
     if (es != cudaSuccess) return es;
+    count_launch();
     expand_kernel<<<g2, 256, 0, st>>>(bm, cnt, row_ptr, D.rows, D.nW, col_capacity, col_idx,
                                       kept_count, status);
     return cudaGetLastError();

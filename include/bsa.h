@@ -112,7 +112,13 @@ typedef struct {
                                       tokens of Q and of K and per 64 centroids), P V in bf16 -- the
                                       B200 form of [STAR] "attention modes" qk_int8_pv_fp16; needs
                                       bf16 inputs, d = 128, extra_tokens 0, method Sol or SLA */
-    int32_t reserved_;
+    int32_t modcent_per_row;       /* E > 0: the workspace holds rows * modcent_per_row modified
+                                      centroids in all (one per block that gave extra tokens and keeps
+                                      some; a row may use more than this as long as the total fits);
+                                      0 = min(E, nKB) per row, always enough.  If the rows' total
+                                      exceeds the capacity, the status word reports BSA_ERR_CAPACITY
+                                      and the rows past it lose the modified centroids that did not
+                                      fit (their other terms are unchanged). */
 } bsa_params;
 
 /* Fill *p with the defaults of the node documentation for `method`
@@ -123,7 +129,11 @@ BSA_API void bsa_default_params(bsa_params *p, int32_t method);
 
 /* Bytes of device workspace the select and attention calls need for these
  * parameters (*bytes), and the largest possible number of kept entries,
- * B*H*nQB*nKB (*max_nnz), an always-sufficient CSR capacity. */
+ * B*H*nQB*nKB (*max_nnz), an always-sufficient CSR capacity.  The scratch of
+ * bsa_select and that of the attention calls share the same bytes (nothing of
+ * one is read by the other; the status word is kept apart): calls that share a
+ * workspace must not overlap on the GPU (issue them on one stream, or order
+ * the streams). */
 BSA_API bsa_status bsa_workspace_size(const bsa_params *p, size_t *bytes, int64_t *max_nnz);
 
 /* Step 1, pooling ([STAR] "SLA", "Sol": Q/K blocks; K/V centroids).
@@ -249,6 +259,11 @@ BSA_API bsa_status bsa_dense_ref_rows(const bsa_params *p, const void *q, const 
  * last call (BSA_OK if none) in *device_status, and clear it.  The return value
  * is BSA_ERR_CUDA if the synchronisation itself failed. */
 BSA_API bsa_status bsa_device_status(void *ws, void *stream, int32_t *device_status);
+
+/* Kernels this library has launched since it was loaded, from every thread and
+ * on every device (a diagnostic: the difference across a stretch of calls is
+ * the number of kernel launches those calls made). */
+BSA_API int64_t bsa_launch_count(void);
 
 /* Self-test of the kernels' bounded waits (not a step of the method): one warp
  * waits on an mbarrier that nothing ever arrives on, with a limit of `cycles`

@@ -39,6 +39,7 @@ def test_params_struct_layout():
     assert bsa.bsa_params.grid_t.offset == 100
     assert bsa.bsa_params.cube_w.offset == 120
     assert bsa.bsa_params.qk_fp8.offset == 124
+    assert bsa.bsa_params.modcent_per_row.offset == 128
 
 
 def _p(**kw):
@@ -74,6 +75,7 @@ FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced (validati
     ("extra_tokens", 300, binding.BSA_ERR_INVALID_ARG),
     ("sink_blocks", -1, binding.BSA_ERR_INVALID_ARG),
     ("centroid", 2, binding.BSA_ERR_INVALID_ARG),
+    ("modcent_per_row", -1, binding.BSA_ERR_INVALID_ARG),
 ])
 def test_bad_params_rejected(field, value, code):
     p = _p(**{field: value})
@@ -161,3 +163,24 @@ def test_defaults_follow_node_documentation():
     assert (p.tau, p.q_block, p.k_block, p.centroid, p.sink_blocks, p.keep_diag) == (1.3, 64, 64, 1, 1, 1)
     bsa.lib.bsa_default_params(ctypes.byref(p), binding.BSA_SLA)
     assert (p.keep_percent, p.q_block, p.centroid) == (10.0, 128, 0)
+
+
+def test_modified_centroid_capacity_sizes_the_workspace():
+    """The modified centroids take rows x modcent_per_row entries (0: min(E, nKB)
+    per row), and the selection's scratch shares its bytes with the attention
+    calls': on the 76k-token, 40-head workload with 256 extra tokens and 88
+    entries per query block the workspace stays under 2.5 GB."""
+    from workloads import CONFIGS
+    w = CONFIGS["sol_sinks"]
+    q = torch.empty((w.B, w.N, w.H, w.d), dtype=torch.bfloat16, device="meta")
+    p = bsa.params_for(w, q)
+    assert p.modcent_per_row == 88
+    tight, _ = bsa.bsa_workspace_size(p)
+    assert tight <= 2.5e9
+    p.modcent_per_row = 0
+    worst, _ = bsa.bsa_workspace_size(p)
+    p.modcent_per_row = 10_000                 # more than min(E, nKB) = 256: the worst case
+    assert bsa.bsa_workspace_size(p)[0] == worst
+    # 2 (K and V) x 128 channels x 2 bytes, plus the bias, the slot and the mask, per entry
+    entries = w.rows * (256 - 88)
+    assert worst - tight >= entries * (2 * 128 * 2 + 4 + 4 + 8) - 4096

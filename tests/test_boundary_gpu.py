@@ -7,6 +7,7 @@ what bsa_attention gives.  The bounded-wait self-test makes one wait run out
 own, report code 7 (timeout) through the workspace status word, and leave the
 context usable for the next launch.
 """
+import numpy as np
 import pytest
 import torch
 
@@ -42,6 +43,49 @@ def test_prepare_then_run_equals_attention(w):
     assert bsa.bsa_device_status(buf.ws) == 0
     assert torch.equal(out_a, out_b)
     assert torch.equal(lse_a, lse_b)
+
+
+def _modified_centroids_needed(w, extra_idx, extra_count):
+    """Entries the modified-centroid arrays need: per query block, the blocks its
+    extra tokens came from that keep at least one token."""
+    ei, ec = extra_idx.cpu().numpy(), extra_count.cpu().numpy()
+    total = 0
+    for r in range(ei.shape[0]):
+        blk, cnt = np.unique(ei[r, :ec[r]] // 64, return_counts=True)
+        total += int(np.sum(np.minimum(64, w.N - 64 * blk) - cnt > 0))
+    return total
+
+
+def _layer_with_capacity(w, q, k, v, per_row):
+    p = bsa.params_for(w, q)
+    p.modcent_per_row = per_row
+    buf = bsa.Buffers(p, q.device)
+    out = torch.empty_like(q)
+    bsa.run_layer(p, q, k, v, out, buf)
+    return buf, out, bsa.bsa_device_status(buf.ws)
+
+
+def test_modified_centroid_capacity():
+    """A capacity that holds exactly the entries the inputs need gives, bit for bit,
+    the worst-case capacity's result; a smaller one is reported through the status
+    word (BSA_ERR_CAPACITY) without a fault, and the next call runs clean."""
+    w = CASES[0].replace(name="capacity", extra_tokens=256, N=3000, grid=(3, 20, 50), prefix_len=0,
+                         dense_rows=(0, 0), seed=64)
+    q, k, v = (t.cuda() for t in make_qkv(w, "cpu"))
+    buf0, out0, st0 = _layer_with_capacity(w, q, k, v, 0)
+    assert st0 == 0
+    need = _modified_centroids_needed(w, buf0.extra_idx, buf0.extra_count)
+    assert need > w.rows                                   # several per query block
+    per_row = -(-need // w.rows)
+    buf1, out1, st1 = _layer_with_capacity(w, q, k, v, per_row)
+    assert st1 == 0
+    assert torch.equal(out0, out1)
+    _, out2, st2 = _layer_with_capacity(w, q, k, v, 1)
+    assert st2 == bsa.BSA_ERR_CAPACITY
+    assert bool(torch.isfinite(out2.float()).all())
+    _, out3, st3 = _layer_with_capacity(w, q, k, v, per_row)
+    assert st3 == 0
+    assert torch.equal(out0, out3)
 
 
 def test_bounded_wait_times_out_and_reports():

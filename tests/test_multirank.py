@@ -46,8 +46,9 @@ def _rank_main(rank, world, port, out):
         ms = 10.0 + 5.0 * rank                      # rank 1 is the slow one
         slowest = bench.max_over_ranks(ms, dist, "cpu")
         tput = bench.job_throughput(w, world, slowest)
+        launches = bench.sum_over_ranks(100 + rank, dist, "cpu")
         dist.barrier()
-        out.put((rank, w.seed, float(q.float().sum()), slowest, tput))
+        out.put((rank, w.seed, float(q.float().sum()), slowest, tput, launches))
     finally:
         dist.destroy_process_group()
 
@@ -58,10 +59,11 @@ def test_two_gloo_ranks_weak_scaling():
     out = ctx.SimpleQueue()
     mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True, start_method="spawn")
     res = sorted(out.get() for _ in range(world))
-    (r0, seed0, sum0, slow0, tp0), (r1, seed1, sum1, slow1, tp1) = res
+    (r0, seed0, sum0, slow0, tp0, n0), (r1, seed1, sum1, slow1, tp1, n1) = res
     assert (r0, r1) == (0, 1)
     assert seed0 != seed1 and sum0 != sum1          # each rank draws its own inputs
     assert slow0 == slow1 == 15.0                   # both see the slowest rank's time
+    assert n0 == n1 == 201                          # launch counts add up over the job
     w = CONFIGS["tiny_sol"]
     expect = world * bench.dense_equiv_flops(w) / (15.0e-3) / 1e12
     assert tp0 == pytest.approx(expect) and tp1 == pytest.approx(expect)
@@ -139,6 +141,7 @@ def test_single_rank_helpers_are_identities():
     w = CONFIGS["sol_mid"]
     assert bench.rank_workload(w, 0, 1) == w
     assert bench.max_over_ranks(3.5, None, "cpu") == 3.5
+    assert bench.sum_over_ranks(7, None, "cpu") == 7
     assert bench.job_throughput(w, 1, 1000.0) == pytest.approx(bench.dense_equiv_flops(w) / 1e12)
 
 

@@ -51,6 +51,7 @@ class Workload:
     grid: Optional[Tuple[int, int, int]] = None   # latent grid (T, Hs, Ws); None = iid tokens
     cube: Tuple[int, int, int] = (4, 4, 4)         # vsa: cube extents (t, y, x)
     qk_fp8: bool = False                           # fine pass with S = Q K^T in fp8 (e4m3)
+    modcent_per_row: int = 0                       # modified-centroid capacity per query block (0: worst case)
     seed: int = 0
     field_sigma: float = 4.0
     noise: float = 0.5
@@ -82,7 +83,8 @@ SLA_TOPK = Workload("sla_topk", B=1, H=24, N=46080, d=128, dtype="bf16", method=
                     grid=(12, 48, 80), seed=3000)
 SOL_SINKS = Workload("sol_sinks", B=1, H=40, N=76112, d=128, dtype="bf16", method="sol",
                      q_block=64, k_block=64, tau=1.3, prefix_len=512, dense_rows=(256, 512),
-                     extra_tokens=256, centroid=1, grid=(21, 45, 80), seed=4000)
+                     extra_tokens=256, centroid=1, grid=(21, 45, 80), seed=4000,
+                     modcent_per_row=88)   # these inputs need 83.9 per query block on average
 LONG = Workload("long", B=1, H=40, N=207872, d=128, dtype="bf16", method="sol",
                 q_block=64, k_block=64, tau=1.5, prefix_len=512, dense_rows=(256, 512),
                 extra_tokens=0, centroid=1, grid=(24, 90, 96), seed=5000)
