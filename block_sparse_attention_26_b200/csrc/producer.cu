@@ -9,11 +9,17 @@
 // same kernel the block means qbar, kbar, vbar of the rounded outputs (the
 // pooling step), so that the 3*N*d read of a separate pooling pass disappears.
 //
-// Persistent tcgen05 GEMM: 128 x 256 output tiles (M = 128 tokens, N = 256
-// columns = 256 / d heads of one of Q, K, V), K steps of 64 through a 3-deep
-// TMA ring, fp32 accumulators double-buffered in TMEM (512 columns) so that a
-// tile's epilogue overlaps the next tile's MMAs.  Warps 0-3 run the epilogue
-// (TMEM lane quarter = warp), warp 4 loads, warp 5 issues the MMAs.
+// Persistent tcgen05 GEMM on CTA pairs (clusters of 2): 256 x 256 output tiles
+// (M = 256 tokens, 128 per CTA; N = 256 columns = 256 / d heads of one of Q, K,
+// V), one M = 256 UMMA per K = 16 step issued by the even CTA for both
+// (cta_group::2): each CTA holds its 128 rows of X and half of the tile's W rows,
+// so an SM brings in 32 KB of operands per K step of 64 where a one-SM 128 x 256
+// tile needs 48 KB (shared-memory bandwidth is what bounds the one-SM form).
+// K steps of 64 through a 4-deep TMA ring per CTA, both CTAs' loads completing
+// on the even CTA's barrier; fp32 accumulators double-buffered in each CTA's
+// TMEM (512 columns) so that a tile's epilogue overlaps the next tile's MMAs.
+// Warps 0-3 run the epilogue (TMEM lane quarter = warp), warp 4 loads, warp 5
+// issues the MMAs (even CTA) and owns TMEM.
 //
 // Epilogue: each thread takes its row, rounds it to bf16 into a staging tile
 // laid out for a TMA store (128-byte swizzle), the tile is stored by TMA, and
@@ -32,11 +38,11 @@
 namespace bsa {
 namespace {
 
-constexpr int kPM = 128;       // tokens per tile
-constexpr int kPN = 256;       // output columns per tile
+constexpr int kPM = 128;       // tokens per CTA (a pair's tile: 256)
+constexpr int kPN = 256;       // output columns per tile (128 W rows per CTA)
 constexpr int kPK = 64;        // K per stage
-constexpr int kPStages = 3;
-constexpr int kBandM = 48;     // m tiles per raster band (their A tiles stay in L2)
+constexpr int kPStages = 4;
+constexpr int kBandM = 24;     // m tiles (of 256 tokens) per raster band (their A tiles stay in L2)
 constexpr int kPThreads = 192;
 
 struct ProdArgs {
@@ -52,7 +58,7 @@ struct ProdArgs {
 
 struct PLay {
     static constexpr int kABytes = kPM * kPK * 2;           // 16 KB
-    static constexpr int kBBytes = kPN * kPK * 2;           // 32 KB
+    static constexpr int kBBytes = kPN / 2 * kPK * 2;       // 16 KB: this CTA's half of the W rows
     static constexpr int kStage = kABytes + kBBytes;
     static constexpr int kOffStages = 0;
     static constexpr int kOffStg = kPStages * kStage;      // staging tile, 64 KB
@@ -62,6 +68,64 @@ struct PLay {
     static constexpr size_t bytes = (size_t)kOffMisc + 16 + 1024;
     static_assert(bytes <= 232448, "producer tile exceeds the per-block shared memory limit");
 };
+
+// ------------------------------------------------------------ CTA pairs
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The shared::cluster address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_rank(const void *p, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// 2-D tile load into this CTA's shared memory, completing on an mbarrier that may
+// sit in the other CTA of the pair (shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem of both] * B[smem of both]^T, M = 256.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive on `bar` in both CTAs of the pair once every pair MMA issued so far completes.
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar)
+{
+    asm volatile(
+        "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
 
 // Tile t of the raster: bands of kBandM m tiles, n-major inside a band.
 __device__ __forceinline__ void tile_mn(const ProdArgs &a, int t, int *m, int *n)
@@ -82,6 +146,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t crank = cluster_rank();          // 0: the CTA that issues the pair's MMAs
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PLay::kOffBar);
     uint64_t *full = bars, *empty = bars + kPStages, *acc_full = bars + 2 * kPStages, *acc_empty = acc_full + 2;
     uint64_t *stg_full = acc_empty + 2, *stg_free = stg_full + 1;
@@ -93,12 +159,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&full[s], 1);      // (used in CTA 0: its own arrival; both CTAs' bytes)
+            mbar_init(&empty[s], 1);     // released by CTA 0's MMAs, in both CTAs
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 4);
+            mbar_init(&acc_empty[i], 8); // (used in CTA 0: both CTAs' epilogue warps)
         }
         mbar_init(stg_full, 4);
         mbar_init(stg_free, 4);
@@ -106,11 +172,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
         fence_mbar_init();
     }
     if (warp == 5) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();                    // both CTAs' barriers exist before either signals the other
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -120,11 +188,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
             prefetch_tmap(&tm_w);
             int g = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x) {
+            for (int t = pair; t < a.ntiles && ok; t += npairs) {
                 int m, n;
                 tile_mn(a, t, &m, &n);
                 const int b = m / a.tiles_m_b, tm = m % a.tiles_m_b;
-                const int row0 = b * a.N + tm * kPM;
+                const int row0 = b * a.N + tm * (2 * kPM) + (int)crank * kPM;
                 for (int kb = 0; kb < ksteps; ++kb, ++g) {
                     const int s = g % kPStages;
                     if (g >= kPStages && !mbar_wait(&empty[s], ((g / kPStages) - 1) & 1, abort_flag, a.status, 80)) {
@@ -132,58 +200,65 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         break;
                     }
                     uint8_t *st = sm + PLay::kOffStages + s * PLay::kStage;
-                    mbar_expect_tx(&full[s], PLay::kStage);
-                    tma_load_2d(st, &tm_x, &full[s], kb * kPK, row0);
-                    tma_load_2d(st + PLay::kABytes, &tm_w, &full[s], kb * kPK, n * kPN);
+                    // both CTAs' bytes complete on CTA 0's barrier, which CTA 0 arms for them
+                    if (crank == 0) mbar_expect_tx(&full[s], 2 * PLay::kStage);
+                    const uint32_t fb = map_rank(&full[s], 0);
+                    tma_load_2d_pair(st, &tm_x, fb, kb * kPK, row0);
+                    tma_load_2d_pair(st + PLay::kABytes, &tm_w, fb, kb * kPK, n * kPN + (int)crank * (kPN / 2));
                 }
             }
-            // no copy may still be in flight at exit
+            // no copy may still be in flight at exit: the last phase of every slot
+            // has been released by the MMAs that read it (CTA 0 waited for its bytes)
             volatile int32_t no_abort = 0;
             for (int s = 0; s < kPStages; ++s) {
                 const int nfill = (g - s + kPStages - 1) / kPStages;
-                if (nfill > 0) mbar_wait(&full[s], (nfill - 1) & 1, &no_abort, a.status, 81);
+                if (nfill > 0) mbar_wait(&empty[s], (nfill - 1) & 1, &no_abort, a.status, 81);
             }
         }
     } else if (warp == 5) {
-        const uint32_t idesc = idesc_bf16_f32(kPM, kPN, 0, 0);
-        int g = 0, it = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < a.ntiles && ok; t += gridDim.x, ++it) {
-            const int ab = it & 1;
-            if (it >= 2 && !mbar_wait(&acc_empty[ab], ((it >> 1) - 1) & 1, abort_flag, a.status, 82)) break;
-            tc_fence_after();
-            for (int kb = 0; kb < ksteps; ++kb, ++g) {
-                const int s = g % kPStages;
-                if (!mbar_wait(&full[s], (g / kPStages) & 1, abort_flag, a.status, 83)) {
-                    ok = false;
-                    break;
-                }
+        if (crank == 0) {
+            const uint32_t idesc = idesc_bf16_f32(2 * kPM, kPN, 0, 0);
+            int g = 0, it = 0;
+            bool ok = true;
+            for (int t = pair; t < a.ntiles && ok; t += npairs, ++it) {
+                const int ab = it & 1;
+                if (it >= 2 && !mbar_wait(&acc_empty[ab], ((it >> 1) - 1) & 1, abort_flag, a.status, 82)) break;
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t sa = smem_u32(sm + PLay::kOffStages + s * PLay::kStage);
-#pragma unroll
-                    for (int kk = 0; kk < kPK / 16; ++kk) {
-                        const uint64_t ad = sdesc_sw128(sa + kk * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(sa + PLay::kABytes + kk * 32, 16, 1024);
-                        umma_bf16(tmem + 256 * ab, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                for (int kb = 0; kb < ksteps; ++kb, ++g) {
+                    const int s = g % kPStages;
+                    if (!mbar_wait(&full[s], (g / kPStages) & 1, abort_flag, a.status, 83)) {
+                        ok = false;
+                        break;
                     }
-                    umma_commit(&empty[s]);
-                    if (kb == ksteps - 1) umma_commit(&acc_full[ab]);
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t sa = smem_u32(sm + PLay::kOffStages + s * PLay::kStage);
+#pragma unroll
+                        for (int kk = 0; kk < kPK / 16; ++kk) {
+                            const uint64_t ad = sdesc_sw128(sa + kk * 32, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(sa + PLay::kABytes + kk * 32, 16, 1024);
+                            umma_bf16_pair(tmem + 256 * ab, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit_pair(&empty[s]);
+                        if (kb == ksteps - 1) umma_commit_pair(&acc_full[ab]);
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
             }
         }
     } else {
         // ---------------------------------------------------------------- epilogue
-        const int r = threadIdx.x;     // row of the tile = TMEM lane
+        const int r = threadIdx.x;     // row of this CTA's half = TMEM lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const uint32_t acc_empty0[2] = {map_rank(&acc_empty[0], 0), map_rank(&acc_empty[1], 0)};
         int it = 0;
-        for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x, ++it) {
+        for (int t = pair; t < a.ntiles; t += npairs, ++it) {
             const int ab = it & 1;
             int m, n;
             tile_mn(a, t, &m, &n);
             const int b = m / a.tiles_m_b, tm = m % a.tiles_m_b;
-            const int nvalid = min(kPM, a.N - tm * kPM);
+            const int tok0 = tm * (2 * kPM) + (int)crank * kPM;   // this CTA's first token of the batch
+            const int nvalid = min(kPM, a.N - tok0);
             const int col0 = n * kPN;
             const int which = col0 / (a.H * a.d);               // 0: Q, 1: K, 2: V
             const int h0 = (col0 % (a.H * a.d)) / a.d;
@@ -193,7 +268,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
             if (it > 0) ok = mbar_wait(stg_free, (it - 1) & 1, abort_flag, a.status, 85) && ok;
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
-            if (ok) {
+            if (ok && nvalid > 0) {
 #pragma unroll 1
                 for (int cc = 0; cc < kPN / 32; ++cc) {
                     uint32_t v[32];
@@ -214,20 +289,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     }
                 }
             }
-            // the accumulator is in registers / staging: release it to the MMAs
+            // the accumulator is in registers / staging: release it to CTA 0's MMAs
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+            if (lane == 0) mbar_arrive_cluster(acc_empty0[ab]);
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(stg_full);
             ok = mbar_wait(stg_full, it & 1, abort_flag, a.status, 86) && ok;
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            if (r == 0) {
+            if (r == 0 && nvalid > 0) {
                 const CUtensorMap *mo = which == 0 ? &tm_q : (which == 1 ? &tm_k : &tm_v);
                 for (int dc = 0; dc < a.d / 64; ++dc)
-                    tma_store_4d(mo, stg + dc * (kPM * HT * 128), dc * 64, h0, tm * kPM, b);
+                    tma_store_4d(mo, stg + dc * (kPM * HT * 128), dc * 64, h0, tok0, b);
                 bulk_commit();
             }
             // block means of the rounded outputs: one thread per (block, column),
@@ -236,7 +311,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
             const int nblk = kPM / blk;
             const int nb_total = which == 0 ? a.nQB : a.nKB;
             float *dst = which == 0 ? a.qbar : (which == 1 ? a.kbar : a.vbar);
-            for (int item = r; item < nblk * kPN; item += kPM) {
+            for (int item = r; item < nblk * kPN && nvalid > 0; item += kPM) {
                 const int j = item / kPN, ct = item % kPN;
                 const int hh = ct / a.d, ch = ct % a.d, dc = ch >> 6, c = ch & 63;
                 const int r0 = j * blk, r1 = min(nvalid, r0 + blk);
@@ -249,7 +324,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         *reinterpret_cast<const uint16_t *>(base + R * 128 + ((((c >> 3) ^ (R & 7))) << 4) + (c & 7) * 2);
                     sum = __dadd_rn(sum, (double)__uint_as_float((uint32_t)bits << 16));
                 }
-                const int bi = tm * nblk + j;
+                const int bi = tok0 / blk + j;
                 if (bi < nb_total)
                     dst[(((int64_t)b * a.H + h0 + hh) * nb_total + bi) * a.d + ch] =
                         __double2float_rn(sum / (double)(r1 - r0));
@@ -263,9 +338,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();                    // no MMA, copy or arrival of the pair is still aimed at this CTA
     if (warp == 5) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
     }
 }
 
@@ -333,7 +409,7 @@ cudaError_t launch_qkv_pool(const bsa_params &p, const Dims &D, const void *x, i
     a.Bq = D.Bq;
     a.nQB = D.nQB;
     a.nKB = D.nKB;
-    a.tiles_m_b = (int)ceil_div(D.N, kPM);
+    a.tiles_m_b = (int)ceil_div(D.N, 2 * kPM);
     a.tiles_m = a.tiles_m_b * D.B;
     a.tiles_n = 3 * D.H * D.d / kPN;
     a.ntiles = a.tiles_m * a.tiles_n;
@@ -344,7 +420,8 @@ cudaError_t launch_qkv_pool(const bsa_params &p, const Dims &D, const void *x, i
     a.status = status;
     CUtensorMap tx, tw, tq, tk, tv;
     const int ht = kPN / D.d;
-    if (!map_matrix(&tx, x, (int64_t)D.B * D.N, d_model, kPM) || !map_matrix(&tw, w, 3LL * D.H * D.d, d_model, kPN) ||
+    if (!map_matrix(&tx, x, (int64_t)D.B * D.N, d_model, kPM) ||
+        !map_matrix(&tw, w, 3LL * D.H * D.d, d_model, kPN / 2) ||
         !map_out(&tq, q, p, ht) || !map_out(&tk, k, p, ht) || !map_out(&tv, v, p, ht)) {
         set_error("cuTensorMapEncodeTiled failed for the projection");
         return cudaErrorInvalidValue;
@@ -352,10 +429,21 @@ cudaError_t launch_qkv_pool(const bsa_params &p, const Dims &D, const void *x, i
     const size_t smem = PLay::bytes;
     cudaError_t e = cudaFuncSetAttribute(qkv_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = std::min(a.ntiles, sm_count());
+    const int pairs = std::max(1, std::min(a.ntiles, sm_count() / 2));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(kPThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     count_launch();
-    qkv_pool_kernel<<<grid, kPThreads, smem, st>>>(tx, tw, tq, tk, tv, a);
-    return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, qkv_pool_kernel, tx, tw, tq, tk, tv, a);
 }
 
 }  // namespace bsa
