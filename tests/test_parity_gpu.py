@@ -41,6 +41,10 @@ SMALL = {
                             grid=(3, 16, 40), seed=21),
     "sol_extra256": Workload("sol_extra256", B=1, H=2, N=3000, d=128, dtype="bf16", method="sol", q_block=64,
                              k_block=64, tau=1.0, extra_tokens=256, grid=(3, 20, 50), seed=22),
+    # extra tokens with d = 64 and two batches: the modified-centroid build's
+    # 64-channel form and its (batch, head) indexing; a ragged last block
+    "sol_extra_b2_d64": Workload("sol_extra_b2_d64", B=2, H=2, N=1500, d=64, dtype="bf16", method="sol",
+                                 q_block=64, k_block=64, tau=1.0, extra_tokens=64, grid=(3, 10, 50), seed=23),
     "no_diag_no_sink": Workload("no_diag_no_sink", B=1, H=2, N=1300, d=128, dtype="bf16", method="sol",
                                 q_block=64, k_block=64, tau=1.0, sink_blocks=0, keep_diag=0,
                                 grid=(2, 13, 50), seed=18),
