@@ -170,6 +170,50 @@ def kept_flops(w, row_ptr: torch.Tensor, col: torch.Tensor, extra_count=None) ->
     return 4.0 * w.d * (sparse + dense)
 
 
+def issued_flops(w, row_ptr: torch.Tensor, col: torch.Tensor, extra_count=None) -> float:
+    """Tensor-core FLOPs the fine pass issues: every 128-key tile costs
+    4 * 128 * 128 * d (S = Q K^T and P V at M = 128), whatever its masks.  A sparse
+    item (128 query rows: two 64-row query blocks, or one 128-row block) runs
+    ceil(|union of its blocks' kept key blocks| / 2) exact tiles, ceil(ceil(nKB /
+    64) / 2) centroid tiles with centroids, and with extra tokens at least
+    ceil(their count / 128) gathered tiles (both blocks' lists counted in full;
+    the modified centroids beside them are left out); items whose rows all lie in
+    the dense range are skipped; the dense rows' 128-row tiles each run
+    ceil(nKB / 2) tiles.  Against kept_flops this is the pairing's overwork."""
+    rp = row_ptr.to(torch.int64)
+    rows = w.B * w.H * w.nQB
+    nnz = int(rp[-1])
+    cnt = rp[1:] - rp[:-1]
+    row_of = torch.repeat_interleave(torch.arange(rows, device=col.device), cnt)
+    mask = torch.zeros((rows, w.nKB), dtype=torch.bool, device=col.device)
+    mask[row_of, col[:nnz].to(torch.int64)] = True
+    mask = mask.view(w.B * w.H, w.nQB, w.nKB)
+    per = 128 // w.q_block                        # query blocks per item
+    n_items = -(-w.N // 128)
+    if w.nQB % per:
+        mask = torch.cat([mask, torch.zeros((w.B * w.H, per - w.nQB % per, w.nKB), dtype=torch.bool,
+                                              device=mask.device)], 1)
+    union = mask.view(w.B * w.H, n_items, per, w.nKB).any(2).sum(2)          # [BH, items]
+    tiles = (union + 1) // 2
+    if w.centroid:
+        tiles = tiles + (-(-w.nKB // 64) + 1) // 2
+    if extra_count is not None and w.extra_tokens > 0:
+        ec = extra_count.to(torch.int64).view(w.B * w.H, w.nQB)
+        if w.nQB % per:
+            ec = torch.cat([ec, torch.zeros((w.B * w.H, per - w.nQB % per), dtype=torch.int64, device=ec.device)], 1)
+        tiles = tiles + (ec.view(w.B * w.H, n_items, per).sum(2) + 127) // 128
+    r0, r1 = w.dense_rows
+    live = torch.ones(n_items, dtype=torch.bool, device=tiles.device)
+    if r1 > r0:
+        for it in range(n_items):
+            if it * 128 >= r0 and min(it * 128 + 128, w.N) <= r1:
+                live[it] = False
+    total = int((tiles * live.view(1, -1)).sum())
+    if r1 > r0:
+        total += w.B * w.H * (-(-(r1 - r0) // 128)) * ((w.nKB + 1) // 2)
+    return 4.0 * 128 * 128 * w.d * total
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -485,6 +529,7 @@ def main():
     if status != 0:
         raise SystemExit(f"device status {status} after warm-up")
     flops_kept = kept_flops(w, buf.row_ptr, buf.col_idx, buf.extra_count)
+    flops_issued = issued_flops(w, buf.row_ptr, buf.col_idx, buf.extra_count)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -570,6 +615,9 @@ def main():
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peak_src} bf16_tflops (burst: the kernel runs inside a sub-second step)",
                      "frac_of_sustained": achieved / peak_sus,
+                     "issued_tflop": flops_issued / 1e12,
+                     "issued_achieved": flops_issued / (fine_ms * 1e-3) / 1e12,
+                     "frac_issued": flops_issued / (fine_ms * 1e-3) / 1e12 / peak,
                      "traffic": attn_traffic(w),
                      "traffic_unit": "bytes per launch (ncu dram read+write, scaled from a 4-head capture)"},
         "roofline_select": {"bound": "hbm", "peak": hbm, "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs",
