@@ -557,13 +557,16 @@ def main():
     ph_ms["attention"] = ph_ms["attention_prepare"] + ph_ms["attention_fine_pass"]
     ms_step = total_ms / args.steps
 
-    # end to end through the public API with host buffers: H2D of this rank's
-    # Q/K/V heads, the layer, D2H of the output, every step
+    # end to end through the public API with host buffers: every step, H2D of this
+    # rank's Q/K/V heads, the layer, D2H of the output -- bsa_layer_host, which
+    # takes the heads in chunks so that one chunk's copies overlap another's kernels
     e2e = None
     if args.e2e_steps > 0:
         hq, hk, hv = (t.contiguous().cpu().pin_memory() for t in (q, k, v))
-        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        dq, dk, dv = torch.empty_like(hq, device=dev), torch.empty_like(hk, device=dev), torch.empty_like(hv, device=dev)
+        hout = torch.empty(hq.shape, dtype=hq.dtype, pin_memory=True)
+        pe = params_for(w, hq)
+        hl = bsa.HostLayer(pe, dev)
+        cin, cout = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if pg:
             pg.barrier()
@@ -571,18 +574,18 @@ def main():
             if i == 1:
                 torch.cuda.synchronize(dev)
                 s0.record(stream)
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            bsa.run_layer(p, dq, dk, dv, out, buf, stream)
-            hout.copy_(out, non_blocking=True)
-        s1.record(stream)
+            bsa.bsa_layer_host(pe, hq, hk, hv, hout, hl, stream, cin, cout)
+        s1.record(stream)   # the call leaves `stream` waiting for its last copy back
         torch.cuda.synchronize(dev)
+        if bsa.bsa_device_status(hl.buf.ws, stream) != 0:
+            raise SystemExit("device status after the end-to-end steps")
         e2e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps, pg, dev)
         nbytes = q.numel() * q.element_size()
         e2e = {"value": job_throughput(w_job, world, e2e_ms, split), "unit": UNIT,
-               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms}
-        del hq, hk, hv, hout, dq, dk, dv
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_ms,
+               "heads_per_chunk": hl.hc}
+        dq = dk = dv = None
+        del hq, hk, hv, hout, dq, dk, dv, hl
 
     peaks, peak_src = _peaks()
     peak = float(peaks.get("bf16_tflops"))

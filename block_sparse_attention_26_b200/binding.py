@@ -46,6 +46,17 @@ class bsa_params(ctypes.Structure):
     ]
 
 
+class bsa_layer_device(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("qbar", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("vbar", ctypes.c_void_p),
+        ("blk_count", ctypes.c_void_p), ("row_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
+        ("col_capacity", ctypes.c_int64), ("kept_count", ctypes.c_void_p),
+        ("extra_idx", ctypes.c_void_p), ("extra_count", ctypes.c_void_p),
+        ("ws", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t),
+    ]
+
+
 class bsa_policy(ctypes.Structure):
     _fields_ = [
         ("start_percent", ctypes.c_double), ("end_percent", ctypes.c_double),
@@ -84,6 +95,7 @@ def _load() -> ctypes.CDLL:
     lib.bsa_launch_count.argtypes = []
     lib.bsa_launch_count.restype = I64
     lib.bsa_dense_ref_rows.argtypes = [PP, P, P, P, I32, I32, P, P, P, SZ, P]
+    lib.bsa_layer_host.argtypes = [PP, P, P, P, P, ctypes.POINTER(bsa_layer_device), I32, P, P, P]
     lib.bsa_device_status.argtypes = [P, P, ctypes.POINTER(I32)]
     PolP = ctypes.POINTER(bsa_policy)
     lib.bsa_default_policy.argtypes = [PolP]
@@ -96,7 +108,7 @@ def _load() -> ctypes.CDLL:
     lib.bsa_last_error.restype = ctypes.c_char_p
     for f in ("bsa_workspace_size", "bsa_pool", "bsa_qkv_pool", "bsa_select", "bsa_select_static", "bsa_attention",
               "bsa_attention_prepare", "bsa_attention_run", "bsa_dense_ref_rows", "bsa_device_status",
-              "bsa_selftest_bounded_wait"):
+              "bsa_selftest_bounded_wait", "bsa_layer_host"):
         getattr(lib, f).restype = I32
     return lib
 
@@ -105,7 +117,8 @@ lib = _load()
 
 EXPORTED = ("bsa_default_params", "bsa_workspace_size", "bsa_pool", "bsa_qkv_pool", "bsa_select", "bsa_select_static",
             "bsa_attention", "bsa_attention_prepare", "bsa_attention_run", "bsa_dense_ref_rows",
-            "bsa_device_status", "bsa_selftest_bounded_wait", "bsa_launch_count", "bsa_default_policy",
+            "bsa_device_status", "bsa_selftest_bounded_wait", "bsa_launch_count", "bsa_layer_host",
+            "bsa_default_policy",
             "bsa_policy_decide",
             "bsa_status_string", "bsa_last_error")
 
@@ -302,6 +315,43 @@ class Buffers:
         self.ws = torch.zeros((ws_bytes + 255) // 256 * 256, dtype=torch.uint8, device=device)
         self.lse = torch.empty((p.B, p.H, p.N), dtype=f32, device=device)
         del BH
+
+
+class HostLayer:
+    """Device buffers for bsa_layer_host: the whole layer's Q, K, V and O
+    ([B, N, H, d], contiguous, as p's strides must be) and one chunk's buffers
+    (heads_per_chunk heads; 0: about a sixteenth of them, as the library chooses)."""
+
+    def __init__(self, p: bsa_params, device, heads_per_chunk: int = 0):
+        if (p.stride_h, p.stride_n, p.stride_b) != (p.d, p.H * p.d, p.N * p.H * p.d):
+            raise ValueError("HostLayer needs contiguous [B, N, H, d] strides")
+        hc = heads_per_chunk if heads_per_chunk > 0 else max(1, (p.H + 15) // 16)
+        self.hc = min(hc, p.H)
+        dt = torch.bfloat16 if p.dtype == BSA_DT_BF16 else torch.float32
+        shape = (p.B, p.N, p.H, p.d)
+        self.q, self.k, self.v, self.out = (torch.empty(shape, dtype=dt, device=device) for _ in range(4))
+        pc = bsa_params.from_buffer_copy(p)
+        pc.H = self.hc
+        self.buf = Buffers(pc, device)
+        b = self.buf
+        self.dev = bsa_layer_device(
+            _vp(self.q), _vp(self.k), _vp(self.v), _vp(self.out), _vp(b.qbar), _vp(b.kbar), _vp(b.vbar),
+            _vp(b.blk_count), _vp(b.row_ptr), _vp(b.col_idx), b.col_idx.numel(), _vp(b.kept_count),
+            _vp(b.extra_idx), _vp(b.extra_count), _vp(b.ws), b.ws.numel())
+
+
+def _vp(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def bsa_layer_host(p: bsa_params, q_host, k_host, v_host, out_host, hl: HostLayer, stream=None,
+                   copy_in=None, copy_out=None):
+    """One layer from pinned host tensors (bsa_layer_host); copy_in / copy_out are
+    torch streams for the copies (None: everything on `stream`)."""
+    cin = None if copy_in is None else ctypes.c_void_p(copy_in.cuda_stream)
+    cout = None if copy_out is None else ctypes.c_void_p(copy_out.cuda_stream)
+    _check(lib.bsa_layer_host(ctypes.byref(p), _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(out_host),
+                              ctypes.byref(hl.dev), hl.hc, _stream(stream), cin, cout), "bsa_layer_host")
 
 
 def run_step(p: bsa_params, pol: bsa_policy, q, k, v, out, buf: Buffers, block_index: int, progress: float,

@@ -15,7 +15,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbsa.so")
-SOURCES = ["bsa_api.cu", "pool.cu", "select.cu", "route.cu", "extra.cu", "attention.cu", "policy.cu", "producer.cu"]
+SOURCES = ["bsa_api.cu", "pool.cu", "select.cu", "route.cu", "extra.cu", "attention.cu", "policy.cu", "producer.cu",
+           "layer.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",

@@ -255,6 +255,41 @@ BSA_API bsa_status bsa_dense_ref_rows(const bsa_params *p, const void *q, const 
                               int32_t row_begin, int32_t row_end, void *out, float *lse,
                               void *ws, size_t ws_bytes, void *stream);
 
+/* Device buffers for bsa_layer_host.  q, k, v, out hold the whole layer ([B, N,
+ * H, d] with p's strides); the others serve one chunk of heads at a time, sized
+ * for heads_per_chunk heads as bsa_pool / bsa_select / bsa_attention describe
+ * them (qbar [B, hc, nQB, d], kbar and vbar [B, hc, nKB, d], blk_count [nKB],
+ * row_ptr [B*hc*nQB + 1], col_idx [col_capacity], kept_count [B*hc*nQB], and
+ * with E > 0 extra_idx [B*hc*nQB, E] and extra_count [B*hc*nQB]); ws holds at
+ * least bsa_workspace_size() bytes for p with H = heads_per_chunk. */
+typedef struct {
+    void *q, *k, *v, *out;
+    float *qbar, *kbar, *vbar;
+    int32_t *blk_count;
+    int64_t *row_ptr;
+    int32_t *col_idx;
+    int64_t col_capacity;
+    int32_t *kept_count;
+    int32_t *extra_idx, *extra_count;
+    void *ws;
+    size_t ws_bytes;
+} bsa_layer_device;
+
+/* One layer (pool, select, attention, dense rows) whose inputs and output live
+ * in host memory: heads are independent, so the layer runs chunk by chunk of
+ * heads_per_chunk heads (0: about a sixteenth of them), the copy of chunk c + 1's
+ * Q, K, V to the device (on copy_in) and of chunk c - 1's output back (on
+ * copy_out) overlapping chunk c's kernels (on stream).  A host array has p's
+ * strides, and a chunk is copied as rows of its heads (cudaMemcpy2DAsync);
+ * pinned host memory lets the copies run asynchronously.  copy_in / copy_out
+ * NULL: everything on `stream`, in order.  No LSE is produced.  Returns after
+ * enqueueing; `stream` then waits for the last copy back, so synchronising it
+ * (or bsa_device_status(dev->ws, stream, ...)) covers the whole layer.
+ * Device-side errors of any chunk go to the status word of dev->ws. */
+BSA_API bsa_status bsa_layer_host(const bsa_params *p, const void *q_host, const void *k_host, const void *v_host,
+                                  void *out_host, const bsa_layer_device *dev, int32_t heads_per_chunk,
+                                  void *stream, void *copy_in, void *copy_out);
+
 /* Synchronise `stream`, return the status the kernels wrote into `ws` since the
  * last call (BSA_OK if none) in *device_status, and clear it.  The return value
  * is BSA_ERR_CUDA if the synchronisation itself failed. */

@@ -184,3 +184,20 @@ def test_modified_centroid_capacity_sizes_the_workspace():
     # 2 (K and V) x 128 channels x 2 bytes, plus the bias, the slot and the mask, per entry
     entries = w.rows * (256 - 88)
     assert worst - tight >= entries * (2 * 128 * 2 + 4 + 4 + 8) - 4096
+
+
+def test_layer_host_arguments_checked():
+    """bsa_layer_host rejects missing arrays, a layout whose heads are not side by
+    side, and a negative chunk size before doing anything."""
+    p = _p()
+    dev = binding.bsa_layer_device()
+    st = bsa.lib.bsa_layer_host(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, None, 0, None, None, None)
+    assert st == binding.BSA_ERR_INVALID_ARG
+    st = bsa.lib.bsa_layer_host(ctypes.byref(p), None, FAKE, FAKE, FAKE, ctypes.byref(dev), 0, None, None, None)
+    assert st == binding.BSA_ERR_INVALID_ARG
+    st = bsa.lib.bsa_layer_host(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, ctypes.byref(dev), -1, None, None, None)
+    assert st == binding.BSA_ERR_INVALID_ARG
+    p.stride_h, p.stride_n = p.N * p.d, p.d           # [B, H, N, d] storage
+    st = bsa.lib.bsa_layer_host(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, ctypes.byref(dev), 0, None, None, None)
+    assert st == binding.BSA_ERR_INVALID_ARG
+    assert bsa.lib.bsa_last_error().decode() != ""

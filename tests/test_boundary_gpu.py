@@ -88,6 +88,38 @@ def test_modified_centroid_capacity():
     assert torch.equal(out0, out3)
 
 
+@pytest.mark.parametrize("case", ["extra_dense_hc1", "b2_ragged_hc2"])
+def test_layer_from_host_memory_equals_device_layer(case):
+    """bsa_layer_host (heads in chunks, copies on their own streams overlapping the
+    kernels) gives, bit for bit, what the whole layer run on device arrays gives:
+    heads are independent, and with at most 256 key blocks the dense rows are not
+    split over keys, so every chunk computes exactly what the whole layer does."""
+    w, hc = {
+        "extra_dense_hc1": (CASES[0], 1),
+        "b2_ragged_hc2": (Workload("host_b2", B=2, H=5, N=1500, d=128, dtype="bf16", method="sol", q_block=64,
+                                   k_block=64, tau=1.0, grid=(3, 10, 50), seed=65), 2),
+    }[case]
+    qc, kc, vc = make_qkv(w, "cpu")
+    q, k, v = (t.cuda() for t in (qc, kc, vc))
+    p = bsa.params_for(w, q)
+    buf = bsa.Buffers(p, q.device)
+    ref = torch.empty_like(q)
+    bsa.run_layer(p, q, k, v, ref, buf)
+    assert bsa.bsa_device_status(buf.ws) == 0
+    hq, hk, hv = (t.contiguous().pin_memory() for t in (qc, kc, vc))
+    hout = torch.full(hq.shape, float("nan"), dtype=hq.dtype).pin_memory()
+    hl = bsa.HostLayer(p, q.device, hc)
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+    for _ in range(2):                                   # twice: the second call reuses every buffer
+        bsa.bsa_layer_host(p, hq, hk, hv, hout, hl, None, cin, cout)
+        assert bsa.bsa_device_status(hl.buf.ws) == 0     # synchronises the stream the call ended on
+        assert torch.equal(hout, ref.cpu())
+        hout.fill_(float("nan"))
+    bsa.bsa_layer_host(p, hq, hk, hv, hout, hl)          # one stream for everything
+    assert bsa.bsa_device_status(hl.buf.ws) == 0
+    assert torch.equal(hout, ref.cpu())
+
+
 def test_bounded_wait_times_out_and_reports():
     ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
