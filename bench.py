@@ -369,6 +369,7 @@ def _config_json(w, world, split="replicas", heads=None):
             "prefix_len": w.prefix_len, "dense_rows": list(w.dense_rows), "extra_tokens": w.extra_tokens,
             "centroid": w.centroid, "grid": list(w.grid) if w.grid else None,
             "qk_fp8": bool(getattr(w, "qk_fp8", False)),
+            "pv_fp8": bool(getattr(w, "pv_fp8", False)),
             "parallelism": par,
             "l2": "inputs larger than L2 (126 MB); no flush" if 3 * w.B * w.N * w.H * w.d * 2 > 126e6
             else "L2 flushed between steps"}
@@ -450,6 +451,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--heads", type=int, default=0, help="override H (profiling a smaller case)")
     ap.add_argument("--qk-fp8", action="store_true", help="fine pass with S = Q K^T in fp8 (e4m3)")
+    ap.add_argument("--pv-fp8", action="store_true", help="with --qk-fp8: P V in fp8 (e4m3) as well")
     ap.add_argument("--producer", action="store_true",
                     help="time the QKV projection with pooling in its epilogue against cuBLAS + bsa_pool")
     args = ap.parse_args()
@@ -461,7 +463,9 @@ def main():
     if args.heads > 0:
         w_job = w_job.replace(H=args.heads)
     if args.qk_fp8:
-        w_job = w_job.replace(qk_fp8=True)
+        w_job = w_job.replace(qk_fp8=True, pv_fp8=bool(args.pv_fp8))
+    elif args.pv_fp8:
+        raise SystemExit("--pv-fp8 needs --qk-fp8")
     split = args.split if world > 1 else "replicas"
     if split == "replicas":
         w_job = rank_workload(w_job, rank, world)
@@ -588,8 +592,12 @@ def main():
         del hq, hk, hv, hout, dq, dk, dv, hl
 
     peaks, peak_src = _peaks()
-    peak = float(peaks.get("bf16_tflops"))
-    peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+    # the fine pass's own dtype: half its FLOP (S = Q K^T) at the fp8 rate with
+    # qk_fp8, all of it with pv_fp8 too; fp8 runs at twice the dense bf16 rate
+    # (nominal 4.5 against 2.25 PFLOP/s), applied to the measured bf16 peak
+    ratio = 2.0 if w.pv_fp8 else (4.0 / 3.0 if w.qk_fp8 else 1.0)
+    peak = float(peaks.get("bf16_tflops")) * ratio
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))) * ratio
     hbm = float(peaks.get("hbm_gbs"))
     fine_ms = ph_ms["attention_fine_pass"]
     achieved = flops_kept / (fine_ms * 1e-3) / 1e12
@@ -606,7 +614,8 @@ def main():
         "higher_is_better": True,
         "scaling": "strong" if split == "heads" and world > 1 else "weak",
         "vs_baseline": None,
-        "dtype": ("bf16 (Q K^T in e4m3)" if w.qk_fp8 else "bf16") if w.dtype == "bf16" else "f32",
+        "dtype": (("bf16 (Q K^T and P V in e4m3)" if w.pv_fp8 else "bf16 (Q K^T in e4m3)") if w.qk_fp8 else "bf16")
+        if w.dtype == "bf16" else "f32",
         "data": "synthetic (smooth Gaussian-filtered fields + noise, seeded)",
         "config": _config_json(w_job, world, split, [h0, h1]),
         "ms_per_layer": ms_step,
@@ -616,7 +625,8 @@ def main():
         "kept_fraction_of_dense": flops_kept / dense_equiv_flops(w),
         "roofline": {"bound": "tensor", "kernel": "attn_kernel (bsa_attention_run: sparse + centroid + dense rows)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_src} bf16_tflops (burst: the kernel runs inside a sub-second step)",
+                     "peak_source": f"{peak_src} bf16_tflops (burst: the kernel runs inside a sub-second step)"
+                     + ("" if ratio == 1.0 else f" x {ratio:.3f} for the e4m3 products (fp8 = 2 x bf16, nominal)"),
                      "frac_of_sustained": achieved / peak_sus,
                      "issued_tflop": flops_issued / 1e12,
                      "issued_achieved": flops_issued / (fine_ms * 1e-3) / 1e12,

@@ -42,7 +42,7 @@ class bsa_params(ctypes.Structure):
         ("extra_tokens", ctypes.c_int32), ("centroid", ctypes.c_int32),
         ("grid_t", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
         ("cube_t", ctypes.c_int32), ("cube_h", ctypes.c_int32), ("cube_w", ctypes.c_int32),
-        ("qk_fp8", ctypes.c_int32), ("modcent_per_row", ctypes.c_int32),
+        ("qk_fp8", ctypes.c_int32), ("modcent_per_row", ctypes.c_int32), ("pv_fp8", ctypes.c_int32),
     ]
 
 
@@ -145,7 +145,7 @@ def make_params(q: torch.Tensor, method: str = "sol", *, q_block: Optional[int] 
                 tau: float = 1.3, keep_percent: float = 10.0, sink_blocks: int = 1,
                 keep_diag: int = 1, prefix_len: int = 0, dense_rows=(0, 0), extra_tokens: int = 0,
                 centroid: Optional[int] = None, grid=None, cube=(4, 4, 4), qk_fp8: bool = False,
-                modcent_per_row: int = 0) -> bsa_params:
+                modcent_per_row: int = 0, pv_fp8: bool = False) -> bsa_params:
     """Parameters for a [B, N, H, d] query tensor `q` (strides taken from q).
     method "vsa" needs `grid` = (T, Hs, Ws) of the tokens after the prefix."""
     m = {"sol": BSA_SOL, "sla": BSA_SLA, "vsa": BSA_VSA}[method]
@@ -166,6 +166,7 @@ def make_params(q: torch.Tensor, method: str = "sol", *, q_block: Optional[int] 
         p.centroid = centroid
     p.qk_fp8 = int(bool(qk_fp8))
     p.modcent_per_row = int(modcent_per_row)
+    p.pv_fp8 = int(bool(pv_fp8))
     if m == BSA_VSA:
         if grid is None:
             raise ValueError("method vsa needs the latent grid (T, Hs, Ws)")
@@ -182,7 +183,8 @@ def params_for(w, q: torch.Tensor) -> bsa_params:
                        sink_blocks=w.sink_blocks, keep_diag=w.keep_diag, prefix_len=w.prefix_len,
                        dense_rows=tuple(w.dense_rows), extra_tokens=w.extra_tokens, centroid=w.centroid,
                        grid=getattr(w, "grid", None), cube=getattr(w, "cube", (4, 4, 4)),
-                       qk_fp8=getattr(w, "qk_fp8", False), modcent_per_row=getattr(w, "modcent_per_row", 0))
+                       qk_fp8=getattr(w, "qk_fp8", False), modcent_per_row=getattr(w, "modcent_per_row", 0),
+                       pv_fp8=getattr(w, "pv_fp8", False))
 
 
 def dims(p: bsa_params):

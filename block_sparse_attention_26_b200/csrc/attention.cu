@@ -151,6 +151,8 @@ struct AttnArgs {
     // fp8 Q K^T: scales of Q per 64 tokens, of K per key block, of the centroids per 64
     const float *sq8, *sk8, *skc8;
     int nb64, nch64;
+    // fp8 P V: scale of V per (b, h, channel)
+    const float *sv8;
 };
 
 // Token of block-order position p (identity without cube tiling).
@@ -180,13 +182,14 @@ __device__ __forceinline__ void load_rows64(uint8_t *dst, const AttnArgs &a, con
     }
 }
 
-template <int D, bool QK8 = false>
+template <int D, bool QK8 = false, bool PV8 = false>
 struct Lay {
-    // Q and K tiles hold 1 byte per channel with fp8 Q K^T (QK8), else 2
+    // Q and K tiles hold 1 byte per channel with fp8 Q K^T (QK8), else 2; V tiles
+    // 1 byte with fp8 P V (PV8)
     static constexpr int kQKElem = QK8 ? 1 : 2;
     static constexpr int kQBytes = kM * D * kQKElem;
     static constexpr int kKTileBytes = kTK * D * kQKElem;       // one K tile (128 keys)
-    static constexpr int kTileBytes = kTK * D * 2;              // one V tile (128 keys)
+    static constexpr int kTileBytes = kTK * D * (PV8 ? 1 : 2);  // one V tile (128 keys)
     static constexpr int kHalfBytes = kBK * 128;                // one 64-key box of one 128-byte channel chunk
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
@@ -268,6 +271,18 @@ __device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint
         "elect.sync _|e, 0xffffffff;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// The same with e4m3 operands (kind::f8f6f4, K = 32): A (4 values a 32-bit column) from TMEM.
+__device__ __forceinline__ void umma_ts_f8_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
@@ -353,7 +368,7 @@ __device__ __forceinline__ void named_bar(int id, int count)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-template <int D, bool QK8>
+template <int D, bool QK8, bool PV8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
@@ -363,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tm_k5, const __grid_constant__ CUtensorMap tm_v5,
                 const AttnArgs a)
 {
-    using L = Lay<D, QK8>;
+    using L = Lay<D, QK8, PV8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~(uintptr_t)1023);
@@ -613,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // half x of the tile lands at row offset 64 x of every channel chunk
         const CUtensorMap *tm_x5 = is_k ? &tm_k5 : &tm_v5;
         auto load_half = [&](uint8_t *dst, int kind, int blk, uint64_t *bar) {
-            if (QK8 && is_k) {
+            if ((QK8 && is_k) || (PV8 && !is_k)) {
                 // 64 keys of 128 fp8 channels: one box
                 if (kind == TILE_EXACT)
                     tma_load_4d(dst, tm_x, bar, 0, h, blk * kBK, b);
@@ -887,6 +902,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idesc_s = idesc_bf16_f32(kM, kTK, 0, 0);
             const uint32_t idesc_s8 = idesc_e4m3_f32(kM, kTK);
             const uint32_t idesc_o = idesc_bf16_f32(kM, D, 0, 1);
+            const uint32_t idesc_o8 = idesc_e4m3_f32(kM, D) | (1u << 16);   // B (V) MN-major
             const uint32_t q_addr = smem_u32(sm + L::kOffQ);
             const uint32_t k_addr = smem_u32(sm + L::kOffK);
             const uint32_t v_addr = smem_u32(sm + L::kOffV);
@@ -942,12 +958,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) return;
                 tc_fence_after();
                 if (!a.gather_tma && info[vs].h[0].x == TILE_GATHER) fence_async_smem();   // rows by cp.async
+                if (PV8) {
+                    // P as e4m3 (4 a column), V as e4m3 rows of 128 channels: K = 32 a step
 #pragma unroll
-                for (int ks = 0; ks < kBK / 16; ++ks) {
-                    const uint64_t bd =
-                        sdesc_sw128(v_addr + vs * L::kTileBytes + hf * L::kHalfBytes + ks * 2048, kTK * 128, 1024);
-                    umma_ts_w(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd, idesc_o,
-                                 (t > 0 || ks > 0) ? 1u : 0u);
+                    for (int ks = 0; ks < kBK / 32; ++ks) {
+                        const uint64_t bd =
+                            sdesc_sw128(v_addr + vs * L::kTileBytes + hf * L::kHalfBytes + ks * 4096, 16, 1024);
+                        umma_ts_f8_w(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd,
+                                     idesc_o8, (t > 0 || ks > 0) ? 1u : 0u);
+                    }
+                } else {
+#pragma unroll
+                    for (int ks = 0; ks < kBK / 16; ++ks) {
+                        const uint64_t bd =
+                            sdesc_sw128(v_addr + vs * L::kTileBytes + hf * L::kHalfBytes + ks * 2048, kTK * 128, 1024);
+                        umma_ts_w(tmem + kColO + 128 * hf, tmem + kColS + 128 * pb + 64 * hf + 8 * ks, bd, idesc_o,
+                                  (t > 0 || ks > 0) ? 1u : 0u);
+                    }
                 }
                 if (hf == 1) umma_commit_w(&v_empty[vs]);   // both halves have used the V slot
                 if (hf == 0 && lane == 0) TRACE(3, t);
@@ -1078,7 +1105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
                         const float p0 = ex2(x.x), p1 = ex2(x.y);
                         acc[c & 1] = fadd2(acc[c & 1], make_float2(p0, p1));
-                        pk[c] = pack_bf16x2(p0, p1);
+                        pk[c] = PV8 ? (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3)
+                                    : pack_bf16x2(p0, p1);
                     }
                 } else {
 #pragma unroll
@@ -1086,14 +1114,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float2 x = fadd2(make_float2(s[2 * c], s[2 * c + 1]), nm2);
                         const float p0 = ex2(x.x), p1 = ex2(x.y);
                         acc[c & 1] = fadd2(acc[c & 1], make_float2(p0, p1));
-                        pk[c] = pack_bf16x2(p0, p1);
+                        pk[c] = PV8 ? (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3)
+                                    : pack_bf16x2(p0, p1);
                     }
                 }
                 l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
             }
             if (r == 0) TRACE(10 + 3 * hf, j);
             if (r == 0) TRACE(11 + 3 * hf, j);
-            tmem_st32(tmem + lane_base + col_s, pk);   // over this half's S, already read
+            if constexpr (PV8) {
+                // e4m3 P: four a column (the row sum l keeps the unrounded values)
+                uint32_t pk8[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk8[i] = (pk[2 * i] & 0xffffu) | (pk[2 * i + 1] << 16);
+                tmem_st16(tmem + lane_base + col_s, pk8);
+            } else {
+                tmem_st32(tmem + lane_base + col_s, pk);   // over this half's S, already read
+            }
             if (__any_sync(0xffffffffu, rescale)) {
                 // the accumulator must hold every earlier P V product before it is scaled
                 // (S(j + 1), or the end marker, is issued after P V(j - 1))
@@ -1153,6 +1190,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float xa = cA > 0.f ? cA * __uint_as_float(oa[e]) : 0.f;
                     const float xb = cB > 0.f ? cB * __uint_as_float(ob[e]) : 0.f;
                     v[e] = xa + xb;
+                }
+                if constexpr (PV8) {
+                    // V was stored divided by its channel's scale
+                    const float4 *sv4 = reinterpret_cast<const float4 *>(a.sv8 + (int64_t)bh * D + cc * 32);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float4 s4 = __ldg(sv4 + e);
+                        v[4 * e] *= s4.x;
+                        v[4 * e + 1] *= s4.y;
+                        v[4 * e + 2] *= s4.z;
+                        v[4 * e + 3] *= s4.w;
+                    }
                 }
                 if (split) {
                     // unnormalised partial in the frame of m, merged by combine_kernel
@@ -1753,6 +1802,101 @@ __global__ void __launch_bounds__(256) quant_cent_kernel(const float *__restrict
     o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
+// ------------------------------------------------------------------ fp8 P V
+
+// Largest |v| per (b, h, channel) of V, as the bits of a non-negative float
+// (atomicMax on them orders like the floats; bits zeroed beforehand).  One CTA
+// per (b * H + h, 256 tokens); thread t: channel t % 128, tokens of half t / 128.
+__global__ void __launch_bounds__(256) vmax_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
+                                                   int64_t sh, int N, int H, uint32_t *__restrict__ maxbits)
+{
+    __shared__ float part[256];
+    const int64_t bh = blockIdx.y;
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    const int c = threadIdx.x & 127, half = threadIdx.x >> 7;
+    const int n0 = blockIdx.x * 256 + half * 128, n1 = min(N, n0 + 128);
+    const __nv_bfloat16 *base = v + (int64_t)b * sb + (int64_t)h * sh + c;
+    float m = 0.f;
+    for (int n = n0; n < n1; ++n) m = fmaxf(m, fabsf(__bfloat162float(base[(int64_t)n * sn])));
+    part[threadIdx.x] = m;
+    __syncthreads();
+    if (half == 0) atomicMax(&maxbits[bh * 128 + c], __float_as_uint(fmaxf(m, part[threadIdx.x + 128])));
+}
+
+// In place: the largest |v| of each channel -> its scale (largest / 448; 1 for
+// an all-zero channel).
+__global__ void sv_scale_kernel(uint32_t *__restrict__ sv, int64_t n)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float m = __uint_as_float(sv[i]);
+        sv[i] = __float_as_uint(m > 0.f ? m / 448.f : 1.f);
+    }
+}
+
+// e4m3 copy of V ([B, N, H, 128] bf16 in, contiguous [B, N, H, 128] e4m3 out),
+// x8 = round-to-nearest(x / scale of its channel), saturating.  One CTA per
+// (b * H + h, 64 tokens); thread t: row t / 4, channels 32 (t % 4) ...
+__global__ void __launch_bounds__(256) quant_v_kernel(const __nv_bfloat16 *__restrict__ src, int64_t sb, int64_t sn,
+                                                      int64_t sh, int N, int H, const float *__restrict__ sv,
+                                                      uint8_t *__restrict__ dst)
+{
+    const int64_t bh = blockIdx.y;
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    const int row = threadIdx.x >> 2, c0 = 32 * (threadIdx.x & 3);
+    const int n = blockIdx.x * 64 + row;
+    if (n >= N) return;
+    const uint4 *p = reinterpret_cast<const uint4 *>(src + (int64_t)b * sb + (int64_t)n * sn + (int64_t)h * sh + c0);
+    const float *s = sv + bh * 128 + c0;
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 w = p[i];
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[2 * e] = __uint_as_float(ww[e] << 16) / s[8 * i + 2 * e];
+            x[2 * e + 1] = __uint_as_float(ww[e] & 0xffff0000u) / s[8 * i + 2 * e + 1];
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const __nv_fp8x2_storage_t lo =
+                __nv_cvt_float2_to_fp8x2(make_float2(x[4 * e], x[4 * e + 1]), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t hi =
+                __nv_cvt_float2_to_fp8x2(make_float2(x[4 * e + 2], x[4 * e + 3]), __NV_SATFINITE, __NV_E4M3);
+            pk[2 * i + e] = (uint32_t)lo | ((uint32_t)hi << 16);
+        }
+    }
+    uint4 *o = reinterpret_cast<uint4 *>(dst + (((int64_t)b * N + n) * H + h) * 128 + c0);
+    o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
+// e4m3 value centroids [BH, nKB, 128] from the f32 means, with the channel scales of V.
+__global__ void __launch_bounds__(256) quant_vcent_kernel(const float *__restrict__ vbar, int nKB,
+                                                          const float *__restrict__ sv, uint8_t *__restrict__ dst)
+{
+    const int64_t bh = blockIdx.y;
+    const int row = threadIdx.x >> 2, c0 = 32 * (threadIdx.x & 3);
+    const int j = blockIdx.x * 64 + row;
+    if (j >= nKB) return;
+    const float4 *p = reinterpret_cast<const float4 *>(vbar + ((int64_t)bh * nKB + j) * 128 + c0);
+    const float *s = sv + bh * 128 + c0;
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 v = p[i];
+        const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+            make_float2(v.x / s[4 * i], v.y / s[4 * i + 1]), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+            make_float2(v.z / s[4 * i + 2], v.w / s[4 * i + 3]), __NV_SATFINITE, __NV_E4M3);
+        pk[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    uint4 *o = reinterpret_cast<uint4 *>(dst + ((int64_t)bh * nKB + j) * 128 + c0);
+    o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
 // ------------------------------------------------------------------ tensor maps
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -1864,18 +2008,18 @@ bool make_map_cube(CUtensorMap *m, const void *base, int P, int H, int d, int gT
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool QK8>
+template <int D, bool QK8, bool PV8>
 cudaError_t launch_attn_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                const CUtensorMap &tkc, const CUtensorMap &tvc, const CUtensorMap (&tg)[4],
                                const CUtensorMap (&t5)[3], const AttnArgs &a, int64_t items, cudaStream_t st)
 {
-    const size_t smem = Lay<D, QK8>::bytes(a.nW);
+    const size_t smem = Lay<D, QK8, PV8>::bytes(a.nW);
     cudaError_t e =
-        cudaFuncSetAttribute(attn_kernel<D, QK8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(attn_kernel<D, QK8, PV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    attn_kernel<D, QK8><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, tg[0], tg[1], tg[2], tg[3],
-                                                                 t5[0], t5[1], t5[2], a);
+    attn_kernel<D, QK8, PV8><<<(unsigned)items, kThreads, smem, st>>>(tq, tk, tv, tkc, tvc, tg[0], tg[1], tg[2],
+                                                                      tg[3], t5[0], t5[1], t5[2], a);
     return cudaGetLastError();
 }
 
@@ -1976,11 +2120,33 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
         if (use_cent)
             quant_cent_kernel<<<dim3((unsigned)nch64, (unsigned)BH), 256, 0, st>>>(kbar, D.nKB, nch64, kc8, skc8);
     }
+    const bool v8 = f8 && p.pv_fp8 != 0;
+    uint8_t *v8p = reinterpret_cast<uint8_t *>(ws + L.v8), *vc8 = reinterpret_cast<uint8_t *>(ws + L.vc8);
+    float *sv8 = reinterpret_cast<float *>(ws + L.sv8);
+    if (v8 && prep) {
+        // V and the value centroids with one scale per (b, h, channel)
+        cudaError_t e = cudaMemsetAsync(sv8, 0, (size_t)BH * D.d * 4, st);
+        if (e != cudaSuccess) return e;
+        count_launch();
+        vmax_kernel<<<dim3((unsigned)ceil_div(D.N, 256), (unsigned)BH), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(v16), sb, sn, sh, D.N, D.H, reinterpret_cast<uint32_t *>(sv8));
+        count_launch();
+        sv_scale_kernel<<<(unsigned)ceil_div(BH * D.d, 256), 256, 0, st>>>(reinterpret_cast<uint32_t *>(sv8),
+                                                                             BH * D.d);
+        count_launch();
+        quant_v_kernel<<<dim3((unsigned)nb64, (unsigned)BH), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(v16), sb, sn, sh, D.N, D.H, sv8, v8p);
+        if (use_cent) count_launch();
+        if (use_cent)
+            quant_vcent_kernel<<<dim3((unsigned)nch64, (unsigned)BH), 256, 0, st>>>(vbar, D.nKB, sv8, vc8);
+    }
     CUtensorMap tq, tk, tv, tkc, tvc;
     if (f8) {
+        const bool vm = v8 ? make_map_u8_bnhd(&tv, v8p, D.B, D.N, D.H, D.d, kBK) && make_map_u8_cent(&tvc, vc8, BH, D.nKB, D.d)
+                           : make_map_bnhd(&tv, v16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) &&
+                                 make_map_cent(&tvc, vc, BH, D.nKB, D.d);
         if (!make_map_u8_bnhd(&tq, q8, D.B, D.N, D.H, D.d, kM) || !make_map_u8_bnhd(&tk, k8, D.B, D.N, D.H, D.d, kBK) ||
-            !make_map_bnhd(&tv, v16, D.B, D.N, D.H, D.d, sb, sn, sh, kBK) ||
-            !make_map_u8_cent(&tkc, kc8, BH, D.nKB, D.d) || !make_map_cent(&tvc, vc, BH, D.nKB, D.d)) {
+            !vm || !make_map_u8_cent(&tkc, kc8, BH, D.nKB, D.d)) {
             set_error("cuTensorMapEncodeTiled failed for the fp8 tiles");
             return cudaErrorInvalidValue;
         }
@@ -2010,6 +2176,7 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
     a.skc8 = skc8;
     a.nb64 = nb64;
     a.nch64 = nch64;
+    a.sv8 = sv8;
     a.cube = D.cube;
     a.pre_blocks = D.pre_blocks;
     a.P = p.prefix_len;
@@ -2160,9 +2327,10 @@ cudaError_t launch_attention(const bsa_params &p, const Dims &D, const void *q, 
             }
         }
     }
-    cudaError_t e = D.d == 64 ? launch_attn_kernel<64, false>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
-                    : p.qk_fp8  ? launch_attn_kernel<128, true>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
-                                : launch_attn_kernel<128, false>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st);
+    cudaError_t e = D.d == 64   ? launch_attn_kernel<64, false, false>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
+                    : v8        ? launch_attn_kernel<128, true, true>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
+                    : p.qk_fp8  ? launch_attn_kernel<128, true, false>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st)
+                                : launch_attn_kernel<128, false, false>(tq, tk, tv, tkc, tvc, tg, t5, a, items, st);
     if (e != cudaSuccess) return e;
     if (a.n_dense > 0 && a.dense_split > 1) {
         count_launch();

@@ -119,6 +119,11 @@ WsLayout ws_layout(const bsa_params &p)
     L.sk8 = take(f8 ? (size_t)BH * D.nKB * 4 : 0);
     L.kc8 = take(f8 ? (size_t)BH * D.nKB * D.d : 0);
     L.skc8 = take(f8 ? (size_t)BH * ceil_div(D.nKB, 64) * 4 : 0);
+    // fp8 P V (pv_fp8): e4m3 V and value centroids, one scale per (b, h, channel)
+    const bool v8 = p.pv_fp8 != 0;
+    L.v8 = take(v8 ? ntok : 0);
+    L.vc8 = take(v8 ? (size_t)BH * D.nKB * D.d : 0);
+    L.sv8 = take(v8 ? (size_t)BH * D.d * 4 : 0);
     L.part_tiles = dense_partial_tiles(D, p.dense_row_end - p.dense_row_begin);
     L.part_o = take((size_t)L.part_tiles * 128 * D.d * sizeof(float));
     L.part_ml = take((size_t)L.part_tiles * 128 * 2 * sizeof(float));
@@ -160,6 +165,8 @@ bsa_status check_params(const bsa_params *p)
     if (p->method != BSA_SOL && !(p->keep_percent > 0.0 && p->keep_percent <= 100.0))
         FAIL(BSA_ERR_INVALID_ARG, "keep_percent must be in (0, 100]");
     if (p->qk_fp8 != 0 && p->qk_fp8 != 1) FAIL(BSA_ERR_INVALID_ARG, "qk_fp8 must be 0 or 1");
+    if (p->pv_fp8 != 0 && p->pv_fp8 != 1) FAIL(BSA_ERR_INVALID_ARG, "pv_fp8 must be 0 or 1");
+    if (p->pv_fp8 && !p->qk_fp8) FAIL(BSA_ERR_UNSUPPORTED, "pv_fp8 needs qk_fp8 (the all-fp8 mode)");
     if (p->qk_fp8) {
         if (p->dtype != BSA_DT_BF16 || p->d != 128 || p->extra_tokens != 0 || p->method == BSA_VSA)
             FAIL(BSA_ERR_UNSUPPORTED, "qk_fp8 needs bf16 inputs, d = 128, extra_tokens 0 and method Sol or SLA");

@@ -99,6 +99,8 @@ struct WsLayout {
     size_t sk8;            // [B*H, nKB] f32 scales of K per key block
     size_t kc8;            // [B*H, nKB, d] e4m3 centroids
     size_t skc8;           // [B*H, ceil(nKB / 64)] f32 scales of the centroids per 64
+    size_t v8, vc8;        // [B, N, H, d] e4m3 V, [B*H, nKB, d] e4m3 value centroids (pv_fp8)
+    size_t sv8;            // [B*H, d] f32 scale of V per channel (its largest |v| / 448)
     size_t part_o;         // [part_tiles, 128, d] f32 dense-row partial outputs
     size_t part_ml;        // [part_tiles, 128, 2] f32 dense-row partial (max, sum)
     int64_t part_tiles;    // capacity of the partial buffers, in 128-row tiles

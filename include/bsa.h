@@ -119,6 +119,10 @@ typedef struct {
                                       exceeds the capacity, the status word reports BSA_ERR_CAPACITY
                                       and the rows past it lose the modified centroids that did not
                                       fit (their other terms are unchanged). */
+    int32_t pv_fp8;                /* 1 (with qk_fp8 = 1): P V in fp8 too -- P rounded to e4m3 as the
+                                      softmax writes it, V and the value centroids in e4m3 with one
+                                      scale per (batch, head, channel) applied to the output -- the
+                                      B200 form of [STAR] "attention modes" all_int8 / Sol "PV INT8" */
 } bsa_params;
 
 /* Fill *p with the defaults of the node documentation for `method`

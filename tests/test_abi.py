@@ -40,6 +40,7 @@ def test_params_struct_layout():
     assert bsa.bsa_params.cube_w.offset == 120
     assert bsa.bsa_params.qk_fp8.offset == 124
     assert bsa.bsa_params.modcent_per_row.offset == 128
+    assert bsa.bsa_params.pv_fp8.offset == 132
 
 
 def _p(**kw):
@@ -76,6 +77,8 @@ FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced (validati
     ("sink_blocks", -1, binding.BSA_ERR_INVALID_ARG),
     ("centroid", 2, binding.BSA_ERR_INVALID_ARG),
     ("modcent_per_row", -1, binding.BSA_ERR_INVALID_ARG),
+    ("pv_fp8", 2, binding.BSA_ERR_INVALID_ARG),
+    ("pv_fp8", 1, binding.BSA_ERR_UNSUPPORTED),             # needs qk_fp8
 ])
 def test_bad_params_rejected(field, value, code):
     p = _p(**{field: value})

@@ -32,6 +32,9 @@ CASES = {
     "fp8_sla": Workload("fp8_sla", B=1, H=2, N=2880, d=128, dtype="bf16", method="sla", q_block=128, k_block=64,
                         keep_percent=15.0, centroid=0, grid=(4, 24, 30), seed=103, qk_fp8=True),
 }
+# all-fp8 (pv_fp8 too: P rounded to e4m3, V with one scale per (head, channel))
+CASES.update({k.replace("fp8_", "fp8pv_"): w.replace(name=w.name.replace("fp8_", "fp8pv_"), pv_fp8=True)
+              for k, w in list(CASES.items())})
 
 
 def _check(w, q, k, v, toks=None):
@@ -60,8 +63,9 @@ def test_fp8_matches_oracle_within_relaxed_tolerance(name):
     _check(w, q, k, v)
 
 
-def test_fp8_full_size_sampled():
-    w = CONFIGS["sol_mid"].replace(qk_fp8=True)
+@pytest.mark.parametrize("pv", [False, True], ids=["qk", "qk_pv"])
+def test_fp8_full_size_sampled(pv):
+    w = CONFIGS["sol_mid"].replace(qk_fp8=True, pv_fp8=pv)
     q, k, v = make_qkv(w, "cuda")
     g = np.random.default_rng(5)
     toks = []

@@ -52,6 +52,7 @@ class Workload:
     cube: Tuple[int, int, int] = (4, 4, 4)         # vsa: cube extents (t, y, x)
     qk_fp8: bool = False                           # fine pass with S = Q K^T in fp8 (e4m3)
     modcent_per_row: int = 0                       # modified-centroid capacity per query block (0: worst case)
+    pv_fp8: bool = False                           # with qk_fp8: P V in fp8 (e4m3) as well
     seed: int = 0
     field_sigma: float = 4.0
     noise: float = 0.5
