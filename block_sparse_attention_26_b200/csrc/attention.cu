@@ -42,9 +42,13 @@
 //              lane issues): S = Q K^T (A and B from
 //              shared memory) runs one tile ahead of the softmax, into two TMEM
 //              buffers; per tile j it issues O_h += P_h V_h (A = P_h from TMEM)
-//              for h = 0, 1 as each half's P comes in, then S(j + 2) into the
-//              buffer P(j) held: the tensor pipe runs one thread's MMAs in issue
-//              order.  The completion of S(j) also frees K slot j % 2, and the
+//              for h = 0, 1, then S(j + 2) into the buffer P(j) held: the tensor
+//              pipe runs one thread's MMAs in issue order.  All of that waits on one
+//              barrier, ready(j): both halves' P(j) written and K(j + 2) landed (or
+//              the list's end reached).  The tensor pipe takes only a couple of
+//              MMAs ahead of its issuer, so every wait between MMA groups leaves it
+//              idle for about a barrier round trip: one wait per tile, not three.
+//              The completion of S(j) also frees K slot j % 2, and the
 //              completion of S(j + 1) tells a softmax warp that wants to rescale
 //              O at tile j that P V(j - 1) is done.
 // TMEM (512 columns): S of tile j at 128 (j & 1), half h's P (bf16 pairs) written
@@ -197,8 +201,8 @@ struct Lay {
     static constexpr int kOffKind = kOffV + kVS * kTileBytes;
     static constexpr int kOffInfo = kOffKind + 16;
     static constexpr int kOffBar = kOffInfo + kVS * (int)sizeof(TileInfo);
-    // q, done, k_full[KS], v_full[VS], v_empty[VS], s_full[2 buffers], p_full[2 halves][2]
-    static constexpr int kNumBar = 2 + kKS + 2 * kVS + 2 + 4;
+    // q, done, k_full[KS], v_full[VS], v_empty[VS], s_full[2 buffers], ready[2 buffers]
+    static constexpr int kNumBar = 2 + kKS + 2 * kVS + 2 + 2;
     static constexpr int kOffMisc = kOffBar + kNumBar * 8;
     static constexpr int kOffML = kOffMisc + 16;                 // [2][128] (m, l) per half
     static constexpr int kOffBias = kOffML + 2 * kM * 8;         // [VS][128] per-column bias (gathers)
@@ -419,7 +423,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *k_full = bars + 2;
     uint64_t *v_full = k_full + kKS, *v_empty = v_full + kVS;
     uint64_t *s_full = v_empty + kVS;         // [buffer]
-    uint64_t *p_full = s_full + 2;            // [half * 2 + buffer]
+    // [buffer] tile j's phase of ready[j & 1]: P(j) from all 8 softmax warps, and the
+    // K producer's tile j + 2 (its TMA bytes, or an arrival past the list's end);
+    // tiles 0 and 1 land on k_full
+    uint64_t *ready = s_full + 2;
     volatile int32_t *kkind = reinterpret_cast<volatile int32_t *>(sm + L::kOffKind);
     volatile TileInfo *info = reinterpret_cast<volatile TileInfo *>(sm + L::kOffInfo);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kOffMisc);
@@ -449,7 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        for (int i = 0; i < 4; ++i) mbar_init(&p_full[i], 4);
+        mbar_init(&ready[0], 9);
+        mbar_init(&ready[1], 9);
         *abort_flag = 0;
         fence_mbar_init();
         // Q first: its load overlaps the rest of the set-up
@@ -686,6 +694,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             uint8_t *dst = ring + s * (is_k ? L::kKTileBytes : L::kTileBytes);
+            // K tile j >= 2 completes tile j - 2's ready barrier (the slot wait above
+            // ordered it after that barrier's previous phase: S(j - 2) was issued after it)
+            uint64_t *fb = (is_k && j >= 2) ? &ready[j & 1] : &full[s];
             if (kind == TILE_GATHER && !is_k)
                 for (int c = lane; c < kTK; c += 32) {
                     // bias 0 for extra tokens, log2 of the remaining count for modified centroids
@@ -698,7 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // 128 rows by TMA, 4 rows per gather: lane l takes columns 4l..4l+3
                 // (unused columns repeat the last entry; the 4 rows of a gather come
                 // from one array because the column list is 4-aligned per array)
-                if (lane == 0) mbar_expect_tx(&full[s], L::kTileBytes);
+                if (lane == 0) mbar_expect_tx(fb, L::kTileBytes);
                 __syncwarp();
                 const int c = 4 * lane;
                 int rw[4];
@@ -712,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
 #pragma unroll
                 for (int dc = 0; dc < D / 64; ++dc)
-                    tma_gather4(dst + dc * (kTK * 128) + c * 128, cent ? tm_gc : tm_gx, &full[s], dc * 64, rw);
+                    tma_gather4(dst + dc * (kTK * 128) + c * 128, cent ? tm_gc : tm_gx, fb, dc * 64, rw);
             } else if (kind == TILE_GATHER) {
                 // 128 rows from arbitrary addresses, written in the 128-byte-swizzled
                 // layout the tensor core reads; completion through the barrier.  Unused
@@ -741,16 +752,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // each lane's copies complete the slot asynchronously (one pending
                 // arrival per lane, added now); lane 0 gives the barrier's own arrival.
                 // The MMA warp orders them before its tensor-core reads with a proxy fence.
-                asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(&full[s])) : "memory");
+                asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(fb)) : "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full[s]);
+                if (lane == 0) mbar_arrive(fb);
             } else if (lane == 0) {
                 if (kind == TILE_END) {
-                    mbar_arrive(&full[s]);
+                    mbar_arrive(fb);
                 } else {
-                    mbar_expect_tx(&full[s], is_k ? L::kKTileBytes : L::kTileBytes);
-                    load_half(dst, kind, blk[0], &full[s]);
-                    load_half(dst + L::kHalfBytes, kind, blk[1], &full[s]);
+                    mbar_expect_tx(fb, is_k ? L::kKTileBytes : L::kTileBytes);
+                    load_half(dst, kind, blk[0], fb);
+                    load_half(dst + L::kHalfBytes, kind, blk[1], fb);
                 }
             }
             ++j;
@@ -882,17 +893,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int bl[2] = {0, 0};
             const uint32_t wh[2] = {0u, 0u};
             const int nc[2] = {0, 0};
+            // the K side marks the end twice: at T (tile T - 2's ready, where the MMA
+            // warp reads it) and at T + 1 (tile T - 1's ready, which has no K tile)
             ok = push(TILE_END, bl, wh, nc, none, 0.f, zero2);
+            if (ok && is_k) ok = push(TILE_END, bl, wh, nc, none, 0.f, zero2);
         }
         if (lane == 0) {
             // no TMA write may still be in flight when the CTA exits: wait for the
-            // last phase every slot was armed with
+            // last phase every barrier was armed with (phases complete in order; the
+            // ready phases also take the softmax warps' arrivals, which every tile
+            // before the end gets)
             volatile int32_t no_abort = 0;
-            for (int s = 0; s < depth; ++s) {
-                const int n = (j - s + depth - 1) / depth;
-                if (n > 0) mbar_wait(&full[s], (n - 1) & 1, &no_abort, a.status, 12);
+            if (is_k) {
+                for (int t = 0; t < 2 && t < j; ++t) mbar_wait(&k_full[t], 0, &no_abort, a.status, 12);
+                for (int t = max(2, j - 2); t < j; ++t)
+                    mbar_wait(&ready[t & 1], ((t - 2) >> 1) & 1, &no_abort, a.status, 15);
+                mbar_wait(bar_q, 0, &no_abort, a.status, 14);
+            } else {
+                for (int s = 0; s < depth; ++s) {
+                    const int n = (j - s + depth - 1) / depth;
+                    if (n > 0) mbar_wait(&full[s], (n - 1) & 1, &no_abort, a.status, 12);
+                }
             }
-            if (is_k) mbar_wait(bar_q, 0, &no_abort, a.status, 14);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");   // this lane's gathered rows have landed
     } else if (warp == 9) {
@@ -908,27 +930,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t v_addr = smem_u32(sm + L::kOffV);
             bool ok = __all_sync(0xffffffffu, mbar_wait(bar_q, 0, abort_flag, a.status, 22));
             tc_fence_after();
-            // Fixed order: S(0), S(1), then for each tile j the P V products of
-            // both halves and S(j + 2), which goes to the buffer P(j) held (the tensor
-            // pipe runs one thread's MMAs in issue order).  Every wait is a blocking
-            // try_wait: polling barriers from this thread between MMAs stalls the
-            // tensor pipe (each test costs tens of cycles while MMAs read shared
-            // memory).
+            // rows copied by cp.async (gathers without TMA) need a proxy fence before
+            // the tensor core reads them
+            const bool cp_gather = a.E > 0 && !a.gather_tma;
+            // Fixed order: S(0), S(1), then for each tile j the P V products of both
+            // halves and S(j + 2), which goes to the buffer P(j) held (the tensor pipe
+            // runs one thread's MMAs in issue order), all behind the one wait on
+            // ready(j).  Every wait is a blocking try_wait: polling barriers from this
+            // thread between MMAs stalls the tensor pipe.
             int T = -1;   // tile count, once the end marker is seen
-            auto issue_s = [&](int ns) -> bool {
+            // S(ns) for a K tile that has landed (kind read after its barrier)
+            auto issue_s = [&](int ns, int kind) {
                 const int ks = ns % kKS;
-                ok = __all_sync(0xffffffffu, mbar_wait(&k_full[ks], (ns / kKS) & 1, abort_flag, a.status, 27));
-                if (!ok) return false;
-                tc_fence_after();
-                const int kind = __shfl_sync(0xffffffffu, (int)kkind[ks], 0);
                 if (kind == TILE_END) {
                     // end-of-list marker for the softmax warps, committed at once: it
                     // completes after every MMA issued so far (P V of tiles < T - 1)
                     umma_commit_w(&s_full[ns & 1]);
                     T = ns;
-                    return false;
+                    return;
                 }
-                if (!a.gather_tma && kind == TILE_GATHER) fence_async_smem();   // rows by cp.async
+                if (cp_gather && kind == TILE_GATHER) fence_async_smem();
                 if (QK8) {
                     // 128 fp8 channels per 128-byte row, 32 per instruction
 #pragma unroll
@@ -948,16 +969,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 umma_commit_w(&s_full[ns & 1]);
                 if (lane == 0) TRACE(2, ns);
-                return true;
             };
-            // P_h(t) is in only after the softmax warps waited for V(t) (they read the
-            // tile's metadata there), so the V rows are in too
+            // O_hf += P_hf(t) V_hf(t); P_h(t) is in only after the softmax warps waited
+            // for V(t) (they read the tile's metadata there), so the V rows are in too
             auto issue_pv = [&](int t, int hf) {
                 const int pb = t & 1, vs = t % kVS;
-                ok = __all_sync(0xffffffffu, mbar_wait(&p_full[2 * hf + pb], (t >> 1) & 1, abort_flag, a.status, 28));
-                if (!ok) return;
-                tc_fence_after();
-                if (!a.gather_tma && info[vs].h[0].x == TILE_GATHER) fence_async_smem();   // rows by cp.async
                 if (PV8) {
                     // P as e4m3 (4 a column), V as e4m3 rows of 128 channels: K = 32 a step
 #pragma unroll
@@ -976,14 +992,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   (t > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
-                if (hf == 1) umma_commit_w(&v_empty[vs]);   // both halves have used the V slot
-                if (hf == 0 && lane == 0) TRACE(3, t);
             };
-            if (ok && issue_s(0)) issue_s(1);
+            for (int ns = 0; ns < 2 && ok && T < 0; ++ns) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&k_full[ns], 0, abort_flag, a.status, 27));
+                if (!ok) break;
+                tc_fence_after();
+                issue_s(ns, kkind[ns]);
+            }
             for (int j = 0; ok && (T < 0 || j < T); ++j) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&ready[j & 1], (j >> 1) & 1, abort_flag, a.status, 28));
+                if (!ok) break;
+                tc_fence_after();
+                // the next K tile's kind, loaded before the P V issue and used after it
+                const int kind2 = T < 0 ? kkind[(j + 2) % kKS] : TILE_END;
+                const int vs = j % kVS;
+                if (cp_gather && info[vs].h[0].x == TILE_GATHER) fence_async_smem();   // rows by cp.async
                 issue_pv(j, 0);
-                if (ok) issue_pv(j, 1);
-                if (ok && T < 0) issue_s(j + 2);
+                if (lane == 0) TRACE(3, j);
+                issue_pv(j, 1);
+                umma_commit_w(&v_empty[vs]);   // both halves have used the V slot
+                if (T < 0) issue_s(j + 2, kind2);
             }
             umma_commit_w(bar_done);
             volatile int32_t no_abort = 0;
@@ -1001,7 +1029,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float scale_q =
             QK8 ? a.scale_log2 * a.sq8[(int64_t)bh * a.nb64 + min(row0 + r, a.N - 1) / 64] : a.scale_log2;
         const uint32_t col_o = kColO + 128 * hf;
-        uint64_t *pf = p_full + 2 * hf;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         int j = 0;
@@ -1151,7 +1178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (r == 0) TRACE(12 + 3 * hf, j);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&pf[j & 1]);
+            if (lane == 0) mbar_arrive(&ready[j & 1]);
             if (r == 0) TRACE(6 + 3 * hf, j);
         }
         const int T = j;
