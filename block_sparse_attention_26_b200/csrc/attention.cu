@@ -230,6 +230,27 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// Non-blocking test of two barrier phases and a 16-byte shared-memory load in
+// one sequence; true if both phases are complete, and only then is the value
+// meaningful (the load is ordered after the tests' acquire).  The three accesses
+// overlap instead of taking a round trip each.
+__device__ __forceinline__ bool test2_load16(uint64_t *b0, uint32_t p0, uint64_t *b1, uint32_t p1, const void *src,
+                                             int4 &v)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred a, b;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 a, [%5], %6;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 b, [%7], %8;\n\t"
+        "ld.volatile.shared.v4.s32 {%0, %1, %2, %3}, [%9];\n\t"
+        "and.pred a, a, b;\n\t"
+        "selp.u32 %4, 1, 0, a;\n\t}"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w), "=r"(ok)
+        : "r"(smem_u32(b0)), "r"(p0), "r"(smem_u32(b1)), "r"(p1), "r"(smem_u32(src))
+        : "memory");
+    return ok != 0;
+}
+
 // UMMA issue in warp-wide form: every lane of the warp executes these with the
 // same operands and one elected lane issues (the operands stay warp-uniform).
 // D[tmem] (+)= A[smem] * B[smem]^T.
@@ -1034,13 +1055,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         int j = 0;
         for (;; ++j) {
             const int vs = j % kVS;
-            ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, a.status, 30) &&
-                 mbar_wait(&v_full[vs], (j / kVS) & 1, abort_flag, a.status, 31);
-            if (!(ok = __all_sync(0xffffffffu, ok))) break;
-            tc_fence_after();
-            // (plain loads: the barrier waits above order them)
             const TileInfo *ti = const_cast<const TileInfo *>(info) + vs;
-            const int4 hq = ti->h[hf];
+            // S(j) and V(j) are usually in by now: test both and load this half's
+            // metadata in one go (one shared-memory round trip); else wait and reload
+            int4 hq;
+            if (!__all_sync(0xffffffffu, test2_load16(&s_full[j & 1], (j >> 1) & 1, &v_full[vs], (j / kVS) & 1,
+                                                      &ti->h[hf], hq))) {
+                ok = mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, a.status, 30) &&
+                     mbar_wait(&v_full[vs], (j / kVS) & 1, abort_flag, a.status, 31);
+                if (!(ok = __all_sync(0xffffffffu, ok))) break;
+                hq = ti->h[hf];   // (a plain load: the waits above order it)
+            }
+            tc_fence_after();
             const int kind = hq.x;
             if (kind == TILE_END) break;
             const float scale = QK8 ? scale_q * ti->ksc[hf] : scale_q;
