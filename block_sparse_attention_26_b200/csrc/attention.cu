@@ -72,6 +72,7 @@ constexpr int kKS = 2;         // K ring depth (tiles)
 constexpr int kVS = 3;         // V ring depth (tiles)
 constexpr int kThreads = 352;  // 2 softmax warpgroups + K producer + MMA + V producer
 constexpr float kRescaleLog2 = 8.0f;
+constexpr float kOptSum = 16777216.0f;   // 2^24: bound on a bf16 tile's sum of P without its maximum
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;          // S of tile j at kColS + 128 (j & 1); P of half h over its own S
 constexpr uint32_t kColO = 256;        // O of half h at kColO + 128 h
@@ -1137,41 +1138,57 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 32; ++c) pk[c] = 0u;
             } else {
-                const float mt = mode == 1 ? max64(s) * scale : max64(s);
-                if (mt > m_ref) {
-                    if (m_ref == -INFINITY) {
-                        m_ref = mt;
-                    } else if (mt > m_ref + kRescaleLog2) {
-                        alpha = ex2(m_ref - mt);
-                        l *= alpha;
-                        m_ref = mt;
-                        rescale = true;
+                // P = 2^(x - m_ref) with a lazily raised reference m_ref.  With bf16 P
+                // the tile's maximum is skipped once m_ref is set: every p is at most
+                // the tile's sum, so a sum within kOptSum proves the tile fits (bf16 P
+                // and the f32 sums keep the same relative precision at any scale, which
+                // cancels in O / l).  A larger sum -- the row's maximum rose by more
+                // than about log2(kOptSum / 64) -- takes the maximum and the rescale,
+                // as does every tile with e4m3 P (at most 448).
+                bool exact = PV8 || m_ref == -INFINITY;
+                float lt;
+                for (;;) {
+                    if (exact) {
+                        const float mt = mode == 1 ? max64(s) * scale : max64(s);
+                        if (mt > m_ref) {
+                            if (m_ref == -INFINITY) {
+                                m_ref = mt;
+                            } else if (mt > m_ref + kRescaleLog2) {
+                                alpha = ex2(m_ref - mt);
+                                l *= alpha;
+                                m_ref = mt;
+                                rescale = true;
+                            }
+                        }
                     }
-                }
-                const float mref = m_ref == -INFINITY ? 0.f : m_ref;
-                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-                const float2 nm2 = make_float2(-mref, -mref);
-                if (mode == 1) {
-                    const float2 sc2 = make_float2(scale, scale);
+                    const float mref = m_ref == -INFINITY ? 0.f : m_ref;
+                    float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    const float2 nm2 = make_float2(-mref, -mref);
+                    if (mode == 1) {
+                        const float2 sc2 = make_float2(scale, scale);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
-                        const float p0 = ex2(x.x), p1 = ex2(x.y);
-                        acc[c & 1] = fadd2(acc[c & 1], make_float2(p0, p1));
-                        pk[c] = PV8 ? (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3)
-                                    : pack_bf16x2(p0, p1);
-                    }
-                } else {
+                        for (int c = 0; c < 32; ++c) {
+                            const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+                            const float p0 = ex2(x.x), p1 = ex2(x.y);
+                            acc[c & 1] = fadd2(acc[c & 1], make_float2(p0, p1));
+                            pk[c] = PV8 ? (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3)
+                                        : pack_bf16x2(p0, p1);
+                        }
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const float2 x = fadd2(make_float2(s[2 * c], s[2 * c + 1]), nm2);
-                        const float p0 = ex2(x.x), p1 = ex2(x.y);
-                        acc[c & 1] = fadd2(acc[c & 1], make_float2(p0, p1));
-                        pk[c] = PV8 ? (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3)
-                                    : pack_bf16x2(p0, p1);
+                        for (int c = 0; c < 32; ++c) {
+                            const float2 x = fadd2(make_float2(s[2 * c], s[2 * c + 1]), nm2);
+                            const float p0 = ex2(x.x), p1 = ex2(x.y);
+                            acc[c & 1] = fadd2(acc[c & 1], make_float2(p0, p1));
+                            pk[c] = PV8 ? (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3)
+                                        : pack_bf16x2(p0, p1);
+                        }
                     }
+                    lt = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
+                    if (exact || lt <= kOptSum) break;   // (a NaN sum takes the exact pass)
+                    exact = true;
                 }
-                l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
+                l += lt;
             }
             if (r == 0) TRACE(10 + 3 * hf, j);
             if (r == 0) TRACE(11 + 3 * hf, j);

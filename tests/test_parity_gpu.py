@@ -235,3 +235,32 @@ def test_certified_route_no_exemptions(runs, name):
     assert status == 0
     mask = csr_to_mask(buf.row_ptr, buf.col_idx, w.rows, w.nKB)
     assert np.array_equal(mask, res.keep.reshape(w.rows, w.nKB))
+
+
+# Row maxima that rise steeply along the keys: key block b is scaled by 1 + 4 b,
+# so a row's largest score grows by about 20 (natural units) from one tile to
+# the next -- more than a tile's sum bound on P allows, which sends those tiles
+# through the online softmax's rescale -- on exact and centroid tiles alike
+# (with sla, no centroids: kept blocks only).
+RISING = {
+    "rising_sol": Workload("rising_sol", B=1, H=2, N=2085, d=128, dtype="bf16", method="sol", q_block=64,
+                           k_block=64, tau=0.8, grid=(3, 5, 139), seed=41),
+    "rising_sla": Workload("rising_sla", B=1, H=2, N=2085, d=128, dtype="bf16", method="sla", q_block=128,
+                           k_block=64, keep_percent=40.0, centroid=0, grid=(3, 5, 139), seed=42),
+}
+
+
+@pytest.mark.parametrize("name", list(RISING))
+def test_rising_row_maxima(name):
+    w = RISING[name]
+    q, k, v = make_qkv(w, "cpu")
+    ramp = 1.0 + 4.0 * (torch.arange(w.N) // 64).double()
+    k = (k.double() * ramp[None, :, None, None]).to(k.dtype)
+    p, buf, out, status = gpu_layer(w, q.cuda(), k.cuda(), v.cuda())
+    assert status == 0
+    raw = [oracle.as_raw(t) for t in (q, k, v)]
+    res = oracle.routing(w, *raw)
+    ref, ref_lse = oracle.layer_rows(w, *raw, res, oracle.all_tokens(w))
+    got = out.float().cpu().permute(0, 2, 1, 3).reshape(-1, w.d).numpy()
+    compare_outputs(got, ref, f"{name} out")
+    assert np.abs(buf.lse.cpu().numpy().reshape(-1) - ref_lse).max() < 2e-2
