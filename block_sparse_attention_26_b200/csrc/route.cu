@@ -466,28 +466,30 @@ __device__ __forceinline__ float exact_score(const QT *qd, const float *k, doubl
     return __double2float_rn(__ddiv_rn(acc, rs));
 }
 
-// Two of them at once (independent chains, one instruction stream).
+// Two of them at once (independent chains, one instruction stream), each with
+// its own query row.
 template <int D>
-__device__ __forceinline__ void exact_score2(const float *q, const float *k0, const float *k1, double rs, float *s0,
-                                             float *s1)
+__device__ __forceinline__ void exact_score2(const float *q0, const float *q1, const float *k0, const float *k1,
+                                             double rs, float *s0, float *s1)
 {
     const float4 *a4 = reinterpret_cast<const float4 *>(k0);
     const float4 *b4 = reinterpret_cast<const float4 *>(k1);
-    const float4 *q4 = reinterpret_cast<const float4 *>(q);
+    const float4 *p4 = reinterpret_cast<const float4 *>(q0);
+    const float4 *q4 = reinterpret_cast<const float4 *>(q1);
     double x = 0.0, y = 0.0;
     float4 ka = __ldg(a4), kb = __ldg(b4);
 #pragma unroll 4
     for (int c4 = 0; c4 < D / 4; ++c4) {
         const float4 na = c4 + 1 < D / 4 ? __ldg(a4 + c4 + 1) : ka;
         const float4 nb = c4 + 1 < D / 4 ? __ldg(b4 + c4 + 1) : kb;
-        const float4 qv = q4[c4];
-        x = __fma_rn((double)qv.x, (double)ka.x, x);
+        const float4 pv = p4[c4], qv = q4[c4];
+        x = __fma_rn((double)pv.x, (double)ka.x, x);
         y = __fma_rn((double)qv.x, (double)kb.x, y);
-        x = __fma_rn((double)qv.y, (double)ka.y, x);
+        x = __fma_rn((double)pv.y, (double)ka.y, x);
         y = __fma_rn((double)qv.y, (double)kb.y, y);
-        x = __fma_rn((double)qv.z, (double)ka.z, x);
+        x = __fma_rn((double)pv.z, (double)ka.z, x);
         y = __fma_rn((double)qv.z, (double)kb.z, y);
-        x = __fma_rn((double)qv.w, (double)ka.w, x);
+        x = __fma_rn((double)pv.w, (double)ka.w, x);
         y = __fma_rn((double)qv.w, (double)kb.w, y);
         ka = na;
         kb = nb;
@@ -707,14 +709,19 @@ __global__ void __launch_bounds__(320, 1) decide_kernel(const __grid_constant__ 
             }
         }
         named_bar_sync(1, 256);
-        // The undecided blocks' scores exactly as the definition computes them
-        // (the two threads of a row take alternate entries), decided against
-        // [thr_lo, thr_hi]; a row with an inconclusive block, more undecided
-        // blocks than the list holds, or mode 1 goes to the exact path.  The
-        // rows' f32 queries are staged in the K ring, idle once every tile has
-        // been read (the MMA warp's last S is in registers by now).
-        float *qs = reinterpret_cast<float *>(sm + L::kOffK);   // [kTM][D + 4]
+        // The undecided blocks' scores exactly as the definition computes them,
+        // decided against [thr_lo, thr_hi]; a row with an inconclusive block, more
+        // undecided blocks than the list holds, or mode 1 goes to the exact path.
+        // The CTA's listed (row, block) pairs are spread evenly over its 256
+        // threads (flat index f: row by binary search in the rows' list offsets),
+        // so that no thread walks a long row alone.  The rows' f32 queries, list
+        // offsets and threshold intervals are staged in the K ring, idle once every
+        // tile has been read (the MMA warp's last S is in registers by now).
         constexpr int QP = D + 4;
+        float *qs = reinterpret_cast<float *>(sm + L::kOffK);                   // [kTM][QP]
+        int32_t *pre_s = reinterpret_cast<int32_t *>(qs + kTM * QP);           // [kTM + 1] list offsets
+        float2 *thr_s = reinterpret_cast<float2 *>(pre_s + kTM + 4);           // [kTM] (thr_lo, thr_hi)
+        static_assert(kTM * QP * 4 + (kTM + 4) * 4 + kTM * 8 <= L::kStages * L::kKBytes, "decide: K ring too small");
         for (int idx = threadIdx.x; idx < kTM * D / 4; idx += 256) {
             const int rr = idx / (D / 4), c4 = idx % (D / 4);
             const float4 v = i0 + rr < a.nQB
@@ -722,36 +729,72 @@ __global__ void __launch_bounds__(320, 1) decide_kernel(const __grid_constant__ 
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
             *reinterpret_cast<float4 *>(qs + rr * QP + 4 * c4) = v;
         }
-        named_bar_sync(1, 256);
-        if (live) {
+        if (g == 0) {
+            // this row's listed blocks that take the exact score here (none for a
+            // row sent to the exact path or past the end)
             const int u = ucnt_s[r];
-            if (info.mode != 0 || u > kUcap) {
-                if (g == 0) push_fallback(a, row);
+            const bool listed = live && info.mode == 0 && u <= kUcap;
+            if (live && !listed) push_fallback(a, row);
+            ucnt_s[r] = listed ? u : 0;
+            thr_s[r] = make_float2(info.thr_lo, info.thr_hi);
+        }
+        named_bar_sync(1, 256);
+        if (warp == 0) {
+            // exclusive scan of the 128 counts, 4 a lane
+            const int c0 = ucnt_s[4 * lane], c1 = ucnt_s[4 * lane + 1], c2 = ucnt_s[4 * lane + 2],
+                      c3 = ucnt_s[4 * lane + 3];
+            const int sum = c0 + c1 + c2 + c3;
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int excl = incl - sum;
+            pre_s[4 * lane] = excl;
+            pre_s[4 * lane + 1] = excl + c0;
+            pre_s[4 * lane + 2] = excl + c0 + c1;
+            pre_s[4 * lane + 3] = excl + c0 + c1 + c2;
+            if (lane == 31) pre_s[kTM] = incl;
+        }
+        named_bar_sync(1, 256);
+        const int total = pre_s[kTM];
+        const float *kb = a.kbar + (int64_t)bh * a.nKB * D;
+        const double rs = sqrt((double)D);
+        // row and block of flat index f (the last row whose list starts at or before f)
+        auto locate = [&](int f, int &rr, int &jj) {
+            int lo = 0, hi = kTM - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (pre_s[mid] <= f)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            rr = lo;
+            jj = ul_s[lo * kUcap + (f - pre_s[lo])];
+        };
+        auto decide1 = [&](int rr, int jj, float sv) {
+            const float2 th = thr_s[rr];
+            const int64_t rw = (int64_t)bh * a.nQB + i0 + rr;
+            if (sv > th.y)
+                atomicOr(&a.bitmask[rw * a.nW + (jj >> 5)], 1u << (jj & 31));
+            else if (!(sv <= th.x) && atomicExch(&amb_s[rr], 1) == 0)
+                push_fallback(a, rw);
+        };
+        for (int f = threadIdx.x; f < total; f += 512) {
+            int r0, j0;
+            locate(f, r0, j0);
+            if (f + 256 < total) {
+                // two independent chains side by side
+                int r1, j1;
+                locate(f + 256, r1, j1);
+                float s0, s1;
+                exact_score2<D>(qs + r0 * QP, qs + r1 * QP, kb + (int64_t)j0 * D, kb + (int64_t)j1 * D, rs, &s0, &s1);
+                decide1(r0, j0, s0);
+                decide1(r1, j1, s1);
             } else {
-                const float *qrow = qs + r * QP;
-                const float *kb = a.kbar + (int64_t)bh * a.nKB * D;
-                const double rs = sqrt((double)D);
-                bool amb = false;
-                auto decide1 = [&](int j, float sv) {
-                    if (sv > info.thr_hi)
-                        atomicOr(&bm[j >> 5], 1u << (j & 31));
-                    else if (!(sv <= info.thr_lo))
-                        amb = true;
-                };
-                int idx = g;
-                for (; idx + 2 < u; idx += 4) {
-                    // two independent chains side by side
-                    const int j0 = ul[idx], j1 = ul[idx + 2];
-                    float s0, s1;
-                    exact_score2<D>(qrow, kb + (int64_t)j0 * D, kb + (int64_t)j1 * D, rs, &s0, &s1);
-                    decide1(j0, s0);
-                    decide1(j1, s1);
-                }
-                for (; idx < u; idx += 2) {
-                    const int j = ul[idx];
-                    decide1(j, exact_score<D>(qrow, kb + (int64_t)j * D, rs));
-                }
-                if (amb && atomicExch(&amb_s[r], 1) == 0) push_fallback(a, row);
+                decide1(r0, j0, exact_score<D>(qs + r0 * QP, kb + (int64_t)j0 * D, rs));
             }
         }
     }
